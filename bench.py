@@ -1,0 +1,366 @@
+"""Benchmark of the sink-aware GQA attention forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                    [--impl {flint,reference}]
+
+One step is one attention-layer forward (flint_attn_fwd: key preparation +
+attention kernel) over one batch of seeded synthetic input already resident
+in HBM.  The default workload is the full-attention layer at S=4096 (32 query
+heads, 4 KV heads, head dim 128, no RoPE, FP32 sinks), the configuration the
+headline metric (attention TFLOP/s, ms per layer) is quoted on.  Inputs are
+smaller than L2, so L2 is flushed (a 256 MiB write) before every timed step.
+
+With --gpus N > 1 (launched by torch.distributed.run) every rank runs its own
+replica on its own GPU (weak scaling, no data-path collective); NCCL is only
+used for the barriers and the max-over-ranks of the timings.
+
+--impl reference times the FP64 CPU oracle on the host cores on a bounded
+sample of the same workload (rank 0 only).
+
+Prints one JSON line on rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads as W  # noqa: E402
+
+METRIC = "sink-attn fwd TFLOP/s (BF16) and % of B200 tensor peak; ms/layer at S=4096"
+UNIT = "TFLOP/s"
+DEFAULT_WORKLOAD = "full_s4096"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def row_flops(w, rows):
+    """Window-aware FLOPs of the given query rows: 4*128*32 per visible key,
+    a valid query i of a segment starting at s seeing min(i-s+1, window) keys."""
+    import oracle
+    doc = oracle.doc_ids(w.T, w.cu_seqlens, w.pad_mask)
+    start = np.zeros(w.T, np.int64)
+    for t in range(1, w.T):
+        start[t] = start[t - 1] if doc[t] == doc[t - 1] else t
+    rows = np.asarray(rows)
+    n = rows - start[rows] + 1
+    if w.window > 0:
+        n = np.minimum(n, w.window)
+    n = np.where(doc[rows] >= 0, n, 0)
+    return 4.0 * 128 * 32 * float(n.sum())
+
+
+# ---------------------------------------------------------------- clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        os.unlink(self.path)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- flint arm
+
+def run_flint(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    import full_gqa_learned_b200 as fa
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    w = W.make(args.workload)
+    T = w.T
+
+    def bf(x):
+        return torch.from_numpy(np.ascontiguousarray(x)).view(torch.bfloat16)
+    host = dict(q=bf(w.q), k=bf(w.k), v=bf(w.v), q_norm_w=torch.from_numpy(w.q_norm_w),
+                k_norm_w=torch.from_numpy(w.k_norm_w),
+                sinks=torch.from_numpy(np.ascontiguousarray(w.sinks, np.float32)))
+    if w.pos_ids is not None:
+        host["pos_ids"] = torch.from_numpy(w.pos_ids)
+    if w.cu_seqlens is not None:
+        host["cu_seqlens"] = torch.from_numpy(w.cu_seqlens)
+    if w.pad_mask is not None:
+        host["pad_mask"] = torch.from_numpy(w.pad_mask)
+    d = {k: v.to(dev) for k, v in host.items()}
+    nseg = (len(w.cu_seqlens) - 1) if w.cu_seqlens is not None else (
+        w.pad_mask.shape[0] if w.pad_mask is not None else 1)
+    out = torch.empty((T, 4096), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((32, T), dtype=torch.float32, device=dev)
+    ws = torch.empty(fa.workspace_bytes(T, nseg), dtype=torch.uint8, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    kw = dict(pos_ids=d.get("pos_ids"), cu_seqlens=d.get("cu_seqlens"),
+              pad_mask=d.get("pad_mask"), window=w.window, use_rope=w.use_rope,
+              rope_theta=w.rope_theta, eps=w.eps, out=out, lse=lse, workspace=ws,
+              stream=stream)
+
+    def step(ev=None):
+        if ev is None:
+            fa.attn_fwd(d["q"], d["k"], d["v"], d["q_norm_w"], d["k_norm_w"], d["sinks"], **kw)
+            return
+        ev[0].record(stream)
+        fa.attn_fwd(d["q"], d["k"], d["v"], d["q_norm_w"], d["k_norm_w"], d["sinks"],
+                    stage="prepare", **kw)
+        ev[1].record(stream)
+        fa.attn_fwd(d["q"], d["k"], d["v"], d["q_norm_w"], d["k_norm_w"], d["sinks"],
+                    stage="attend", **kw)
+        ev[2].record(stream)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    # warm-up, then a ~1 s soak so the clock sampler sees the part under load
+    for _ in range(args.warmup):
+        flush.fill_(1)
+        step()
+    st = fa.device_status(ws)
+    if st != 0:
+        raise RuntimeError("device status %s" % fa.STATUS.get(st, st))
+    sampler = ClockSampler(local_rank if "CUDA_VISIBLE_DEVICES" not in os.environ else
+                           os.environ["CUDA_VISIBLE_DEVICES"].split(",")[local_rank])
+    sampler.start()
+    time.sleep(0.3)
+    t_end = time.time() + args.soak
+    while time.time() < t_end:
+        for _ in range(20):
+            step()
+        torch.cuda.synchronize(dev)
+
+    # timed region: exactly K steps, L2 flushed before each
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    barrier()
+    torch.cuda.synchronize(dev)
+    for i in range(args.steps):
+        flush.fill_(i & 0xFF)
+        step(evs[i])
+    torch.cuda.synchronize(dev)
+    barrier()
+    clocks = sampler.stop()
+    st = fa.device_status(ws)
+    if st != 0:
+        raise RuntimeError("device status %s" % fa.STATUS.get(st, st))
+    prep_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    attn_ms = [e[1].elapsed_time(e[2]) for e in evs]
+    step_ms = [e[0].elapsed_time(e[2]) for e in evs]
+    total_ms = sum(step_ms)
+    attn_avg = sum(attn_ms) / len(attn_ms)
+
+    # end-to-end through the public API from pinned host buffers
+    pinned = {k: v.pin_memory() for k, v in host.items()}
+    out_h = torch.empty((T, 4096), dtype=torch.bfloat16).pin_memory()
+    lse_h = torch.empty((32, T), dtype=torch.float32).pin_memory()
+    h2d = sum(v.numel() * v.element_size() for v in pinned.values())
+    d2h = out_h.numel() * 2 + lse_h.numel() * 4
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e2e_steps = max(3, min(args.steps, 20))
+    for _ in range(2):
+        dd = {k: v.to(dev, non_blocking=True) for k, v in pinned.items()}
+        o, l = fa.attn_fwd(dd["q"], dd["k"], dd["v"], dd["q_norm_w"], dd["k_norm_w"],
+                           dd["sinks"], pos_ids=dd.get("pos_ids"), cu_seqlens=dd.get("cu_seqlens"),
+                           pad_mask=dd.get("pad_mask"), window=w.window, use_rope=w.use_rope,
+                           rope_theta=w.rope_theta, eps=w.eps, workspace=ws)
+        out_h.copy_(o, non_blocking=True)
+        lse_h.copy_(l, non_blocking=True)
+    torch.cuda.synchronize(dev)
+    barrier()
+    e2e_ms = 0.0
+    for _ in range(e2e_steps):
+        flush.fill_(3)
+        e0.record(stream)
+        dd = {k: v.to(dev, non_blocking=True) for k, v in pinned.items()}
+        o, l = fa.attn_fwd(dd["q"], dd["k"], dd["v"], dd["q_norm_w"], dd["k_norm_w"],
+                           dd["sinks"], pos_ids=dd.get("pos_ids"), cu_seqlens=dd.get("cu_seqlens"),
+                           pad_mask=dd.get("pad_mask"), window=w.window, use_rope=w.use_rope,
+                           rope_theta=w.rope_theta, eps=w.eps, workspace=ws)
+        out_h.copy_(o, non_blocking=True)
+        lse_h.copy_(l, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        e2e_ms += e0.elapsed_time(e1)
+    e2e_ms /= e2e_steps
+
+    # max over ranks
+    vals = torch.tensor([total_ms, attn_avg, e2e_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
+    total_ms, attn_avg, e2e_ms = [float(x) for x in vals.cpu()]
+    return dict(w=w, total_ms=total_ms, attn_avg=attn_avg, prep_avg=sum(prep_ms) / len(prep_ms),
+                e2e_ms=e2e_ms, h2d=h2d, d2h=d2h, clocks=clocks, launches=2 * args.steps)
+
+
+def cpu_baseline(w, budget_s, nthreads=0):
+    """The oracle, as it stands, on a bounded sample of query rows."""
+    import oracle
+    rng = np.random.default_rng(12345)
+    n = 32
+    rows = np.sort(rng.choice(w.T, n, replace=False))
+    t0 = time.time()
+    oracle.attn_fwd_workload(w, rows=rows, nthreads=nthreads)
+    dt = time.time() - t0
+    # grow the sample to roughly the time budget
+    if dt < budget_s / 4:
+        n = int(min(w.T, n * max(1.0, budget_s / max(dt, 1e-3) * 0.8)))
+        rows = np.sort(rng.choice(w.T, n, replace=False))
+        t0 = time.time()
+        oracle.attn_fwd_workload(w, rows=rows, nthreads=nthreads)
+        dt = time.time() - t0
+    fl = row_flops(w, rows)
+    cores = nthreads if nthreads > 0 else os.cpu_count()
+    return dict(value=fl / dt / 1e12, unit=UNIT, cores=cores, kind="oracle",
+                sample="%d of %d query rows x 32 heads of %s (seeded), %.1f s" %
+                (len(rows), w.T, w.name, dt))
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(W.CONFIGS))
+    ap.add_argument("--impl", default="flint", choices=["flint", "reference"])
+    ap.add_argument("--soak", type=float, default=1.0, help="seconds of untimed load before timing")
+    ap.add_argument("--cpu-budget", type=float, default=12.0)
+    ap.add_argument("--traffic", type=float, default=None,
+                    help="ncu DRAM bytes per attention launch, if captured for this kernel")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        w = W.make(args.workload)
+        times, cb = [], None
+        for i in range(args.warmup + args.steps):
+            r = cpu_baseline(w, budget_s=min(args.cpu_budget, 120.0 / max(1, args.steps + args.warmup)))
+            if i >= args.warmup:
+                times.append(r["value"])
+            cb = r
+        value = statistics.median(times)
+        cb["value"] = value
+        line = dict(impl="reference", metric=METRIC, value=value, unit=UNIT, n_gpus=args.gpus,
+                    steps=args.steps, warmup=args.warmup, ms_per_step=None,
+                    higher_is_better=True, scaling="weak", vs_baseline=None, dtype="f64",
+                    data="synthetic", config=dict(workload=w.name, T=w.T, window=w.window,
+                                                  use_rope=w.use_rope),
+                    cpu_baseline=cb,
+                    e2e=dict(value=value, unit=UNIT, h2d_bytes_per_step=0, d2h_bytes_per_step=0))
+        print(json.dumps(line))
+        return 0
+
+    import torch
+    import torch.distributed as dist
+    if world > 1:
+        torch.cuda.set_device(local_rank)
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        r = run_flint(args, rank, world, local_rank)
+    finally:
+        pass
+    w = r["w"]
+    peaks, src = load_peaks()
+    flops = w.flops()
+    value = world * flops * args.steps / (r["total_ms"] * 1e-3) / 1e12
+    attn_tflops = flops / (r["attn_avg"] * 1e-3) / 1e12
+    peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    line = dict(
+        metric=METRIC, value=round(value, 3), unit=UNIT, n_gpus=world, steps=args.steps,
+        warmup=args.warmup, ms_per_step=round(r["total_ms"] / args.steps, 5),
+        higher_is_better=True, scaling="weak", vs_baseline=None, dtype="bf16",
+        data="synthetic (seeded N(0,1) BF16 q/k/v, 1+N(0,0.1) norm weights, N(0,1) sinks)",
+        config=dict(workload=w.name, T=w.T, window=w.window, use_rope=bool(w.use_rope),
+                    q_heads=32, kv_heads=4, head_dim=128, qk_operands="fp16 (post-norm)",
+                    pv_operands="bf16", l2="flushed before every timed step (256 MiB write)",
+                    per_rank="independent replica"),
+        roofline=dict(bound="tensor", achieved=round(attn_tflops, 3), peak=peak, unit=UNIT,
+                      frac=round(attn_tflops / peak, 4), traffic=args.traffic,
+                      kernel="flint::attn_fwd_kernel", peak_source="%s bf16_tflops (burst)" % src,
+                      flops_per_launch=flops,
+                      kernel_ms=round(r["attn_avg"], 5), prep_kernel_ms=round(r["prep_avg"], 5)),
+        e2e=dict(value=round(world * flops / (r["e2e_ms"] * 1e-3) / 1e12, 3), unit=UNIT,
+                 h2d_bytes_per_step=r["h2d"], d2h_bytes_per_step=r["d2h"],
+                 ms_per_step=round(r["e2e_ms"], 4)),
+        gpu_launches=r["launches"], clocks=r["clocks"],
+        pct_of_tensor_peak=round(100.0 * value / world / peak, 2),
+    )
+    if rank == 0 and world == 1:
+        line["cpu_baseline"] = cpu_baseline(w, budget_s=args.cpu_budget)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line))
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

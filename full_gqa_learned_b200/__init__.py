@@ -1,0 +1,164 @@
+"""B200 (sm_100a) sink-aware GQA attention forward of the Flint decoder.
+
+This package is a thin ctypes binding over ``libflint_attn.so``, whose C ABI
+is declared in ``include/flint_attn.h``.  The binding only marshals
+arguments: every step of the computation (key preparation, planning,
+normalisation, rotation, attention, sink, masking, epilogue) runs in the
+library's CUDA kernels.  PyTorch is used for device memory and streams.
+
+There is no fallback: if the library is missing or the device is not an
+sm_100 GPU, the call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+from typing import Optional, Tuple
+
+__all__ = ["attn_fwd", "workspace_bytes", "device_status", "load_library", "FlintError",
+           "LIB_PATH", "HQ", "HKV", "HEAD_DIM", "STATUS"]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libflint_attn.so")
+HQ, HKV, HEAD_DIM = 32, 4, 128
+STATUS = {0: "FLINT_OK", 1: "FLINT_ERR_INVALID_ARG", 2: "FLINT_ERR_UNSUPPORTED",
+          3: "FLINT_ERR_CUDA", 4: "FLINT_ERR_TIMEOUT", 5: "FLINT_ERR_WORKSPACE"}
+
+_lock = threading.Lock()
+_lib = None
+
+
+class FlintError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__("%s: %s" % (STATUS.get(status, status), message))
+        self.status = status
+
+
+def load_library() -> ctypes.CDLL:
+    """Load libflint_attn.so (built in-tree by ``full_gqa_learned_b200.build``)."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        if not os.path.exists(LIB_PATH):
+            raise ImportError("libflint_attn.so is not built; run "
+                              "`python -m full_gqa_learned_b200.build`")
+        lib = ctypes.CDLL(LIB_PATH)
+        P, I32, F32 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_float
+        lib.flint_attn_abi_version.restype = I32
+        lib.flint_attn_abi_version.argtypes = []
+        lib.flint_attn_workspace_bytes.restype = ctypes.c_size_t
+        lib.flint_attn_workspace_bytes.argtypes = [I32, I32]
+        fwd_args = [P, P, P, P, P, P, P, P, I32, P, I32, I32, I32, I32, I32,
+                    F32, F32, P, P, P, ctypes.c_size_t, P]
+        for name in ("flint_attn_fwd", "flint_attn_prepare", "flint_attn_attend"):
+            getattr(lib, name).restype = ctypes.c_int
+            getattr(lib, name).argtypes = fwd_args
+        lib.flint_attn_device_status.restype = ctypes.c_int
+        lib.flint_attn_device_status.argtypes = [P, P]
+        lib.flint_attn_last_error.restype = ctypes.c_char_p
+        lib.flint_attn_last_error.argtypes = []
+        lib.flint_attn_status_string.restype = ctypes.c_char_p
+        lib.flint_attn_status_string.argtypes = [ctypes.c_int]
+        _lib = lib
+        return lib
+
+
+def workspace_bytes(T: int, num_segments: int = 1) -> int:
+    return int(load_library().flint_attn_workspace_bytes(int(T), int(num_segments)))
+
+
+def _ptr(t) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _check(t, name, dtype, shape=None):
+    import torch
+    if not isinstance(t, torch.Tensor):
+        raise TypeError("%s must be a torch.Tensor" % name)
+    if not t.is_cuda:
+        raise ValueError("%s must be a CUDA tensor" % name)
+    if t.dtype != dtype:
+        raise TypeError("%s must be %s, got %s" % (name, dtype, t.dtype))
+    if not t.is_contiguous():
+        raise ValueError("%s must be contiguous" % name)
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError("%s must have shape %s, got %s" % (name, tuple(shape), tuple(t.shape)))
+
+
+def attn_fwd(q, k, v, q_norm_w, k_norm_w, sinks, *, pos_ids=None, cu_seqlens=None,
+             pad_mask=None, window: int = 513, use_rope: bool = True,
+             rope_theta: float = 10000.0, eps: float = 1e-6, out=None, lse=None,
+             workspace=None, stream=None, want_lse: bool = True,
+             stage: str = "both") -> Tuple[object, object]:
+    """Sink-aware GQA attention forward (see include/flint_attn.h).
+
+    q [T,32,128], k/v [T,4,128] bf16 CUDA tensors; q_norm_w, k_norm_w [128]
+    and sinks [32] float32; pos_ids [T] int32 or None; cu_seqlens [n+1] int32
+    (packed THD) or pad_mask [B,S] uint8 (trailing padding) or neither.
+    window 0 = full causal.  Returns (out [T,4096] bf16, lse [32,T] f32 or
+    None).  Asynchronous on ``stream`` (default: torch's current stream).
+    ``stage``: "both" (flint_attn_fwd), or "prepare" / "attend" to enqueue
+    the two kernels separately (same arguments and workspace for both).
+    """
+    import torch
+    lib = load_library()
+    T = int(q.shape[0]) if q.dim() >= 1 else 0
+    _check(q, "q", torch.bfloat16, (T, HQ, HEAD_DIM))
+    _check(k, "k", torch.bfloat16, (T, HKV, HEAD_DIM))
+    _check(v, "v", torch.bfloat16, (T, HKV, HEAD_DIM))
+    _check(q_norm_w, "q_norm_w", torch.float32, (HEAD_DIM,))
+    _check(k_norm_w, "k_norm_w", torch.float32, (HEAD_DIM,))
+    _check(sinks, "sinks", torch.float32, (HQ,))
+    num_docs, batch, seqlen, nseg = 0, 0, 0, 1
+    if pos_ids is not None:
+        _check(pos_ids, "pos_ids", torch.int32, (T,))
+    if cu_seqlens is not None:
+        _check(cu_seqlens, "cu_seqlens", torch.int32)
+        num_docs = int(cu_seqlens.numel()) - 1
+        nseg = max(num_docs, 1)
+    if pad_mask is not None:
+        _check(pad_mask, "pad_mask", torch.uint8)
+        if pad_mask.dim() != 2:
+            raise ValueError("pad_mask must be [batch, seqlen]")
+        batch, seqlen = int(pad_mask.shape[0]), int(pad_mask.shape[1])
+        nseg = batch
+    dev = q.device
+    if out is None:
+        out = torch.empty((T, HQ * HEAD_DIM), dtype=torch.bfloat16, device=dev)
+    _check(out, "out", torch.bfloat16, (T, HQ * HEAD_DIM))
+    if lse is None and want_lse:
+        lse = torch.empty((HQ, T), dtype=torch.float32, device=dev)
+    if lse is not None:
+        _check(lse, "lse", torch.float32, (HQ, T))
+    need = workspace_bytes(T, nseg)
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
+    _check(workspace, "workspace", torch.uint8)
+    if stream is None:
+        stream = torch.cuda.current_stream(dev)
+    sptr = stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+    with torch.cuda.device(dev):
+        fn = {"both": lib.flint_attn_fwd, "prepare": lib.flint_attn_prepare,
+              "attend": lib.flint_attn_attend}[stage]
+        st = fn(
+            _ptr(q), _ptr(k), _ptr(v), _ptr(q_norm_w), _ptr(k_norm_w), _ptr(sinks),
+            _ptr(pos_ids), _ptr(cu_seqlens), num_docs, _ptr(pad_mask), batch, seqlen, T,
+            int(window), int(bool(use_rope)), float(rope_theta), float(eps), _ptr(out),
+            _ptr(lse), _ptr(workspace), int(workspace.numel()), sptr)
+    if st != 0:
+        raise FlintError(st, lib.flint_attn_last_error().decode())
+    attn_fwd.last_workspace = workspace
+    return out, lse
+
+
+def device_status(workspace, stream=None) -> int:
+    """Synchronise and return the device-side status of the last call that
+    used ``workspace`` (0 = FLINT_OK)."""
+    import torch
+    lib = load_library()
+    if stream is None:
+        stream = torch.cuda.current_stream(workspace.device)
+    sptr = stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+    return int(lib.flint_attn_device_status(_ptr(workspace), sptr))

@@ -1,0 +1,282 @@
+// Host side of the C ABI declared in include/flint_attn.h: argument
+// validation, workspace layout, TMA tensor maps and the two launches
+// (preparation kernel, attention kernel).  No allocation, no host<->device
+// copies, no synchronisation on the call path.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/flint_attn.h"
+#include "flint_common.cuh"
+
+namespace flint {
+__global__ void prep_kernel(PrepParams p);
+__global__ void attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q,
+                                const __grid_constant__ CUtensorMap tm_k,
+                                const __grid_constant__ CUtensorMap tm_v, const AttnParams p);
+extern const unsigned kAttnSmemBytes;
+}  // namespace flint
+
+using namespace flint;
+
+namespace {
+
+thread_local char g_err[512] = "";
+
+flint_status_t fail(flint_status_t s, const char* fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_err, sizeof(g_err), fmt, ap);
+    va_end(ap);
+    return s;
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+std::mutex g_mu;
+EncodeTiledFn g_encode = nullptr;
+constexpr int kMaxDevices = 64;
+int g_sms[kMaxDevices] = {0};
+bool g_attr_set[kMaxDevices] = {false};
+
+flint_status_t get_encoder(EncodeTiledFn* fn) {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!g_encode) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q);
+        if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !p)
+            return fail(FLINT_ERR_CUDA, "cuTensorMapEncodeTiled unavailable: %s",
+                        cudaGetErrorString(e));
+        g_encode = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    *fn = g_encode;
+    return FLINT_OK;
+}
+
+flint_status_t device_setup(int* sms) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return fail(FLINT_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+    if (dev < 0 || dev >= kMaxDevices) return fail(FLINT_ERR_UNSUPPORTED, "device index %d", dev);
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!g_attr_set[dev]) {
+        int major = 0, minor = 0;
+        cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+        if (major != 10 || minor != 0)
+            return fail(FLINT_ERR_UNSUPPORTED, "needs an sm_100 GPU, found sm_%d%d", major, minor);
+        e = cudaFuncSetAttribute(attn_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)kAttnSmemBytes);
+        if (e != cudaSuccess)
+            return fail(FLINT_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+        cudaDeviceGetAttribute(&g_sms[dev], cudaDevAttrMultiProcessorCount, dev);
+        g_attr_set[dev] = true;
+    }
+    *sms = g_sms[dev];
+    return FLINT_OK;
+}
+
+// 3-D map over a [T, heads, 128] tensor of 16-bit elements: dims (128, heads,
+// T), box (64, box_heads, box_tokens), 128-byte swizzle, zero fill outside.
+flint_status_t make_map(EncodeTiledFn enc, CUtensorMap* m, CUtensorMapDataType dt, const void* base,
+                        int heads, int T, int box_heads, int box_tokens) {
+    cuuint64_t dims[3] = {(cuuint64_t)kHD, (cuuint64_t)heads, (cuuint64_t)T};
+    cuuint64_t strides[2] = {(cuuint64_t)kHD * 2, (cuuint64_t)heads * kHD * 2};
+    cuuint32_t box[3] = {64, (cuuint32_t)box_heads, (cuuint32_t)box_tokens};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = enc(m, dt, 3, const_cast<void*>(base), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(FLINT_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+    return FLINT_OK;
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+}  // namespace
+
+extern "C" {
+
+int32_t flint_attn_abi_version(void) { return 1; }
+
+size_t flint_attn_workspace_bytes(int32_t T, int32_t num_segments) {
+    if (T < 0 || T > FLINT_MAX_TOKENS || num_segments < 0 || num_segments > FLINT_MAX_TOKENS)
+        return 0;
+    int nseg = num_segments < 1 ? 1 : num_segments;
+    return ws_layout(T, nseg).total;
+}
+
+const char* flint_attn_last_error(void) { return g_err; }
+
+const char* flint_attn_status_string(flint_status_t s) {
+    switch (s) {
+        case FLINT_OK: return "FLINT_OK";
+        case FLINT_ERR_INVALID_ARG: return "FLINT_ERR_INVALID_ARG";
+        case FLINT_ERR_UNSUPPORTED: return "FLINT_ERR_UNSUPPORTED";
+        case FLINT_ERR_CUDA: return "FLINT_ERR_CUDA";
+        case FLINT_ERR_TIMEOUT: return "FLINT_ERR_TIMEOUT";
+        case FLINT_ERR_WORKSPACE: return "FLINT_ERR_WORKSPACE";
+    }
+    return "FLINT_ERR_UNKNOWN";
+}
+
+}  // extern "C"
+
+namespace {
+
+enum Stage : int { kStagePrepare = 1, kStageAttend = 2, kStageBoth = 3 };
+
+flint_status_t run(int stages, const void* q, const void* k, const void* v, const float* q_norm_w,
+                   const float* k_norm_w, const float* sinks, const int32_t* pos_ids,
+                   const int32_t* cu_seqlens, int32_t num_docs, const uint8_t* pad_mask,
+                   int32_t batch, int32_t seqlen, int32_t T, int32_t window, int32_t use_rope,
+                   float rope_theta, float eps, void* out, float* lse, void* workspace,
+                   size_t workspace_bytes, void* stream) {
+    g_err[0] = '\0';
+    // ---- host-side validation: nothing below touches the GPU until it passes
+    if (T < 0 || T > FLINT_MAX_TOKENS)
+        return fail(FLINT_ERR_INVALID_ARG, "T=%d outside [0, %d]", T, FLINT_MAX_TOKENS);
+    if (window < 0) return fail(FLINT_ERR_INVALID_ARG, "window=%d < 0", window);
+    if (use_rope != 0 && use_rope != 1) return fail(FLINT_ERR_INVALID_ARG, "use_rope must be 0 or 1");
+    if (!(eps > 0.f) || !std::isfinite(eps)) return fail(FLINT_ERR_INVALID_ARG, "eps must be > 0");
+    if (use_rope && (!(rope_theta > 1.f) || !std::isfinite(rope_theta)))
+        return fail(FLINT_ERR_INVALID_ARG, "rope_theta must be > 1");
+    if (cu_seqlens && pad_mask)
+        return fail(FLINT_ERR_INVALID_ARG, "give at most one of cu_seqlens and pad_mask");
+    int mode = kMaskSingle, nseg = 1;
+    if (cu_seqlens) {
+        if (num_docs < 0 || num_docs > FLINT_MAX_TOKENS)
+            return fail(FLINT_ERR_INVALID_ARG, "num_docs=%d", num_docs);
+        mode = kMaskThd;
+        nseg = num_docs;
+    } else if (pad_mask) {
+        if (batch < 1 || seqlen < 1 || (long long)batch * seqlen != (long long)T)
+            return fail(FLINT_ERR_INVALID_ARG, "pad_mask needs batch*seqlen == T (%d*%d vs %d)",
+                        batch, seqlen, T);
+        mode = kMaskPad;
+        nseg = batch;
+    }
+    if (T == 0) return FLINT_OK;
+    if (!q || !k || !v || !q_norm_w || !k_norm_w || !sinks || !out)
+        return fail(FLINT_ERR_INVALID_ARG, "null tensor pointer");
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16))
+        return fail(FLINT_ERR_INVALID_ARG, "q, k, v and out must be 16-byte aligned");
+    if (!aligned(q_norm_w, 4) || !aligned(k_norm_w, 4) || !aligned(sinks, 4) ||
+        (lse && !aligned(lse, 4)) || (pos_ids && !aligned(pos_ids, 4)) ||
+        (cu_seqlens && !aligned(cu_seqlens, 4)))
+        return fail(FLINT_ERR_INVALID_ARG, "misaligned 32-bit array");
+    const WsLayout L = ws_layout(T, nseg < 1 ? 1 : nseg);
+    if (!workspace || !aligned(workspace, 256))
+        return fail(FLINT_ERR_WORKSPACE, "workspace missing or not 256-byte aligned");
+    if (workspace_bytes < L.total)
+        return fail(FLINT_ERR_WORKSPACE, "workspace too small: %zu < %zu bytes", workspace_bytes,
+                    L.total);
+
+    // ---- launch
+    int sms = 0;
+    flint_status_t st = device_setup(&sms);
+    if (st != FLINT_OK) return st;
+    EncodeTiledFn enc = nullptr;
+    st = get_encoder(&enc);
+    if (st != FLINT_OK) return st;
+    char* ws = static_cast<char*>(workspace);
+    CUtensorMap tm_q, tm_k, tm_v;
+    st = make_map(enc, &tm_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, q, kHQ, T, kGroup, kTokPerTile);
+    if (st != FLINT_OK) return st;
+    st = make_map(enc, &tm_k, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, ws + L.kn, kHKV, T, 1, kKeyChunk);
+    if (st != FLINT_OK) return st;
+    st = make_map(enc, &tm_v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, v, kHKV, T, 1, kKeyChunk);
+    if (st != FLINT_OK) return st;
+
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaSuccess;
+    PrepParams pp;
+    pp.k = static_cast<const __nv_bfloat16*>(k);
+    pp.k_norm_w = k_norm_w;
+    pp.sinks = sinks;
+    pp.pos_ids = pos_ids;
+    pp.cu_seqlens = cu_seqlens;
+    pp.pad_mask = pad_mask;
+    pp.out = static_cast<__nv_bfloat16*>(out);
+    pp.lse = lse;
+    pp.ws = ws;
+    pp.T = T;
+    pp.nseg = nseg < 1 ? (mode == kMaskThd ? 0 : 1) : nseg;
+    pp.batch = batch;
+    pp.seqlen = seqlen;
+    pp.window = window;
+    pp.use_rope = use_rope;
+    pp.mode = mode;
+    pp.rope_theta = rope_theta;
+    pp.eps = eps;
+    // ws_layout is always evaluated with max(nseg, 1) segments
+    int prep_blocks = 1 + (T + 31) / 32;
+    if (prep_blocks > 1 + 4 * sms) prep_blocks = 1 + 4 * sms;
+    if (prep_blocks < 2) prep_blocks = 2;
+    if (stages & kStagePrepare) {
+        prep_kernel<<<prep_blocks, 1024, 0, s>>>(pp);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return fail(FLINT_ERR_CUDA, "prep launch: %s", cudaGetErrorString(e));
+    }
+    if (!(stages & kStageAttend)) return FLINT_OK;
+
+    AttnParams ap;
+    ap.q_norm_w = q_norm_w;
+    ap.k_norm_w = k_norm_w;
+    ap.sinks = sinks;
+    ap.pos_ids = pos_ids;
+    ap.out = static_cast<__nv_bfloat16*>(out);
+    ap.lse = lse;
+    ap.ws = ws;
+    ap.T = T;
+    ap.nseg = pp.nseg;
+    ap.window = window;
+    ap.use_rope = use_rope;
+    ap.rope_theta = rope_theta;
+    ap.eps = eps;
+    const int max_units = L.max_items * kHKV;
+    const int grid = max_units < sms ? max_units : sms;
+    attn_fwd_kernel<<<grid, 384, kAttnSmemBytes, s>>>(tm_q, tm_k, tm_v, ap);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return fail(FLINT_ERR_CUDA, "attention launch: %s", cudaGetErrorString(e));
+    return FLINT_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+#define FLINT_ARGS                                                                            \
+    const void *q, const void *k, const void *v, const float *q_norm_w, const float *k_norm_w, \
+        const float *sinks, const int32_t *pos_ids, const int32_t *cu_seqlens, int32_t num_docs, \
+        const uint8_t *pad_mask, int32_t batch, int32_t seqlen, int32_t T, int32_t window,       \
+        int32_t use_rope, float rope_theta, float eps, void *out, float *lse, void *workspace,   \
+        size_t workspace_bytes, void *stream
+#define FLINT_FWD_ARGS                                                                         \
+    q, k, v, q_norm_w, k_norm_w, sinks, pos_ids, cu_seqlens, num_docs, pad_mask, batch, seqlen, \
+        T, window, use_rope, rope_theta, eps, out, lse, workspace, workspace_bytes, stream
+
+flint_status_t flint_attn_fwd(FLINT_ARGS) { return run(kStageBoth, FLINT_FWD_ARGS); }
+flint_status_t flint_attn_prepare(FLINT_ARGS) { return run(kStagePrepare, FLINT_FWD_ARGS); }
+flint_status_t flint_attn_attend(FLINT_ARGS) { return run(kStageAttend, FLINT_FWD_ARGS); }
+
+flint_status_t flint_attn_device_status(const void* workspace, void* stream) {
+    if (!workspace) return fail(FLINT_ERR_WORKSPACE, "workspace is null");
+    cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return fail(FLINT_ERR_CUDA, "stream sync: %s", cudaGetErrorString(e));
+    int st = 0;
+    e = cudaMemcpy(&st, workspace, sizeof(int), cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return fail(FLINT_ERR_CUDA, "status read: %s", cudaGetErrorString(e));
+    return static_cast<flint_status_t>(st);
+}
+
+}  // extern "C"

@@ -1,0 +1,568 @@
+// Sink-aware causal GQA attention forward for sm_100a (tcgen05 + TMEM + TMA).
+//
+// Computes, for every valid query token i and query head h (KV head g = h/8),
+//   out[i,h,:] = sum_j e^{s_ij} v[j,g,:] / (e^{sink_h} + sum_j e^{s_ij}),
+//   lse[h,i]   = ln(e^{sink_h} + sum_j e^{s_ij}),
+// with s_ij = q~_i . k~_j / sqrt(128) over the keys j of the same document,
+// j <= i, and i - j < window on sliding layers.  q~ is q after the weight-form
+// RMSNorm and, on sliding layers, NeoX RoPE (FlintAttention.forward and
+// _apply_rope on the NeMo AutoModel "flint.layers" API page; the sink as an
+// extra zero-value softmax column in natural-logit units: HF discussion #26 on
+// RecursiveSI/flint).  k~ was prepared by the preparation kernel.
+//
+// Layout of one CTA (one per SM, persistent, 384 threads):
+//   warp 0      dynamic scheduler + TMA producer (Q tiles, K/V chunks)
+//   warp 1      TMEM owner; lane 0 issues every tcgen05.mma and commit
+//   warps 4-7   softmax warpgroup of tile 0 (tokens q0..q0+15)
+//   warps 8-11  softmax warpgroup of tile 1 (tokens q0+16..q0+31)
+// A tile is 128 MMA rows = 16 tokens x the 8 query heads of one KV group, so
+// every K/V chunk in shared memory serves 8 heads x 32 tokens.
+//
+// Tensor memory (512 columns): S_t at column 128 t, O_t at 256 + 128 t.  P_t
+// (BF16) overwrites the first 64 columns of S_t and feeds the PV MMA straight
+// from TMEM.  The online softmax starts from m = sink*log2(e), l = 1, which
+// is exactly the extra sink column; the running max is only raised (and O
+// rescaled) when it grows by more than 2^8, so the rescale is rare.
+#include <cuda.h>
+#include <cmath>
+#include "flint_common.cuh"
+#include "sm100.cuh"
+
+namespace flint {
+
+constexpr int kThreads = 384;
+constexpr uint32_t kTileBytes = 128 * kHD * 2;       // 32 KiB: 128 rows x 128 x 16-bit
+constexpr uint32_t kHalfTile = kTileBytes / 2;       // one 64-column swizzled half
+
+// Shared memory plan (offsets from a 1024-aligned base).
+constexpr uint32_t kOffQ = 0;                        // 2 Q tiles
+constexpr uint32_t kOffK = kOffQ + 2 * kTileBytes;   // 2 K stages
+constexpr uint32_t kOffV = kOffK + 2 * kTileBytes;   // 2 V stages
+constexpr uint32_t kOffRope = kOffV + 2 * kTileBytes;        // 2 x [16][64] float2
+constexpr uint32_t kRopeBytes = kTokPerTile * 64 * 8;
+constexpr uint32_t kOffW = kOffRope + 2 * kRopeBytes;        // q_norm_w [128] f32
+constexpr uint32_t kOffInv = kOffW + kHD * 4;                // inv_freq [64] f64
+constexpr uint32_t kOffBar = kOffInv + 64 * 8;               // mbarriers
+constexpr uint32_t kNumBars = 32;
+constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
+constexpr uint32_t kSmemUsed = kOffMisc + 64;
+constexpr uint32_t kSmemBytes = kSmemUsed + 1024;            // + alignment slack
+
+// barrier indices
+enum : uint32_t {
+    B_SCHED_FULL = 0, B_SCHED_EMPTY = 2,
+    B_Q_FULL = 4, B_Q_READY = 6, B_Q_EMPTY = 8,
+    B_K_FULL = 10, B_K_EMPTY = 12, B_V_FULL = 14, B_V_EMPTY = 16,
+    B_S_FULL = 18, B_P_FULL = 20, B_O_FULL = 22, B_DRAIN = 24
+};
+
+struct Misc {
+    int sched[2];
+    uint32_t tmem_base;
+    int abort_flag;
+    float q_scale;       // 2^eq
+    float logit_scale;   // log2(e)/sqrt(128) * 2^-(eq+ek)
+};
+
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// Two FP32 values -> packed 16-bit pair, `lo` in the low half.
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+    uint32_t r;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+__device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
+    uint32_t r;
+    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+__device__ __forceinline__ float bf16_lo(uint32_t u) { return __uint_as_float(u << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t u) { return __uint_as_float(u & 0xffff0000u); }
+
+// Warpgroup-uniform AND of a per-thread flag over named barrier `id`.
+__device__ __forceinline__ bool wg_all(uint32_t id, bool ok) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "bar.red.and.pred q, %2, 128, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)ok), "r"(id)
+        : "memory");
+    return r != 0;
+}
+
+__device__ __forceinline__ int chunk_cols(int ks, int ke) {
+    int n = ke - ks;
+    n = n > kKeyChunk ? kKeyChunk : n;
+    return (n + 15) & ~15;
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                               ~uintptr_t(1023));
+    const uint32_t sbase = smem_u32(smem);
+    const uint32_t bar0 = sbase + kOffBar;
+    auto bar = [&](uint32_t i) { return bar0 + 8u * i; };
+    Misc* misc = reinterpret_cast<Misc*>(smem + kOffMisc);
+    float* s_wq = reinterpret_cast<float*>(smem + kOffW);
+    double* s_inv = reinterpret_cast<double*>(smem + kOffInv);
+    volatile int* abort_flag = &misc->abort_flag;
+
+    const WsLayout L = ws_layout(p.T, p.nseg);
+    PlanHeader* hdr = reinterpret_cast<PlanHeader*>(p.ws + L.header);
+    const int4* items = reinterpret_cast<const int4*>(p.ws + L.items);
+    int* status = &hdr->status;
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+    // ---------------------------------------------------------------- setup
+    if (tid == 0) {
+        mbar_init(bar(B_SCHED_FULL + 0), 1);
+        mbar_init(bar(B_SCHED_FULL + 1), 1);
+        mbar_init(bar(B_SCHED_EMPTY + 0), 3);
+        mbar_init(bar(B_SCHED_EMPTY + 1), 3);
+        for (int t = 0; t < 2; ++t) {
+            mbar_init(bar(B_Q_FULL + t), 1);
+            mbar_init(bar(B_Q_READY + t), 1);
+            mbar_init(bar(B_Q_EMPTY + t), 1);
+            mbar_init(bar(B_K_FULL + t), 1);
+            mbar_init(bar(B_K_EMPTY + t), 1);
+            mbar_init(bar(B_V_FULL + t), 1);
+            mbar_init(bar(B_V_EMPTY + t), 1);
+            mbar_init(bar(B_S_FULL + t), 1);
+            mbar_init(bar(B_P_FULL + t), 1);
+            mbar_init(bar(B_O_FULL + t), 1);
+        }
+        mbar_init(bar(B_DRAIN), 1);
+        misc->abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&tm_q);
+        tma_prefetch_desc(&tm_k);
+        tma_prefetch_desc(&tm_v);
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(&misc->tmem_base), 512);
+        tmem_relinquish();
+    }
+    if (tid < kHD) s_wq[tid] = p.q_norm_w[tid];
+    if (tid >= 128 && tid < 192) s_inv[tid - 128] = exp2(-(double)(tid - 128) / 64.0 * log2((double)p.rope_theta));
+    if (warp == 2) {
+        const float mq = warp_max_abs128(p.q_norm_w);
+        const float mk = warp_max_abs128(p.k_norm_w);
+        if (lane == 0) {
+            const int eq = prescale_exponent(mq), ek = prescale_exponent(mk);
+            misc->q_scale = ldexpf(1.f, eq);
+            misc->logit_scale = ldexpf(1.4426950408889634f * 0.08838834764831845f, -(eq + ek));
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = misc->tmem_base;
+    const int n_units = hdr->n_items * kHKV;
+
+    if (warp == 0) {
+        // ============================================================ producer
+        if (lane == 0) {
+            uint32_t sslot = 0, sph = 0, qph = 0, kst = 0, kph = 0, vst = 0, vph = 0;
+            uint32_t narm_q = 0, narm_k[2] = {0, 0}, narm_v[2] = {0, 0};
+            for (;;) {
+                int u = atomicAdd(&hdr->counter, 1);
+                if (u >= n_units) u = -1;
+                if (!mbar_wait(bar(B_SCHED_EMPTY + sslot), sph ^ 1, abort_flag, status)) break;
+                misc->sched[sslot] = u;
+                mbar_arrive(bar(B_SCHED_FULL + sslot));
+                sslot ^= 1; if (sslot == 0) sph ^= 1;
+                if (u < 0) break;
+                const int4 it = items[u >> 2];
+                const int g = u & 3;
+                const int q0 = it.x, nq = it.y, ds = it.z, nch = it.w;
+                bool ok = true;
+                for (int t = 0; t < 2 && ok; ++t) {
+                    ok = mbar_wait(bar(B_Q_EMPTY + t), qph ^ 1, abort_flag, status);
+                    if (!ok) break;
+                    const uint32_t dst = sbase + kOffQ + t * kTileBytes;
+                    mbar_expect_tx(bar(B_Q_FULL + t), kTileBytes);
+                    tma_load_3d(dst, &tm_q, bar(B_Q_FULL + t), 0, kGroup * g, q0 + kTokPerTile * t);
+                    tma_load_3d(dst + kHalfTile, &tm_q, bar(B_Q_FULL + t), 64, kGroup * g,
+                                q0 + kTokPerTile * t);
+                }
+                if (!ok) break;
+                ++narm_q;
+                qph ^= 1;
+                const int ke = q0 + nq;
+                const int kb = p.window > 0 ? max(ds, q0 - p.window + 1) : ds;
+                (void)ke;
+                for (int c = 0; c < nch && ok; ++c) {
+                    const int ks = kb + kKeyChunk * c;
+                    ok = mbar_wait(bar(B_K_EMPTY + kst), kph ^ 1, abort_flag, status);
+                    if (!ok) break;
+                    uint32_t dst = sbase + kOffK + kst * kTileBytes;
+                    mbar_expect_tx(bar(B_K_FULL + kst), kTileBytes);
+                    tma_load_3d(dst, &tm_k, bar(B_K_FULL + kst), 0, g, ks);
+                    tma_load_3d(dst + kHalfTile, &tm_k, bar(B_K_FULL + kst), 64, g, ks);
+                    ++narm_k[kst];
+                    kst ^= 1; if (kst == 0) kph ^= 1;
+                    ok = mbar_wait(bar(B_V_EMPTY + vst), vph ^ 1, abort_flag, status);
+                    if (!ok) break;
+                    dst = sbase + kOffV + vst * kTileBytes;
+                    mbar_expect_tx(bar(B_V_FULL + vst), kTileBytes);
+                    tma_load_3d(dst, &tm_v, bar(B_V_FULL + vst), 0, g, ks);
+                    tma_load_3d(dst + kHalfTile, &tm_v, bar(B_V_FULL + vst), 64, g, ks);
+                    ++narm_v[vst];
+                    vst ^= 1; if (vst == 0) vph ^= 1;
+                }
+                if (!ok) break;
+            }
+            // drain: every armed load has landed before shared memory is released
+            const unsigned long long lim = 100ull * 1000ull * 1000ull;
+            volatile int never = 0;
+            for (int t = 0; t < 2; ++t)
+                if (narm_q) mbar_wait(bar(B_Q_FULL + t), (narm_q - 1) & 1, &never, nullptr, lim);
+            for (int s = 0; s < 2; ++s) {
+                if (narm_k[s]) mbar_wait(bar(B_K_FULL + s), (narm_k[s] - 1) & 1, &never, nullptr, lim);
+                if (narm_v[s]) mbar_wait(bar(B_V_FULL + s), (narm_v[s] - 1) & 1, &never, nullptr, lim);
+            }
+        }
+    } else if (warp == 1) {
+        // ============================================================ MMA issuer
+        if (lane == 0) {
+            const uint32_t idesc_pv = idesc_f16(1, 1, 1, 128);
+            const uint32_t q_addr[2] = {sbase + kOffQ, sbase + kOffQ + kTileBytes};
+            uint32_t sslot = 0, sph = 0, qrph = 0, kst = 0, kph = 0, vst = 0, vph = 0, pph = 0;
+            auto issue_s = [&](int t, uint32_t kstage, int ncols) {
+                const uint32_t idesc = idesc_f16(0, 0, 0, (uint32_t)ncols);
+                const uint32_t kaddr = sbase + kOffK + kstage * kTileBytes;
+#pragma unroll
+                for (int kk = 0; kk < kHD / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * kHalfTile + (kk & 3) * 32;
+                    mma_ss(tmem + 128u * t, smem_desc_sw128(q_addr[t] + off, 16, 1024),
+                           smem_desc_sw128(kaddr + off, 16, 1024), idesc, kk > 0);
+                }
+            };
+            auto issue_pv = [&](int t, uint32_t vstage, int ncols, bool acc) {
+                const uint32_t vaddr = sbase + kOffV + vstage * kTileBytes;
+                for (int kk = 0; kk < ncols / 16; ++kk) {
+                    mma_ts(tmem + 256u + 128u * t, tmem + 128u * t + 8u * kk,
+                           smem_desc_sw128(vaddr + kk * 2048, kHalfTile, 1024), idesc_pv,
+                           (acc || kk > 0) ? 1u : 0u);
+                }
+            };
+            for (;;) {
+                if (!mbar_wait(bar(B_SCHED_FULL + sslot), sph, abort_flag, status)) break;
+                const int u = misc->sched[sslot];
+                mbar_arrive(bar(B_SCHED_EMPTY + sslot));
+                sslot ^= 1; if (sslot == 0) sph ^= 1;
+                if (u < 0) break;
+                const int4 it = items[u >> 2];
+                const int q0 = it.x, nq = it.y, ds = it.z, nch = it.w;
+                const int ke = q0 + nq;
+                const int kb = p.window > 0 ? max(ds, q0 - p.window + 1) : ds;
+                if (!mbar_wait(bar(B_Q_READY + 0), qrph, abort_flag, status)) break;
+                if (!mbar_wait(bar(B_Q_READY + 1), qrph, abort_flag, status)) break;
+                qrph ^= 1;
+                tc_fence_after();
+                // S for chunk 0
+                if (!mbar_wait(bar(B_K_FULL + kst), kph, abort_flag, status)) break;
+                tc_fence_after();
+                int ncol = chunk_cols(kb, ke);
+                issue_s(0, kst, ncol);
+                mma_commit(bar(B_S_FULL + 0));
+                issue_s(1, kst, ncol);
+                mma_commit(bar(B_S_FULL + 1));
+                if (nch == 1) {
+                    mma_commit(bar(B_Q_EMPTY + 0));
+                    mma_commit(bar(B_Q_EMPTY + 1));
+                }
+                mma_commit(bar(B_K_EMPTY + kst));
+                kst ^= 1; if (kst == 0) kph ^= 1;
+                bool ok = true;
+                for (int c = 0; c < nch && ok; ++c) {
+                    const int nc_cur = ncol;
+                    int nc_next = 0;
+                    if (c + 1 < nch) nc_next = chunk_cols(kb + kKeyChunk * (c + 1), ke);
+                    ok = mbar_wait(bar(B_V_FULL + vst), vph, abort_flag, status);
+                    if (!ok) break;
+                    ok = mbar_wait(bar(B_P_FULL + 0), pph, abort_flag, status);
+                    if (!ok) break;
+                    tc_fence_after();
+                    issue_pv(0, vst, nc_cur, c > 0);
+                    if (c + 1 < nch) {
+                        ok = mbar_wait(bar(B_K_FULL + kst), kph, abort_flag, status);
+                        if (!ok) break;
+                        tc_fence_after();
+                        issue_s(0, kst, nc_next);
+                        mma_commit(bar(B_S_FULL + 0));
+                        if (c + 2 == nch) mma_commit(bar(B_Q_EMPTY + 0));
+                    } else {
+                        mma_commit(bar(B_O_FULL + 0));
+                    }
+                    ok = mbar_wait(bar(B_P_FULL + 1), pph, abort_flag, status);
+                    if (!ok) break;
+                    tc_fence_after();
+                    issue_pv(1, vst, nc_cur, c > 0);
+                    mma_commit(bar(B_V_EMPTY + vst));
+                    vst ^= 1; if (vst == 0) vph ^= 1;
+                    if (c + 1 < nch) {
+                        issue_s(1, kst, nc_next);
+                        mma_commit(bar(B_S_FULL + 1));
+                        if (c + 2 == nch) mma_commit(bar(B_Q_EMPTY + 1));
+                        mma_commit(bar(B_K_EMPTY + kst));
+                        kst ^= 1; if (kst == 0) kph ^= 1;
+                    } else {
+                        mma_commit(bar(B_O_FULL + 1));
+                    }
+                    pph ^= 1;
+                    ncol = nc_next;
+                }
+                if (!ok) break;
+            }
+            // drain: every MMA issued so far has completed
+            mma_commit(bar(B_DRAIN));
+            volatile int never = 0;
+            mbar_wait(bar(B_DRAIN), 0, &never, nullptr, 100ull * 1000ull * 1000ull);
+        }
+    } else if (warp >= 4) {
+        // ============================================================ softmax
+        const int t = (warp - 4) >> 2;               // tile 0 or 1
+        const int r = tid - 128 - 128 * t;           // row = TMEM lane, 0..127
+        const int tl = r >> 3, hl = r & 7;           // token within tile, head within group
+        const uint32_t wg_bar = 1 + t;
+        const uint32_t lane_base = (uint32_t)(warp & 3) * 32u;
+        const uint32_t t_s = tmem + (lane_base << 16) + 128u * t;
+        const uint32_t t_o = tmem + (lane_base << 16) + 256u + 128u * t;
+        const uint32_t q_tile = sbase + kOffQ + t * kTileBytes;
+        uint8_t* q_tile_ptr = smem + kOffQ + t * kTileBytes;
+        float2* rope_tab = reinterpret_cast<float2*>(smem + kOffRope + t * kRopeBytes);
+        const float C = misc->logit_scale;
+        const float qs = misc->q_scale;
+        uint32_t sslot = 0, sph = 0, qph = 0, s_ph = 0, oph = 0;
+        (void)q_tile;
+        for (;;) {
+            bool ok = mbar_wait(bar(B_SCHED_FULL + sslot), sph, abort_flag, status);
+            int u = ok ? misc->sched[sslot] : -1;
+            if (!wg_all(wg_bar, ok)) break;
+            if (r == 0) mbar_arrive(bar(B_SCHED_EMPTY + sslot));
+            sslot ^= 1; if (sslot == 0) sph ^= 1;
+            if (u < 0) break;
+            const int4 it = items[u >> 2];
+            const int g = u & 3;
+            const int q0 = it.x, nq = it.y, ds = it.z, nch = it.w;
+            const int h = kGroup * g + hl;
+            const int tok0 = q0 + kTokPerTile * t;
+            const int i = tok0 + tl;
+            const bool row_valid = (kTokPerTile * t + tl) < nq;
+            const int ke = q0 + nq;
+            const int kb = p.window > 0 ? max(ds, q0 - p.window + 1) : ds;
+
+            // ---- rope table for this tile's 16 tokens: thread r fills token
+            // tl, pair indices 8*hl .. 8*hl+7
+            if (p.use_rope) {
+                int pos = 0;
+                const int tok = min(i, p.T - 1);
+                pos = p.pos_ids ? p.pos_ids[tok] : (i - ds);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    float c, s;
+                    rope_cos_sin(pos, s_inv[8 * hl + e], &c, &s);
+                    rope_tab[tl * 64 + 8 * hl + e] = make_float2(c, s);
+                }
+            }
+            ok = mbar_wait(bar(B_Q_FULL + t), qph, abort_flag, status);
+            if (!wg_all(wg_bar, ok)) break;   // also publishes the rope table
+            qph ^= 1;
+
+            // ---- Q prologue, in place: RMSNorm (weight form), RoPE, x 2^eq, FP16.
+            // Thread r owns row r; chunk c of each 64-channel half sits at the
+            // 128-byte-swizzled position (c ^ (r & 7)).  Two passes over shared
+            // memory keep the row out of registers.
+            {
+                const int sw = r & 7;
+                float ss = 0.f;
+#pragma unroll 2
+                for (int c = 0; c < 8; ++c) {
+                    const int off = r * 128 + ((c ^ sw) << 4);
+                    const uint4 ua = *reinterpret_cast<const uint4*>(q_tile_ptr + off);
+                    const uint4 ub = *reinterpret_cast<const uint4*>(q_tile_ptr + kHalfTile + off);
+                    const uint32_t w8[8] = {ua.x, ua.y, ua.z, ua.w, ub.x, ub.y, ub.z, ub.w};
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        const float x0 = bf16_lo(w8[j]), x1 = bf16_hi(w8[j]);
+                        ss = fmaf(x0, x0, ss);
+                        ss = fmaf(x1, x1, ss);
+                    }
+                }
+                const float rn = rsqrtf(ss * (1.f / kHD) + p.eps) * qs;
+#pragma unroll 1
+                for (int c = 0; c < 8; ++c) {
+                    const int off = r * 128 + ((c ^ sw) << 4);
+                    const uint4 ua = *reinterpret_cast<const uint4*>(q_tile_ptr + off);
+                    const uint4 ub = *reinterpret_cast<const uint4*>(q_tile_ptr + kHalfTile + off);
+                    const uint32_t wa4[4] = {ua.x, ua.y, ua.z, ua.w};
+                    const uint32_t wb4[4] = {ub.x, ub.y, ub.z, ub.w};
+                    uint32_t oa[4], ob[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int d0 = 8 * c + 2 * e;          // channels d0, d0+1 and 64+d0, 65+d0
+                        float a0 = bf16_lo(wa4[e]) * rn * s_wq[d0];
+                        float a1 = bf16_hi(wa4[e]) * rn * s_wq[d0 + 1];
+                        float b0 = bf16_lo(wb4[e]) * rn * s_wq[64 + d0];
+                        float b1 = bf16_hi(wb4[e]) * rn * s_wq[65 + d0];
+                        if (p.use_rope) {
+                            const float2 cs0 = rope_tab[tl * 64 + d0];
+                            const float2 cs1 = rope_tab[tl * 64 + d0 + 1];
+                            const float y0 = a0 * cs0.x - b0 * cs0.y, z0 = b0 * cs0.x + a0 * cs0.y;
+                            const float y1 = a1 * cs1.x - b1 * cs1.y, z1 = b1 * cs1.x + a1 * cs1.y;
+                            a0 = y0; b0 = z0; a1 = y1; b1 = z1;
+                        }
+                        oa[e] = pack_f16(a0, a1);
+                        ob[e] = pack_f16(b0, b1);
+                    }
+                    *reinterpret_cast<uint4*>(q_tile_ptr + off) = make_uint4(oa[0], oa[1], oa[2], oa[3]);
+                    *reinterpret_cast<uint4*>(q_tile_ptr + kHalfTile + off) = make_uint4(ob[0], ob[1], ob[2], ob[3]);
+                }
+            }
+            fence_proxy_async_smem();
+            named_bar_sync(wg_bar, 128);
+            if (r == 0) mbar_arrive(bar(B_Q_READY + t));
+
+            // ---- online softmax over the key chunks
+            const float sink = p.sinks[h];
+            float m = sink * 1.4426950408889634f;      // log2 domain
+            float l = (sink == -INFINITY) ? 0.f : 1.f;
+            const int lo = p.window > 0 ? i - p.window + 1 : -(1 << 30);
+            bool alive = true;
+            for (int c = 0; c < nch; ++c) {
+                const int ks = kb + kKeyChunk * c;
+                const int nc = chunk_cols(ks, ke);
+                const int nblk = (nc + 31) >> 5;
+                ok = mbar_wait(bar(B_S_FULL + t), s_ph, abort_flag, status);
+                if (!wg_all(wg_bar, ok)) { alive = false; break; }
+                s_ph ^= 1;
+                tc_fence_after();
+                float s[128];
+#pragma unroll
+                for (int b = 0; b < 4; ++b) {
+                    if (b < nblk) {
+                        uint32_t v[32];
+                        tmem_ld32(t_s + 32u * b, v);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) s[32 * b + j] = __uint_as_float(v[j]);
+                    }
+                }
+                const bool boundary = (c == nch - 1) || (ks + nc - 1 > tok0) ||
+                                      (p.window > 0 && ks < tok0 + kTokPerTile - p.window);
+                float mx = -INFINITY;
+                if (boundary) {
+                    const int jlo = lo - ks, jhi = i - ks;
+#pragma unroll
+                    for (int b = 0; b < 4; ++b) {
+                        if (b < nblk) {
+#pragma unroll
+                            for (int j = 32 * b; j < 32 * b + 32; ++j) {
+                                const bool vis = (j >= jlo) && (j <= jhi);
+                                s[j] = vis ? s[j] : -INFINITY;
+                                mx = fmaxf(mx, s[j]);
+                            }
+                        }
+                    }
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 128; ++j) mx = fmaxf(mx, s[j]);
+                }
+                const float m_new = fmaxf(m, mx * C);
+                float m_use = m;
+                if (c == 0 ? (m_new > m) : (m_new > m + 8.f)) m_use = m_new;
+                const float alpha = (m_use == m) ? 1.f : ex2(m - m_use);
+                l *= alpha;
+                // rescale O in TMEM (warp-uniform: tcgen05.ld/st are .sync.aligned)
+                if (c > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+#pragma unroll 1
+                    for (int b = 0; b < 8; ++b) {
+                        uint32_t v[16];
+                        tmem_ld16(t_o + 16u * b, v);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) * alpha);
+                        tmem_st16(t_o + 16u * b, v);
+                    }
+                }
+                m = m_use;
+                const float negm = (m == -INFINITY) ? 0.f : -m;
+                float lsum = 0.f;
+#pragma unroll
+                for (int b = 0; b < 4; ++b) {
+                    if (b < nblk) {
+                        uint32_t pk[16];
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) {
+                            const float p0 = ex2(fmaf(s[32 * b + 2 * j], C, negm));
+                            const float p1 = ex2(fmaf(s[32 * b + 2 * j + 1], C, negm));
+                            lsum += p0 + p1;
+                            pk[j] = pack_bf16(p0, p1);
+                        }
+                        tmem_st16(t_s + 16u * b, pk);
+                    }
+                }
+                l += lsum;
+                tmem_wait_st();
+                tc_fence_before();
+                named_bar_sync(wg_bar, 128);
+                if (r == 0) mbar_arrive(bar(B_P_FULL + t));
+            }
+            if (!alive) break;
+
+            // ---- epilogue: O / l -> BF16, LSE
+            ok = mbar_wait(bar(B_O_FULL + t), oph, abort_flag, status);
+            if (!wg_all(wg_bar, ok)) break;
+            oph ^= 1;
+            tc_fence_after();
+            const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
+            __nv_bfloat16* orow = p.out + ((size_t)i * kHQ + h) * kHD;
+#pragma unroll
+            for (int b = 0; b < 4; ++b) {
+                uint32_t v[32];
+                tmem_ld32(t_o + 32u * b, v);
+                tmem_wait_ld();
+                uint32_t w[16];
+#pragma unroll
+                for (int j = 0; j < 16; ++j)
+                    w[j] = pack_bf16(__uint_as_float(v[2 * j]) * inv_l, __uint_as_float(v[2 * j + 1]) * inv_l);
+                if (row_valid) {
+                    uint4* dst = reinterpret_cast<uint4*>(orow + 32 * b);
+#pragma unroll
+                    for (int j = 0; j < 4; ++j)
+                        dst[j] = make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+                }
+            }
+            if (row_valid && p.lse) p.lse[(size_t)h * p.T + i] = m * 0.6931471805599453f + logf(l);
+            tc_fence_before();
+        }
+    }
+
+    // ---------------------------------------------------------------- teardown
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+extern const unsigned kAttnSmemBytes = kSmemBytes;
+
+}  // namespace flint

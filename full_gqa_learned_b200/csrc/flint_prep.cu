@@ -1,0 +1,299 @@
+// Preparation kernel of the Flint attention forward.
+//
+// Block 0 builds the work plan: it reads the document boundaries (packed THD
+// cu_seqlens) or the per-row valid lengths of a trailing padding mask,
+// splits every document into work items of 32 tokens and orders the items by
+// their number of 128-key chunks, longest first, so the attention kernel's
+// dynamic scheduler hands out the largest items first.
+//
+// The other blocks prepare the keys once per token instead of once per use:
+// per-head RMSNorm with k_norm_w (weight form; HF discussion #26 on
+// RecursiveSI/flint), then on sliding layers NeoX RoPE at the document-local
+// position (FlintAttention._apply_rope), scaled by a power of two and rounded
+// to FP16 into the workspace.  They also write the outputs of padded query
+// tokens: zeros and lse = sink (FlintAttention.forward, attention_mask: the
+// sink remains valid for padded queries).
+#include "flint_common.cuh"
+
+namespace flint {
+
+// ---------------------------------------------------------------- block scan
+// Inclusive prefix sum over the 1024 threads of the block; returns the block
+// total in *total.  `sh` holds 33 ints.
+__device__ int block_incl_scan(int v, int* sh, int* total) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        int t = __shfl_up_sync(0xffffffffu, v, o);
+        if (lane >= o) v += t;
+    }
+    if (lane == 31) sh[warp] = v;
+    __syncthreads();
+    if (warp == 0) {
+        int w = (lane < (int)(blockDim.x >> 5)) ? sh[lane] : 0;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            int t = __shfl_up_sync(0xffffffffu, w, o);
+            if (lane >= o) w += t;
+        }
+        sh[lane] = w;  // inclusive warp totals
+    }
+    __syncthreads();
+    int r = v + (warp > 0 ? sh[warp - 1] : 0);
+    *total = sh[(blockDim.x >> 5) - 1];
+    __syncthreads();
+    return r;
+}
+
+// Last segment s with prefix[s] <= it (prefix non-decreasing, prefix[0] = 0).
+__device__ __forceinline__ int find_segment(const int* prefix, int nseg, int it) {
+    int lo = 0, hi = nseg - 1;
+    while (lo < hi) {
+        int mid = (lo + hi + 1) >> 1;
+        if (prefix[mid] <= it) lo = mid; else hi = mid - 1;
+    }
+    return lo;
+}
+
+struct ItemDesc { int q0, nq, ds, nch; };
+
+__device__ __forceinline__ ItemDesc describe_item(const int2* seg, const int* prefix, int nseg,
+                                                 int it, int window) {
+    int s = find_segment(prefix, nseg, it);
+    // skip empty segments that share the same prefix value
+    while (s + 1 < nseg && prefix[s + 1] <= it) ++s;
+    int li = it - prefix[s];
+    int2 sg = seg[s];
+    ItemDesc d;
+    d.ds = sg.x;
+    d.q0 = sg.x + kTokPerItem * li;
+    d.nq = min(kTokPerItem, sg.y - kTokPerItem * li);
+    int ke = d.q0 + d.nq;
+    int kb = window > 0 ? max(d.ds, d.q0 - window + 1) : d.ds;
+    d.nch = (ke - kb + kKeyChunk - 1) / kKeyChunk;
+    return d;
+}
+
+__device__ void build_plan(const PrepParams& p) {
+    __shared__ int sh[33];
+    __shared__ int s_status;
+    const WsLayout L = ws_layout(p.T, p.nseg);
+    PlanHeader* hdr = reinterpret_cast<PlanHeader*>(p.ws + L.header);
+    int2* seg = reinterpret_cast<int2*>(p.ws + L.seg);
+    int* prefix = reinterpret_cast<int*>(p.ws + L.prefix);
+    int* hist = reinterpret_cast<int*>(p.ws + L.hist);
+    int4* items = reinterpret_cast<int4*>(p.ws + L.items);
+    const int tid = threadIdx.x, nthr = blockDim.x;
+    const int lane = tid & 31, warp = tid >> 5, nwarp = nthr >> 5;
+
+    if (tid == 0) s_status = kStatusOk;
+    for (int i = tid; i < L.hist_len; i += nthr) hist[i] = 0;
+    __syncthreads();
+
+    // 1. segments (start, valid length)
+    if (p.mode == kMaskThd) {
+        const int* cu = p.cu_seqlens;
+        if (tid == 0 && (cu[0] != 0 || cu[p.nseg] > p.T || cu[p.nseg] < 0))
+            atomicExch(&s_status, kStatusInvalid);
+        for (int s = tid; s < p.nseg; s += nthr) {
+            int a = cu[s], b = cu[s + 1];
+            if (b < a || a < 0) atomicExch(&s_status, kStatusInvalid);
+            seg[s] = make_int2(a, max(b - a, 0));
+        }
+    } else if (p.mode == kMaskPad) {
+        for (int row = warp; row < p.batch; row += nwarp) {
+            const uint8_t* m = p.pad_mask + (size_t)row * p.seqlen;
+            int cnt = 0, first_zero = p.seqlen, bad = 0;
+            for (int j = lane; j < p.seqlen; j += 32) {
+                int v = m[j];
+                if (v == 1) ++cnt;
+                else if (v == 0) first_zero = min(first_zero, j);
+                else bad = 1;
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
+                first_zero = min(first_zero, __shfl_xor_sync(0xffffffffu, first_zero, o));
+                bad |= __shfl_xor_sync(0xffffffffu, bad, o);
+            }
+            if (lane == 0) {
+                if (bad) atomicExch(&s_status, kStatusInvalid);
+                else if (first_zero < cnt) atomicCAS(&s_status, kStatusOk, kStatusUnsupported);
+                seg[row] = make_int2(row * p.seqlen, cnt);
+            }
+        }
+    } else {
+        if (tid == 0) seg[0] = make_int2(0, p.T);
+    }
+    __syncthreads();
+
+    // 2. items per segment, exclusive prefix over segments
+    int running = 0;
+    for (int base = 0; base < p.nseg; base += nthr) {
+        int s = base + tid;
+        int n = 0;
+        if (s < p.nseg) n = (seg[s].y + kTokPerItem - 1) / kTokPerItem;
+        int tot;
+        int incl = block_incl_scan(n, sh, &tot);
+        if (s < p.nseg) prefix[s] = running + incl - n;
+        running += tot;
+    }
+    if (tid == 0) prefix[p.nseg] = running;
+    const int n_items = (s_status == kStatusOk) ? running : 0;
+    __syncthreads();
+
+    // 3. histogram of chunk counts
+    for (int it = tid; it < n_items; it += nthr) {
+        ItemDesc d = describe_item(seg, prefix, p.nseg, it, p.window);
+        atomicAdd(&hist[d.nch], 1);
+    }
+    __syncthreads();
+
+    // 4. descending exclusive offsets: bin c starts after all bins c' > c
+    running = 0;
+    for (int base = 0; base < L.hist_len; base += nthr) {
+        int rb = base + tid;                       // reversed bin index
+        int c = L.hist_len - 1 - rb;
+        int n = (rb < L.hist_len) ? hist[c] : 0;
+        int tot;
+        int incl = block_incl_scan(n, sh, &tot);
+        if (rb < L.hist_len) hist[c] = running + incl - n;
+        running += tot;
+    }
+    __syncthreads();
+
+    // 5. scatter
+    for (int it = tid; it < n_items; it += nthr) {
+        ItemDesc d = describe_item(seg, prefix, p.nseg, it, p.window);
+        int at = atomicAdd(&hist[d.nch], 1);
+        items[at] = make_int4(d.q0, d.nq, d.ds, d.nch);
+    }
+    __syncthreads();
+    if (tid == 0) {
+        hdr->status = s_status;
+        hdr->n_items = n_items;
+        hdr->counter = 0;
+    }
+}
+
+// ---------------------------------------------------------------- key prep
+
+__device__ __forceinline__ int thd_segment_start(const int* cu, int ndocs, int t) {
+    // last d with cu[d] <= t
+    int lo = 0, hi = ndocs - 1;
+    while (lo < hi) {
+        int mid = (lo + hi + 1) >> 1;
+        if (cu[mid] <= t) lo = mid; else hi = mid - 1;
+    }
+    return cu[lo];
+}
+
+__device__ void prepare_keys(const PrepParams& p) {
+    __shared__ double s_inv_freq[64];
+    __shared__ float s_w[kHD];
+    __shared__ float s_scale;
+    __shared__ int s_thd_end;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const WsLayout L = ws_layout(p.T, p.nseg);
+    __half* kn = reinterpret_cast<__half*>(p.ws + L.kn);
+
+    if (tid < 64) s_inv_freq[tid] = exp2(-(double)tid / 64.0 * log2((double)p.rope_theta));
+    if (tid < kHD) s_w[tid] = p.k_norm_w[tid];
+    if (warp == 0) {
+        float m = warp_max_abs128(p.k_norm_w);
+        if (lane == 0) s_scale = ldexpf(1.f, prescale_exponent(m));
+    }
+    if (tid == 0) s_thd_end = (p.mode == kMaskThd) ? p.cu_seqlens[p.nseg] : p.T;
+    __syncthreads();
+
+    const int head = lane >> 3, sub = lane & 7;
+    const int nwarps_total = (gridDim.x - 1) * (blockDim.x >> 5);
+    const float scale = s_scale;
+    for (int t = (blockIdx.x - 1) * (blockDim.x >> 5) + warp; t < p.T; t += nwarps_total) {
+        // ---- normalise (and rotate) the 4 key heads of token t
+        const __nv_bfloat16* row = p.k + ((size_t)t * kHKV + head) * kHD;
+        uint4 a = *reinterpret_cast<const uint4*>(row + 8 * sub);
+        uint4 b = *reinterpret_cast<const uint4*>(row + 64 + 8 * sub);
+        float x0[8], x1[8];
+        {
+            const __nv_bfloat162* pa = reinterpret_cast<const __nv_bfloat162*>(&a);
+            const __nv_bfloat162* pb = reinterpret_cast<const __nv_bfloat162*>(&b);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                float2 fa = __bfloat1622float2(pa[e]);
+                float2 fb = __bfloat1622float2(pb[e]);
+                x0[2 * e] = fa.x; x0[2 * e + 1] = fa.y;
+                x1[2 * e] = fb.x; x1[2 * e + 1] = fb.y;
+            }
+        }
+        float ss = 0.f;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) ss = fmaf(x0[e], x0[e], fmaf(x1[e], x1[e], ss));
+        ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+        ss += __shfl_xor_sync(0xffffffffu, ss, 2);
+        ss += __shfl_xor_sync(0xffffffffu, ss, 4);
+        const float r = rsqrtf(ss * (1.f / kHD) + p.eps) * scale;
+        float n0[8], n1[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            n0[e] = x0[e] * r * s_w[8 * sub + e];
+            n1[e] = x1[e] * r * s_w[64 + 8 * sub + e];
+        }
+        if (p.use_rope) {
+            int pos;
+            if (p.pos_ids) pos = p.pos_ids[t];
+            else if (p.mode == kMaskThd) pos = t - (t < s_thd_end ? thd_segment_start(p.cu_seqlens, p.nseg, t) : s_thd_end);
+            else if (p.mode == kMaskPad) pos = t % p.seqlen;
+            else pos = t;
+            // lane computes the pairs f = 2*lane and 2*lane + 1
+            float c0, s0, c1, s1;
+            rope_cos_sin(pos, s_inv_freq[2 * lane], &c0, &s0);
+            rope_cos_sin(pos, s_inv_freq[2 * lane + 1], &c1, &s1);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const int f = 8 * sub + e;             // pair index of this element
+                const int src = f >> 1;
+                float cc = __shfl_sync(0xffffffffu, (f & 1) ? c1 : c0, src);
+                float sn = __shfl_sync(0xffffffffu, (f & 1) ? s1 : s0, src);
+                // (e & 1) is uniform across the warp for a given e, so the
+                // selected register is the same in every lane
+                float y0 = n0[e] * cc - n1[e] * sn;
+                float y1 = n1[e] * cc + n0[e] * sn;
+                n0[e] = y0; n1[e] = y1;
+            }
+        }
+        uint4 oa, ob;
+        {
+            __half2* ha = reinterpret_cast<__half2*>(&oa);
+            __half2* hb = reinterpret_cast<__half2*>(&ob);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                ha[e] = __floats2half2_rn(n0[2 * e], n0[2 * e + 1]);
+                hb[e] = __floats2half2_rn(n1[2 * e], n1[2 * e + 1]);
+            }
+        }
+        __half* dst = kn + ((size_t)t * kHKV + head) * kHD;
+        *reinterpret_cast<uint4*>(dst + 8 * sub) = oa;
+        *reinterpret_cast<uint4*>(dst + 64 + 8 * sub) = ob;
+
+        // ---- padded query token: zero output row, lse = sink
+        bool padded;
+        if (p.mode == kMaskThd) padded = t >= s_thd_end;
+        else if (p.mode == kMaskPad) padded = p.pad_mask[t] == 0;
+        else padded = false;
+        if (padded) {
+            uint4 z = make_uint4(0, 0, 0, 0);
+            uint4* o = reinterpret_cast<uint4*>(p.out + (size_t)t * kHQ * kHD);
+#pragma unroll 4
+            for (int i = lane; i < kHQ * kHD / 8; i += 32) o[i] = z;
+            if (p.lse) p.lse[(size_t)lane * p.T + t] = p.sinks[lane];
+        }
+    }
+}
+
+__global__ void __launch_bounds__(1024, 1) prep_kernel(PrepParams p) {
+    if (blockIdx.x == 0) build_plan(p);
+    else prepare_keys(p);
+}
+
+}  // namespace flint

@@ -1,0 +1,178 @@
+/*
+ * flint_attn.h - C ABI of the B200 (sm_100a) sink-aware GQA attention forward
+ * of the Flint hybrid-attention MoE decoder.
+ *
+ * The operation is the core of FlintAttention.forward (NeMo AutoModel API
+ * page "nemo_automodel.components.models.flint.layers", FlintAttention.forward:
+ * "full-sequence causal attention with a zero-value sink category"), from the
+ * projected Q/K/V up to the input of o_proj:
+ *
+ *   1. per-head RMSNorm on Q and K in weight form, x / sqrt(mean(x^2) + eps) * w
+ *      (HF discussion #26 on RecursiveSI/flint: plain RMSNorm, not 1+w;
+ *      FlintConfig.rms_norm_eps = 1e-6; model page, "Model Architecture":
+ *      query/key normalisation precedes RoPE);
+ *   2. on sliding layers only, NeoX RoPE over all 128 channels, channel i
+ *      rotated against channel i+64 at the token's document-local position
+ *      (FlintAttention._apply_rope; FlintConfig: sliding layers rotate all
+ *      head channels);
+ *   3. causal attention of 32 query heads over 4 key/value heads (query head h
+ *      reads KV head h/8), logits scaled by 1/sqrt(128), full or restricted to
+ *      a window that counts the current token (513 = current + 512 preceding;
+ *      model page "Model Architecture", FlintConfig.sliding_window);
+ *   4. one learned FP32 sink per query head acting as an extra softmax column
+ *      with zero value, in natural-logit units and not scaled by 1/sqrt(d)
+ *      (HF discussion #26, learned-sink semantics and item 5;
+ *      _FlintSinkParameters.forward returns unscaled sink logits);
+ *   5. padded queries and keys are excluded, the sink stays valid, so a padded
+ *      query's output is zero and its LSE equals the sink
+ *      (FlintAttention.forward, attention_mask).
+ *
+ * Memory: every pointer argument except the host-side `stream` handle is a
+ * DEVICE pointer owned by the caller.  The library never allocates; the call
+ * is asynchronous on `stream` (a cudaStream_t; NULL = legacy default stream).
+ * Argument errors are detected on the host before any launch and return a
+ * status without touching the GPU.  Errors that can only be seen on the
+ * device (an ill-formed cu_seqlens or padding mask, a timed-out wait inside a
+ * kernel) are recorded in the workspace and read back with
+ * flint_attn_device_status().
+ */
+#ifndef FLINT_ATTN_H_
+#define FLINT_ATTN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define FLINT_API __attribute__((visibility("default")))
+#else
+#define FLINT_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    FLINT_OK = 0,
+    FLINT_ERR_INVALID_ARG = 1,  /* bad pointer, size, alignment or flag */
+    FLINT_ERR_UNSUPPORTED = 2,  /* well-formed but outside what the kernels do
+                                   (non-trailing padding mask, no sm_100 GPU) */
+    FLINT_ERR_CUDA = 3,         /* a CUDA runtime/driver call failed */
+    FLINT_ERR_TIMEOUT = 4,      /* a bounded wait inside a kernel ran out */
+    FLINT_ERR_WORKSPACE = 5     /* workspace missing, misaligned or too small */
+} flint_status_t;
+
+#define FLINT_HQ 32      /* query heads            */
+#define FLINT_HKV 4      /* key/value heads        */
+#define FLINT_HEAD_DIM 128
+#define FLINT_MAX_TOKENS (1 << 24)
+
+/* ABI revision of this header (bumped on any signature change). */
+FLINT_API int32_t flint_attn_abi_version(void);
+
+/*
+ * Bytes of device workspace flint_attn_fwd needs for T tokens split into
+ * `num_segments` documents or batch rows (1 for a single sequence).  The
+ * workspace holds the normalised/rotated keys (FP16, 1 KiB per token), the
+ * work plan and a status word.  Returns 0 for invalid sizes.
+ */
+FLINT_API size_t flint_attn_workspace_bytes(int32_t T, int32_t num_segments);
+
+/*
+ * Sink-aware GQA attention forward.
+ *
+ *  q          bf16 [T,32,128] contiguous: projected queries, before q_norm.
+ *  k, v       bf16 [T,4,128] contiguous: projected keys (before k_norm), values.
+ *             q, k, v and out must be 16-byte aligned.  K and V must be finite
+ *             at every token, padded ones included.
+ *  q_norm_w   fp32 [128] q_norm weight, shared by all query heads.
+ *  k_norm_w   fp32 [128] k_norm weight, shared by all key heads.
+ *  sinks      fp32 [32] sink logits in natural-log units (may be +-inf).
+ *  pos_ids    int32 [T] document-local positions used by RoPE; NULL means the
+ *             index of the token within its document / batch row.  Ignored
+ *             when use_rope == 0.
+ *  cu_seqlens int32 [num_docs+1] packed-THD document boundaries: cu[0] = 0,
+ *             non-decreasing, cu[num_docs] <= T; tokens >= cu[num_docs] are
+ *             padding.  NULL when not packed.
+ *  pad_mask   uint8 [batch, seqlen], 1 = valid token, 0 = padding; every row
+ *             must be ones followed by zeros (trailing padding), otherwise the
+ *             device status becomes FLINT_ERR_UNSUPPORTED and no output is
+ *             produced.  NULL when unpadded.  At most one of cu_seqlens and
+ *             pad_mask may be non-NULL; with neither, q is one sequence.
+ *  batch, seqlen  shape of pad_mask (batch * seqlen == T); ignored otherwise.
+ *  T          total tokens, 0 <= T <= FLINT_MAX_TOKENS (T == 0: no-op).
+ *  window     0 for full causal attention; W > 0 keeps keys j with
+ *             i - W < j <= i (W = 513 on Flint's sliding layers).
+ *  use_rope   1 on sliding layers, 0 on full layers.
+ *  rope_theta RoPE base (> 1), e.g. 10000.
+ *  eps        RMSNorm epsilon (> 0), 1e-6 for Flint.
+ *  out        bf16 [T,4096]: out[t, h*128 + c], the o_proj input.  Rows of
+ *             padded tokens are written as +0.0.
+ *  lse        fp32 [32,T] natural-log sum of exponentials including the sink
+ *             (lse[h*T + t]); padded tokens get sinks[h].  May be NULL.
+ *  workspace  device buffer of at least flint_attn_workspace_bytes(T, n)
+ *             bytes, 256-byte aligned, where n = num_docs, batch or 1.
+ *             Must not be shared by calls that may overlap on the GPU.
+ *  stream     cudaStream_t as void*.
+ *
+ * Returns FLINT_OK once the kernels are enqueued.
+ */
+FLINT_API flint_status_t flint_attn_fwd(const void* q, const void* k, const void* v,
+                              const float* q_norm_w, const float* k_norm_w,
+                              const float* sinks, const int32_t* pos_ids,
+                              const int32_t* cu_seqlens, int32_t num_docs,
+                              const uint8_t* pad_mask, int32_t batch, int32_t seqlen,
+                              int32_t T, int32_t window, int32_t use_rope,
+                              float rope_theta, float eps,
+                              void* out, float* lse,
+                              void* workspace, size_t workspace_bytes,
+                              void* stream);
+
+/*
+ * The two stages flint_attn_fwd enqueues, exposed so a caller (or a profiler)
+ * can time them apart.  flint_attn_prepare runs the preparation kernel: the
+ * work plan, the normalised/rotated FP16 keys in the workspace and the
+ * outputs of padded query tokens.  flint_attn_attend runs the attention
+ * kernel on a workspace that flint_attn_prepare filled with the same
+ * arguments; calling it with other arguments is undefined.  Both take the
+ * arguments of flint_attn_fwd and validate them the same way.
+ */
+FLINT_API flint_status_t flint_attn_prepare(const void* q, const void* k, const void* v,
+                              const float* q_norm_w, const float* k_norm_w,
+                              const float* sinks, const int32_t* pos_ids,
+                              const int32_t* cu_seqlens, int32_t num_docs,
+                              const uint8_t* pad_mask, int32_t batch, int32_t seqlen,
+                              int32_t T, int32_t window, int32_t use_rope,
+                              float rope_theta, float eps,
+                              void* out, float* lse,
+                              void* workspace, size_t workspace_bytes,
+                              void* stream);
+FLINT_API flint_status_t flint_attn_attend(const void* q, const void* k, const void* v,
+                              const float* q_norm_w, const float* k_norm_w,
+                              const float* sinks, const int32_t* pos_ids,
+                              const int32_t* cu_seqlens, int32_t num_docs,
+                              const uint8_t* pad_mask, int32_t batch, int32_t seqlen,
+                              int32_t T, int32_t window, int32_t use_rope,
+                              float rope_theta, float eps,
+                              void* out, float* lse,
+                              void* workspace, size_t workspace_bytes,
+                              void* stream);
+
+/*
+ * Synchronises `stream`, then returns the status the kernels of the last
+ * flint_attn_fwd on `workspace` recorded (FLINT_OK, FLINT_ERR_INVALID_ARG for
+ * an ill-formed cu_seqlens, FLINT_ERR_UNSUPPORTED for a non-trailing mask,
+ * FLINT_ERR_TIMEOUT), or FLINT_ERR_CUDA if synchronising failed.
+ */
+FLINT_API flint_status_t flint_attn_device_status(const void* workspace, void* stream);
+
+/* Text of the last error raised on the calling host thread ("" if none). */
+FLINT_API const char* flint_attn_last_error(void);
+
+/* Fixed name of a status code. */
+FLINT_API const char* flint_attn_status_string(flint_status_t status);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* FLINT_ATTN_H_ */

@@ -1,0 +1,125 @@
+"""Host-only checks of the C ABI: the library builds and loads, exports every
+function include/flint_attn.h declares, and rejects bad arguments before it
+touches the GPU (these calls pass fake, never-dereferenced addresses)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import full_gqa_learned_b200 as fa
+from full_gqa_learned_b200 import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "flint_attn.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return fa.load_library()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(flint_attn_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for n in ("flint_attn_fwd", "flint_attn_workspace_bytes", "flint_attn_device_status",
+              "flint_attn_last_error", "flint_attn_status_string", "flint_attn_abi_version"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for n in declared_functions():
+        assert hasattr(lib, n), n
+
+
+def test_no_unexpected_exports(lib):
+    import subprocess
+    out = subprocess.run(["nm", "-D", "--defined-only", fa.LIB_PATH], capture_output=True,
+                         text=True).stdout
+    exported = set(re.findall(r" T (flint_\w+)", out))
+    assert exported == set(declared_functions())
+
+
+def test_version_and_status_strings(lib):
+    assert lib.flint_attn_abi_version() == 1
+    assert lib.flint_attn_status_string(0) == b"FLINT_OK"
+    assert lib.flint_attn_status_string(5) == b"FLINT_ERR_WORKSPACE"
+
+
+def test_workspace_bytes(lib):
+    assert fa.workspace_bytes(0, 1) > 0
+    a = fa.workspace_bytes(4096, 1)
+    # normalised FP16 keys dominate: 1 KiB per token
+    assert 4096 * 1024 <= a < 4096 * 1024 + (1 << 20)
+    assert fa.workspace_bytes(-1, 1) == 0
+    assert fa.workspace_bytes(1 << 25, 1) == 0
+    assert fa.workspace_bytes(4096, 8) >= a
+
+
+A = 0x100000  # fake, 256-byte aligned, never dereferenced
+
+
+def call(lib, **kw):
+    args = dict(q=A, k=A, v=A, wq=A, wk=A, sinks=A, pos=None, cu=None, ndocs=0, mask=None,
+                batch=0, seqlen=0, T=64, window=513, use_rope=1, theta=1e4, eps=1e-6,
+                out=A, lse=A, ws=A, ws_bytes=1 << 40, stream=None)
+    args.update(kw)
+    return lib.flint_attn_fwd(args["q"], args["k"], args["v"], args["wq"], args["wk"],
+                              args["sinks"], args["pos"], args["cu"], args["ndocs"],
+                              args["mask"], args["batch"], args["seqlen"], args["T"],
+                              args["window"], args["use_rope"], args["theta"], args["eps"],
+                              args["out"], args["lse"], args["ws"], args["ws_bytes"],
+                              args["stream"])
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(T=-1), 1),
+    (dict(T=(1 << 24) + 1), 1),
+    (dict(window=-5), 1),
+    (dict(use_rope=2), 1),
+    (dict(eps=0.0), 1),
+    (dict(eps=float("nan")), 1),
+    (dict(theta=1.0), 1),
+    (dict(cu=A, mask=A), 1),
+    (dict(cu=A, ndocs=-1), 1),
+    (dict(mask=A, batch=3, seqlen=5, T=16), 1),
+    (dict(mask=A, batch=0, seqlen=5, T=0), 1),
+    (dict(q=None), 1),
+    (dict(sinks=None), 1),
+    (dict(out=None), 1),
+    (dict(q=A + 8), 1),
+    (dict(out=A + 2), 1),
+    (dict(wq=A + 2), 1),
+    (dict(ws=None), 5),
+    (dict(ws=A + 64), 5),
+    (dict(ws_bytes=1024), 5),
+])
+def test_invalid_arguments_rejected_on_host(lib, kw, status):
+    assert call(lib, **kw) == status
+    assert lib.flint_attn_last_error() != b""
+
+
+def test_empty_input_is_a_noop(lib):
+    assert call(lib, T=0) == 0
+    assert call(lib, T=0, q=None, k=None, v=None, out=None, ws=None) == 0
+
+
+def test_rope_theta_ignored_without_rope(lib):
+    # theta is only validated on sliding layers; the call then fails on the
+    # workspace size, before any device work
+    assert call(lib, use_rope=0, theta=0.0, ws_bytes=16) == 5
+
+
+def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
+    import importlib
+    monkeypatch.setattr(fa, "LIB_PATH", str(tmp_path / "missing.so"))
+    monkeypatch.setattr(fa, "_lib", None)
+    with pytest.raises(ImportError):
+        fa.load_library()
+    importlib.reload(fa)
