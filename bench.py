@@ -182,8 +182,9 @@ def run_flint(args, rank, world, local_rank):
     sampler = ClockSampler(local_rank if "CUDA_VISIBLE_DEVICES" not in os.environ else
                            os.environ["CUDA_VISIBLE_DEVICES"].split(",")[local_rank])
     sampler.start()
-    time.sleep(0.3)
-    t_end = time.time() + args.soak
+    if not args.profile:
+        time.sleep(0.3)
+    t_end = time.time() + (0.0 if args.profile else args.soak)
     while time.time() < t_end:
         for _ in range(20):
             step()
@@ -207,6 +208,10 @@ def run_flint(args, rank, world, local_rank):
     step_ms = [e[0].elapsed_time(e[2]) for e in evs]
     total_ms = sum(step_ms)
     attn_avg = sum(attn_ms) / len(attn_ms)
+
+    if args.profile:
+        return dict(w=w, total_ms=total_ms, attn_avg=attn_avg, prep_avg=sum(prep_ms) / len(prep_ms),
+                    e2e_ms=float("nan"), h2d=0, d2h=0, clocks=clocks, launches=2 * args.steps)
 
     # end-to-end through the public API from pinned host buffers
     pinned = {k: v.pin_memory() for k, v in host.items()}
@@ -283,6 +288,8 @@ def main():
     ap.add_argument("--impl", default="flint", choices=["flint", "reference"])
     ap.add_argument("--soak", type=float, default=1.0, help="seconds of untimed load before timing")
     ap.add_argument("--cpu-budget", type=float, default=12.0)
+    ap.add_argument("--profile", action="store_true",
+                    help="warm-up and timed steps only (for ncu captures): no soak, e2e or CPU leg")
     ap.add_argument("--traffic", type=float, default=None,
                     help="ncu DRAM bytes per attention launch, if captured for this kernel")
     args = ap.parse_args()
@@ -352,7 +359,7 @@ def main():
         gpu_launches=r["launches"], clocks=r["clocks"],
         pct_of_tensor_peak=round(100.0 * value / world / peak, 2),
     )
-    if rank == 0 and world == 1:
+    if rank == 0 and world == 1 and not args.profile:
         line["cpu_baseline"] = cpu_baseline(w, budget_s=args.cpu_budget)
     if world > 1:
         dist.barrier()

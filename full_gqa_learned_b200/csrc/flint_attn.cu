@@ -31,6 +31,9 @@
 namespace flint {
 
 constexpr int kThreads = 384;
+constexpr uint32_t kRegsControl = 80;
+constexpr uint32_t kRegsSoftmax = 208;
+static_assert(128 * kRegsControl + 256 * kRegsSoftmax <= 384 * 168, "register split");
 constexpr uint32_t kTileBytes = 128 * kHD * 2;       // 32 KiB: 128 rows x 128 x 16-bit
 constexpr uint32_t kHalfTile = kTileBytes / 2;       // one 64-column swizzled half
 
@@ -173,11 +176,16 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const uint32_t tmem = misc->tmem_base;
     const int n_units = hdr->n_items * kHKV;
 
-    if (warp == 0) {
+    // Registers: launched with 384 x 168 = 64512.  Warps 0-3 (producer, MMA,
+    // two idle) drop to kRegsControl, the two softmax warpgroups rise to
+    // kRegsSoftmax; 128*80 + 256*208 = 63488 <= 64512.
+    if (warp < 4) {
+      regs_dec<kRegsControl>();
+      if (warp == 0) {
         // ============================================================ producer
         if (lane == 0) {
             uint32_t sslot = 0, sph = 0, qph = 0, kst = 0, kph = 0, vst = 0, vph = 0;
-            uint32_t narm_q = 0, narm_k[2] = {0, 0}, narm_v[2] = {0, 0};
+            uint32_t narm_q = 0, narm_k = 0, narm_v = 0;   // loads armed so far
             for (;;) {
                 int u = atomicAdd(&hdr->counter, 1);
                 if (u >= n_units) u = -1;
@@ -213,7 +221,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     mbar_expect_tx(bar(B_K_FULL + kst), kTileBytes);
                     tma_load_3d(dst, &tm_k, bar(B_K_FULL + kst), 0, g, ks);
                     tma_load_3d(dst + kHalfTile, &tm_k, bar(B_K_FULL + kst), 64, g, ks);
-                    ++narm_k[kst];
+                    ++narm_k;
                     kst ^= 1; if (kst == 0) kph ^= 1;
                     ok = mbar_wait(bar(B_V_EMPTY + vst), vph ^ 1, abort_flag, status);
                     if (!ok) break;
@@ -221,7 +229,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     mbar_expect_tx(bar(B_V_FULL + vst), kTileBytes);
                     tma_load_3d(dst, &tm_v, bar(B_V_FULL + vst), 0, g, ks);
                     tma_load_3d(dst + kHalfTile, &tm_v, bar(B_V_FULL + vst), 64, g, ks);
-                    ++narm_v[vst];
+                    ++narm_v;
                     vst ^= 1; if (vst == 0) vph ^= 1;
                 }
                 if (!ok) break;
@@ -231,34 +239,40 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             volatile int never = 0;
             for (int t = 0; t < 2; ++t)
                 if (narm_q) mbar_wait(bar(B_Q_FULL + t), (narm_q - 1) & 1, &never, nullptr, lim);
-            for (int s = 0; s < 2; ++s) {
-                if (narm_k[s]) mbar_wait(bar(B_K_FULL + s), (narm_k[s] - 1) & 1, &never, nullptr, lim);
-                if (narm_v[s]) mbar_wait(bar(B_V_FULL + s), (narm_v[s] - 1) & 1, &never, nullptr, lim);
+            for (uint32_t s = 0; s < 2; ++s) {
+                // stage s received loads number s, s+2, s+4, ...
+                const uint32_t nk = (narm_k + 1 - s) / 2, nv = (narm_v + 1 - s) / 2;
+                if (nk) mbar_wait(bar(B_K_FULL + s), (nk - 1) & 1, &never, nullptr, lim);
+                if (nv) mbar_wait(bar(B_V_FULL + s), (nv - 1) & 1, &never, nullptr, lim);
             }
         }
-    } else if (warp == 1) {
+      } else if (warp == 1) {
         // ============================================================ MMA issuer
         if (lane == 0) {
             const uint32_t idesc_pv = idesc_f16(1, 1, 1, 128);
-            const uint32_t q_addr[2] = {sbase + kOffQ, sbase + kOffQ + kTileBytes};
+            // Base descriptors; the start-address field (bits 0..13, in 16-byte
+            // units) is advanced by adding the byte offset >> 4, which stays
+            // inside the field for every offset used below.
+            const uint64_t dq0 = smem_desc_sw128(sbase + kOffQ, 16, 1024);
+            const uint64_t dk0 = smem_desc_sw128(sbase + kOffK, 16, 1024);
+            const uint64_t dv0 = smem_desc_sw128(sbase + kOffV, kHalfTile, 1024);
+            constexpr uint64_t kTileStep = kTileBytes >> 4;
             uint32_t sslot = 0, sph = 0, qrph = 0, kst = 0, kph = 0, vst = 0, vph = 0, pph = 0;
-            auto issue_s = [&](int t, uint32_t kstage, int ncols) {
+            auto issue_s = [=](uint32_t t, uint32_t kstage, int ncols) {
                 const uint32_t idesc = idesc_f16(0, 0, 0, (uint32_t)ncols);
-                const uint32_t kaddr = sbase + kOffK + kstage * kTileBytes;
+                const uint64_t dq = dq0 + t * kTileStep, dk = dk0 + kstage * kTileStep;
 #pragma unroll
-                for (int kk = 0; kk < kHD / 16; ++kk) {
-                    const uint32_t off = (kk >> 2) * kHalfTile + (kk & 3) * 32;
-                    mma_ss(tmem + 128u * t, smem_desc_sw128(q_addr[t] + off, 16, 1024),
-                           smem_desc_sw128(kaddr + off, 16, 1024), idesc, kk > 0);
+                for (uint32_t kk = 0; kk < kHD / 16; ++kk) {
+                    const uint64_t off = (kk >> 2) * (kHalfTile >> 4) + (kk & 3) * 2;
+                    mma_ss(tmem + 128u * t, dq + off, dk + off, idesc, kk > 0);
                 }
             };
-            auto issue_pv = [&](int t, uint32_t vstage, int ncols, bool acc) {
-                const uint32_t vaddr = sbase + kOffV + vstage * kTileBytes;
-                for (int kk = 0; kk < ncols / 16; ++kk) {
+            auto issue_pv = [=](uint32_t t, uint32_t vstage, int ncols, bool acc) {
+                const uint64_t dv = dv0 + vstage * kTileStep;
+                const int nk = ncols >> 4;
+                for (int kk = 0; kk < nk; ++kk)
                     mma_ts(tmem + 256u + 128u * t, tmem + 128u * t + 8u * kk,
-                           smem_desc_sw128(vaddr + kk * 2048, kHalfTile, 1024), idesc_pv,
-                           (acc || kk > 0) ? 1u : 0u);
-                }
+                           dv + (uint64_t)kk * (2048 >> 4), idesc_pv, (acc || kk > 0) ? 1u : 0u);
             };
             for (;;) {
                 if (!mbar_wait(bar(B_SCHED_FULL + sslot), sph, abort_flag, status)) break;
@@ -334,7 +348,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             volatile int never = 0;
             mbar_wait(bar(B_DRAIN), 0, &never, nullptr, 100ull * 1000ull * 1000ull);
         }
-    } else if (warp >= 4) {
+      }
+    } else {
+        regs_inc<kRegsSoftmax>();
         // ============================================================ softmax
         const int t = (warp - 4) >> 2;               // tile 0 or 1
         const int r = tid - 128 - 128 * t;           // row = TMEM lane, 0..127
@@ -452,20 +468,19 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 if (!wg_all(wg_bar, ok)) { alive = false; break; }
                 s_ph ^= 1;
                 tc_fence_after();
-                float s[128];
+                // all S columns of this chunk: one TMEM load per 32 columns,
+                // a single wait
+                uint32_t sv[128];
 #pragma unroll
-                for (int b = 0; b < 4; ++b) {
-                    if (b < nblk) {
-                        uint32_t v[32];
-                        tmem_ld32(t_s + 32u * b, v);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int j = 0; j < 32; ++j) s[32 * b + j] = __uint_as_float(v[j]);
-                    }
-                }
+                for (int b = 0; b < 4; ++b)
+                    if (b < nblk) tmem_ld32(t_s + 32u * b, sv + 32 * b);
+                tmem_wait_ld();
                 const bool boundary = (c == nch - 1) || (ks + nc - 1 > tok0) ||
                                       (p.window > 0 && ks < tok0 + kTokPerTile - p.window);
-                float mx = -INFINITY;
+                // row max over visible keys, 8 independent chains
+                float mxp[8];
+#pragma unroll
+                for (int k8 = 0; k8 < 8; ++k8) mxp[k8] = -INFINITY;
                 if (boundary) {
                     const int jlo = lo - ks, jhi = i - ks;
 #pragma unroll
@@ -474,15 +489,18 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 #pragma unroll
                             for (int j = 32 * b; j < 32 * b + 32; ++j) {
                                 const bool vis = (j >= jlo) && (j <= jhi);
-                                s[j] = vis ? s[j] : -INFINITY;
-                                mx = fmaxf(mx, s[j]);
+                                const float x = vis ? __uint_as_float(sv[j]) : -INFINITY;
+                                sv[j] = __float_as_uint(x);
+                                mxp[j & 7] = fmaxf(mxp[j & 7], x);
                             }
                         }
                     }
                 } else {
 #pragma unroll
-                    for (int j = 0; j < 128; ++j) mx = fmaxf(mx, s[j]);
+                    for (int j = 0; j < 128; ++j) mxp[j & 7] = fmaxf(mxp[j & 7], __uint_as_float(sv[j]));
                 }
+                const float mx = fmaxf(fmaxf(fmaxf(mxp[0], mxp[1]), fmaxf(mxp[2], mxp[3])),
+                                       fmaxf(fmaxf(mxp[4], mxp[5]), fmaxf(mxp[6], mxp[7])));
                 const float m_new = fmaxf(m, mx * C);
                 float m_use = m;
                 if (c == 0 ? (m_new > m) : (m_new > m + 8.f)) m_use = m_new;
@@ -502,21 +520,24 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 }
                 m = m_use;
                 const float negm = (m == -INFINITY) ? 0.f : -m;
-                float lsum = 0.f;
+                float lp[8];
+#pragma unroll
+                for (int k8 = 0; k8 < 8; ++k8) lp[k8] = 0.f;
 #pragma unroll
                 for (int b = 0; b < 4; ++b) {
                     if (b < nblk) {
                         uint32_t pk[16];
 #pragma unroll
                         for (int j = 0; j < 16; ++j) {
-                            const float p0 = ex2(fmaf(s[32 * b + 2 * j], C, negm));
-                            const float p1 = ex2(fmaf(s[32 * b + 2 * j + 1], C, negm));
-                            lsum += p0 + p1;
+                            const float p0 = ex2(fmaf(__uint_as_float(sv[32 * b + 2 * j]), C, negm));
+                            const float p1 = ex2(fmaf(__uint_as_float(sv[32 * b + 2 * j + 1]), C, negm));
+                            lp[j & 7] += p0 + p1;
                             pk[j] = pack_bf16(p0, p1);
                         }
                         tmem_st16(t_s + 16u * b, pk);
                     }
                 }
+                const float lsum = ((lp[0] + lp[1]) + (lp[2] + lp[3])) + ((lp[4] + lp[5]) + (lp[6] + lp[7]));
                 l += lsum;
                 tmem_wait_st();
                 tc_fence_before();
