@@ -73,6 +73,32 @@ __device__ __forceinline__ float ex2(float x) {
     return y;
 }
 
+// Coefficients of the degree-4 polynomial for 2^f on [-1/2, 1/2], written by
+// exp2_poly_fit.py (max relative error 2.6e-6).
+constexpr float kExp2C0 = 9.999992847e-01f;
+constexpr float kExp2C1 = 6.931217909e-01f;
+constexpr float kExp2C2 = 2.402474433e-01f;
+constexpr float kExp2C3 = 5.591785908e-02f;
+constexpr float kExp2C4 = 9.570101276e-03f;
+
+// 2^x on the FMA and integer pipes, for finite x <= 64 (results below 2^-126
+// flush towards 2^-126).  Cody-Waite split x = n + f with n rounded to nearest
+// by the 1.5*2^23 shifter, polynomial for 2^f, then n added to the exponent
+// field.  Takes load off the MUFU unit, which ex2.approx occupies.
+__device__ __forceinline__ float exp2_poly(float x) {
+    x = fmaxf(x, -126.f);
+    const float shifter = 12582912.f;              // 1.5 * 2^23
+    const float t = x + shifter;                   // n in the low mantissa bits
+    const float n = t - shifter;
+    const float f = x - n;                         // in [-1/2, 1/2]
+    float q = fmaf(kExp2C4, f, kExp2C3);
+    q = fmaf(q, f, kExp2C2);
+    q = fmaf(q, f, kExp2C1);
+    q = fmaf(q, f, kExp2C0);
+    const int ni = __float_as_int(t) - 0x4B400000;
+    return __int_as_float(__float_as_int(q) + (ni << 23));
+}
+
 // Two FP32 values -> packed 16-bit pair, `lo` in the low half.
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     uint32_t r;
@@ -86,20 +112,6 @@ __device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
 }
 __device__ __forceinline__ float bf16_lo(uint32_t u) { return __uint_as_float(u << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t u) { return __uint_as_float(u & 0xffff0000u); }
-
-// Warpgroup-uniform AND of a per-thread flag over named barrier `id`.
-__device__ __forceinline__ bool wg_all(uint32_t id, bool ok) {
-    uint32_t r;
-    asm volatile(
-        "{\n\t.reg .pred p, q;\n\t"
-        "setp.ne.u32 p, %1, 0;\n\t"
-        "bar.red.and.pred q, %2, 128, p;\n\t"
-        "selp.u32 %0, 1, 0, q;\n\t}"
-        : "=r"(r)
-        : "r"((uint32_t)ok), "r"(id)
-        : "memory");
-    return r != 0;
-}
 
 __device__ __forceinline__ int chunk_cols(int ks, int ke) {
     int n = ke - ks;
@@ -132,18 +144,19 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     if (tid == 0) {
         mbar_init(bar(B_SCHED_FULL + 0), 1);
         mbar_init(bar(B_SCHED_FULL + 1), 1);
-        mbar_init(bar(B_SCHED_EMPTY + 0), 3);
-        mbar_init(bar(B_SCHED_EMPTY + 1), 3);
+        // released by the MMA thread and by lane 0 of each of the 8 softmax warps
+        mbar_init(bar(B_SCHED_EMPTY + 0), 1 + 8);
+        mbar_init(bar(B_SCHED_EMPTY + 1), 1 + 8);
         for (int t = 0; t < 2; ++t) {
             mbar_init(bar(B_Q_FULL + t), 1);
-            mbar_init(bar(B_Q_READY + t), 1);
+            mbar_init(bar(B_Q_READY + t), 128);     // every softmax thread of tile t
             mbar_init(bar(B_Q_EMPTY + t), 1);
             mbar_init(bar(B_K_FULL + t), 1);
             mbar_init(bar(B_K_EMPTY + t), 1);
             mbar_init(bar(B_V_FULL + t), 1);
             mbar_init(bar(B_V_EMPTY + t), 1);
             mbar_init(bar(B_S_FULL + t), 1);
-            mbar_init(bar(B_P_FULL + t), 1);
+            mbar_init(bar(B_P_FULL + t), 128);      // every softmax thread of tile t
             mbar_init(bar(B_O_FULL + t), 1);
         }
         mbar_init(bar(B_DRAIN), 1);
@@ -355,7 +368,6 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         const int t = (warp - 4) >> 2;               // tile 0 or 1
         const int r = tid - 128 - 128 * t;           // row = TMEM lane, 0..127
         const int tl = r >> 3, hl = r & 7;           // token within tile, head within group
-        const uint32_t wg_bar = 1 + t;
         const uint32_t lane_base = (uint32_t)(warp & 3) * 32u;
         const uint32_t t_s = tmem + (lane_base << 16) + 128u * t;
         const uint32_t t_o = tmem + (lane_base << 16) + 256u + 128u * t;
@@ -367,10 +379,14 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         uint32_t sslot = 0, sph = 0, qph = 0, s_ph = 0, oph = 0;
         (void)q_tile;
         for (;;) {
-            bool ok = mbar_wait(bar(B_SCHED_FULL + sslot), sph, abort_flag, status);
-            int u = ok ? misc->sched[sslot] : -1;
-            if (!wg_all(wg_bar, ok)) break;
-            if (r == 0) mbar_arrive(bar(B_SCHED_EMPTY + sslot));
+            // Warps of the warpgroup run without block-level barriers; every
+            // wait's outcome is made warp-uniform (tcgen05.ld/st are
+            // .sync.aligned) and a warp that gives up simply leaves the loop.
+            bool ok = __all_sync(0xffffffffu, mbar_wait(bar(B_SCHED_FULL + sslot), sph, abort_flag, status));
+            if (!ok) break;
+            const int u = misc->sched[sslot];
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(B_SCHED_EMPTY + sslot));
             sslot ^= 1; if (sslot == 0) sph ^= 1;
             if (u < 0) break;
             const int4 it = items[u >> 2];
@@ -384,7 +400,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             const int kb = p.window > 0 ? max(ds, q0 - p.window + 1) : ds;
 
             // ---- rope table for this tile's 16 tokens: thread r fills token
-            // tl, pair indices 8*hl .. 8*hl+7
+            // tl, pair indices 8*hl .. 8*hl+7.  The 8 threads of a token are
+            // lanes of one warp, so a warp barrier publishes the entries.
+            __syncwarp();
             if (p.use_rope) {
                 int pos = 0;
                 const int tok = min(i, p.T - 1);
@@ -396,8 +414,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     rope_tab[tl * 64 + 8 * hl + e] = make_float2(c, s);
                 }
             }
-            ok = mbar_wait(bar(B_Q_FULL + t), qph, abort_flag, status);
-            if (!wg_all(wg_bar, ok)) break;   // also publishes the rope table
+            __syncwarp();
+            ok = __all_sync(0xffffffffu, mbar_wait(bar(B_Q_FULL + t), qph, abort_flag, status));
+            if (!ok) break;
             qph ^= 1;
 
             // ---- Q prologue, in place: RMSNorm (weight form), RoPE, x 2^eq, FP16.
@@ -451,8 +470,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 }
             }
             fence_proxy_async_smem();
-            named_bar_sync(wg_bar, 128);
-            if (r == 0) mbar_arrive(bar(B_Q_READY + t));
+            mbar_arrive(bar(B_Q_READY + t));
 
             // ---- online softmax over the key chunks
             const float sink = p.sinks[h];
@@ -464,8 +482,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 const int ks = kb + kKeyChunk * c;
                 const int nc = chunk_cols(ks, ke);
                 const int nblk = (nc + 31) >> 5;
-                ok = mbar_wait(bar(B_S_FULL + t), s_ph, abort_flag, status);
-                if (!wg_all(wg_bar, ok)) { alive = false; break; }
+                ok = __all_sync(0xffffffffu, mbar_wait(bar(B_S_FULL + t), s_ph, abort_flag, status));
+                if (!ok) { alive = false; break; }
                 s_ph ^= 1;
                 tc_fence_after();
                 // all S columns of this chunk: one TMEM load per 32 columns,
@@ -523,32 +541,53 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 float lp[8];
 #pragma unroll
                 for (int k8 = 0; k8 < 8; ++k8) lp[k8] = 0.f;
+                // Every fourth column of an unmasked chunk goes through the
+                // polynomial; masked chunks and infinite maxima keep ex2 so
+                // -inf maps to exactly 0.
+                const bool use_poly =
+                    __all_sync(0xffffffffu, !boundary && m > -INFINITY && m < INFINITY);
+                if (use_poly) {
 #pragma unroll
-                for (int b = 0; b < 4; ++b) {
-                    if (b < nblk) {
+                    for (int b = 0; b < 4; ++b) {
                         uint32_t pk[16];
 #pragma unroll
                         for (int j = 0; j < 16; ++j) {
-                            const float p0 = ex2(fmaf(__uint_as_float(sv[32 * b + 2 * j]), C, negm));
-                            const float p1 = ex2(fmaf(__uint_as_float(sv[32 * b + 2 * j + 1]), C, negm));
+                            const float x0 = fmaf(__uint_as_float(sv[32 * b + 2 * j]), C, negm);
+                            const float x1 = fmaf(__uint_as_float(sv[32 * b + 2 * j + 1]), C, negm);
+                            const float p0 = ex2(x0);
+                            const float p1 = (j & 1) ? exp2_poly(x1) : ex2(x1);
                             lp[j & 7] += p0 + p1;
                             pk[j] = pack_bf16(p0, p1);
                         }
                         tmem_st16(t_s + 16u * b, pk);
+                    }
+                } else {
+#pragma unroll
+                    for (int b = 0; b < 4; ++b) {
+                        if (b < nblk) {
+                            uint32_t pk[16];
+#pragma unroll
+                            for (int j = 0; j < 16; ++j) {
+                                const float p0 = ex2(fmaf(__uint_as_float(sv[32 * b + 2 * j]), C, negm));
+                                const float p1 = ex2(fmaf(__uint_as_float(sv[32 * b + 2 * j + 1]), C, negm));
+                                lp[j & 7] += p0 + p1;
+                                pk[j] = pack_bf16(p0, p1);
+                            }
+                            tmem_st16(t_s + 16u * b, pk);
+                        }
                     }
                 }
                 const float lsum = ((lp[0] + lp[1]) + (lp[2] + lp[3])) + ((lp[4] + lp[5]) + (lp[6] + lp[7]));
                 l += lsum;
                 tmem_wait_st();
                 tc_fence_before();
-                named_bar_sync(wg_bar, 128);
-                if (r == 0) mbar_arrive(bar(B_P_FULL + t));
+                mbar_arrive(bar(B_P_FULL + t));
             }
             if (!alive) break;
 
             // ---- epilogue: O / l -> BF16, LSE
-            ok = mbar_wait(bar(B_O_FULL + t), oph, abort_flag, status);
-            if (!wg_all(wg_bar, ok)) break;
+            ok = __all_sync(0xffffffffu, mbar_wait(bar(B_O_FULL + t), oph, abort_flag, status));
+            if (!ok) break;
             oph ^= 1;
             tc_fence_after();
             const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
