@@ -81,23 +81,64 @@ constexpr float kExp2C2 = 2.402474433e-01f;
 constexpr float kExp2C3 = 5.591785908e-02f;
 constexpr float kExp2C4 = 9.570101276e-03f;
 
-// 2^x on the FMA and integer pipes, for finite x <= 64 (results below 2^-126
-// flush towards 2^-126).  Cody-Waite split x = n + f with n rounded to nearest
-// by the 1.5*2^23 shifter, polynomial for 2^f, then n added to the exponent
-// field.  Takes load off the MUFU unit, which ex2.approx occupies.
-__device__ __forceinline__ float exp2_poly(float x) {
-    x = fmaxf(x, -126.f);
-    const float shifter = 12582912.f;              // 1.5 * 2^23
-    const float t = x + shifter;                   // n in the low mantissa bits
-    const float n = t - shifter;
-    const float f = x - n;                         // in [-1/2, 1/2]
-    float q = fmaf(kExp2C4, f, kExp2C3);
-    q = fmaf(q, f, kExp2C2);
-    q = fmaf(q, f, kExp2C1);
-    q = fmaf(q, f, kExp2C0);
-    const int ni = __float_as_int(t) - 0x4B400000;
-    return __int_as_float(__float_as_int(q) + (ni << 23));
+// Packed FP32 pairs (Blackwell f32x2 arithmetic): one instruction acts on both
+// halves of a 64-bit register.
+__device__ __forceinline__ uint64_t f2(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
 }
+__device__ __forceinline__ float f2_lo(uint64_t v) {
+    float lo, hi;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+    return lo;
+}
+__device__ __forceinline__ float f2_hi(uint64_t v) {
+    float lo, hi;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+    return hi;
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t r;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+    return r;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ float max3(float a, float b, float c) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
+// 2^x for a pair of finite x <= 64 on the FMA and integer pipes (results below
+// 2^-126 flush towards 2^-126).  Cody-Waite split x = n + f with n rounded to
+// nearest by the 1.5*2^23 shifter (the float t = x + shifter holds n in its
+// low mantissa bits), degree-4 polynomial for 2^f on [-1/2, 1/2], then n
+// added to the exponent field.  Because 0x4B400000 << 23 vanishes modulo 2^32,
+// adding (bits(t) << 23) adds n << 23.  Takes load off the MUFU unit.
+__device__ __forceinline__ uint64_t exp2_poly2(uint64_t x) {
+    x = f2(fmaxf(f2_lo(x), -126.f), fmaxf(f2_hi(x), -126.f));
+    const uint64_t sh = f2(12582912.f, 12582912.f);          // 1.5 * 2^23
+    const uint64_t nsh = f2(-12582912.f, -12582912.f);
+    const uint64_t neg1 = f2(-1.f, -1.f);
+    const uint64_t t = f2_add(x, sh);
+    const uint64_t n = f2_add(t, nsh);
+    const uint64_t f = f2_fma(n, neg1, x);                   // in [-1/2, 1/2]
+    uint64_t q = f2_fma(f2(kExp2C4, kExp2C4), f, f2(kExp2C3, kExp2C3));
+    q = f2_fma(q, f, f2(kExp2C2, kExp2C2));
+    q = f2_fma(q, f, f2(kExp2C1, kExp2C1));
+    q = f2_fma(q, f, f2(kExp2C0, kExp2C0));
+    const float p0 = __int_as_float(__float_as_int(f2_lo(q)) + (__float_as_int(f2_lo(t)) << 23));
+    const float p1 = __int_as_float(__float_as_int(f2_hi(q)) + (__float_as_int(f2_hi(t)) << 23));
+    return f2(p0, p1);
+}
+
+// Pairs j of each 16-pair block with (j % 8) < kPolyPairs take the polynomial.
+constexpr int kPolyPairs = 3;
 
 // Two FP32 values -> packed 16-bit pair, `lo` in the low half.
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
@@ -495,7 +536,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 tmem_wait_ld();
                 const bool boundary = (c == nch - 1) || (ks + nc - 1 > tok0) ||
                                       (p.window > 0 && ks < tok0 + kTokPerTile - p.window);
-                // row max over visible keys, 8 independent chains
+                // row max over visible keys: 3-input max, 8 independent chains
                 float mxp[8];
 #pragma unroll
                 for (int k8 = 0; k8 < 8; ++k8) mxp[k8] = -INFINITY;
@@ -505,20 +546,22 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     for (int b = 0; b < 4; ++b) {
                         if (b < nblk) {
 #pragma unroll
-                            for (int j = 32 * b; j < 32 * b + 32; ++j) {
-                                const bool vis = (j >= jlo) && (j <= jhi);
-                                const float x = vis ? __uint_as_float(sv[j]) : -INFINITY;
-                                sv[j] = __float_as_uint(x);
-                                mxp[j & 7] = fmaxf(mxp[j & 7], x);
+                            for (int j = 32 * b; j < 32 * b + 32; j += 2) {
+                                const float x0 = ((j >= jlo) && (j <= jhi)) ? __uint_as_float(sv[j]) : -INFINITY;
+                                const float x1 = ((j + 1 >= jlo) && (j + 1 <= jhi)) ? __uint_as_float(sv[j + 1]) : -INFINITY;
+                                sv[j] = __float_as_uint(x0);
+                                sv[j + 1] = __float_as_uint(x1);
+                                mxp[(j >> 1) & 7] = max3(mxp[(j >> 1) & 7], x0, x1);
                             }
                         }
                     }
                 } else {
 #pragma unroll
-                    for (int j = 0; j < 128; ++j) mxp[j & 7] = fmaxf(mxp[j & 7], __uint_as_float(sv[j]));
+                    for (int j = 0; j < 128; j += 2)
+                        mxp[(j >> 1) & 7] = max3(mxp[(j >> 1) & 7], __uint_as_float(sv[j]), __uint_as_float(sv[j + 1]));
                 }
-                const float mx = fmaxf(fmaxf(fmaxf(mxp[0], mxp[1]), fmaxf(mxp[2], mxp[3])),
-                                       fmaxf(fmaxf(mxp[4], mxp[5]), fmaxf(mxp[6], mxp[7])));
+                const float mx = max3(max3(mxp[0], mxp[1], mxp[2]), max3(mxp[3], mxp[4], mxp[5]),
+                                      fmaxf(mxp[6], mxp[7]));
                 const float m_new = fmaxf(m, mx * C);
                 float m_use = m;
                 if (c == 0 ? (m_new > m) : (m_new > m + 8.f)) m_use = m_new;
@@ -538,10 +581,11 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 }
                 m = m_use;
                 const float negm = (m == -INFINITY) ? 0.f : -m;
-                float lp[8];
+                const uint64_t C2 = f2(C, C), negm2 = f2(negm, negm);
+                uint64_t lp[4];
 #pragma unroll
-                for (int k8 = 0; k8 < 8; ++k8) lp[k8] = 0.f;
-                // Every fourth column of an unmasked chunk goes through the
+                for (int k4 = 0; k4 < 4; ++k4) lp[k4] = 0ull;   // (+0.0f, +0.0f)
+                // Part of the pairs of an unmasked chunk go through the
                 // polynomial; masked chunks and infinite maxima keep ex2 so
                 // -inf maps to exactly 0.
                 const bool use_poly =
@@ -552,12 +596,13 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                         uint32_t pk[16];
 #pragma unroll
                         for (int j = 0; j < 16; ++j) {
-                            const float x0 = fmaf(__uint_as_float(sv[32 * b + 2 * j]), C, negm);
-                            const float x1 = fmaf(__uint_as_float(sv[32 * b + 2 * j + 1]), C, negm);
-                            const float p0 = ex2(x0);
-                            const float p1 = (j & 1) ? exp2_poly(x1) : ex2(x1);
-                            lp[j & 7] += p0 + p1;
-                            pk[j] = pack_bf16(p0, p1);
+                            const uint64_t x = f2_fma(f2(__uint_as_float(sv[32 * b + 2 * j]),
+                                                         __uint_as_float(sv[32 * b + 2 * j + 1])), C2, negm2);
+                            uint64_t pp;
+                            if ((j & 7) < kPolyPairs) pp = exp2_poly2(x);
+                            else pp = f2(ex2(f2_lo(x)), ex2(f2_hi(x)));
+                            lp[j & 3] = f2_add(lp[j & 3], pp);
+                            pk[j] = pack_bf16(f2_lo(pp), f2_hi(pp));
                         }
                         tmem_st16(t_s + 16u * b, pk);
                     }
@@ -568,16 +613,18 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                             uint32_t pk[16];
 #pragma unroll
                             for (int j = 0; j < 16; ++j) {
-                                const float p0 = ex2(fmaf(__uint_as_float(sv[32 * b + 2 * j]), C, negm));
-                                const float p1 = ex2(fmaf(__uint_as_float(sv[32 * b + 2 * j + 1]), C, negm));
-                                lp[j & 7] += p0 + p1;
-                                pk[j] = pack_bf16(p0, p1);
+                                const uint64_t x = f2_fma(f2(__uint_as_float(sv[32 * b + 2 * j]),
+                                                             __uint_as_float(sv[32 * b + 2 * j + 1])), C2, negm2);
+                                const uint64_t pp = f2(ex2(f2_lo(x)), ex2(f2_hi(x)));
+                                lp[j & 3] = f2_add(lp[j & 3], pp);
+                                pk[j] = pack_bf16(f2_lo(pp), f2_hi(pp));
                             }
                             tmem_st16(t_s + 16u * b, pk);
                         }
                     }
                 }
-                const float lsum = ((lp[0] + lp[1]) + (lp[2] + lp[3])) + ((lp[4] + lp[5]) + (lp[6] + lp[7]));
+                const uint64_t ls = f2_add(f2_add(lp[0], lp[1]), f2_add(lp[2], lp[3]));
+                const float lsum = f2_lo(ls) + f2_hi(ls);
                 l += lsum;
                 tmem_wait_st();
                 tc_fence_before();

@@ -40,9 +40,14 @@ def exp2_poly(x, c):
     q = fma32(q, f, c[2])
     q = fma32(q, f, c[1])
     q = fma32(q, f, c[0])
+    # the kernel adds bits(t) << 23 modulo 2^32, which equals n << 23 because
+    # 0x4B400000 << 23 vanishes modulo 2^32
+    tb = t.view(np.uint32).astype(np.uint64)
+    bits = (q.view(np.uint32).astype(np.uint64) + (tb << np.uint64(23))) & np.uint64(0xFFFFFFFF)
     ni = t.view(np.int32).astype(np.int64) - 0x4B400000
-    bits = q.view(np.int32).astype(np.int64) + (ni << 23)
-    return bits.astype(np.int32).view(np.float32)
+    ref_bits = (q.view(np.int32).astype(np.int64) + (ni << 23)) & 0xFFFFFFFF
+    assert np.array_equal(bits.astype(np.int64), ref_bits)
+    return bits.astype(np.uint32).view(np.float32)
 
 
 def test_relative_error_bound():
