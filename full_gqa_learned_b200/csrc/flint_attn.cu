@@ -304,29 +304,36 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         // ============================================================ MMA issuer
         if (lane == 0) {
             const uint32_t idesc_pv = idesc_f16(1, 1, 1, 128);
-            // Base descriptors; the start-address field (bits 0..13, in 16-byte
-            // units) is advanced by adding the byte offset >> 4, which stays
-            // inside the field for every offset used below.
+            // Descriptor words.  Only the low word (start address) changes
+            // between MMAs; the issuing thread shares its scheduler with two
+            // busy softmax warps, so each MMA is kept to a 32-bit add and the
+            // instruction itself.
             const uint64_t dq0 = smem_desc_sw128(sbase + kOffQ, 16, 1024);
             const uint64_t dk0 = smem_desc_sw128(sbase + kOffK, 16, 1024);
             const uint64_t dv0 = smem_desc_sw128(sbase + kOffV, kHalfTile, 1024);
-            constexpr uint64_t kTileStep = kTileBytes >> 4;
+            const uint32_t q_lo = (uint32_t)dq0, q_hi = (uint32_t)(dq0 >> 32);
+            const uint32_t k_lo = (uint32_t)dk0, k_hi = (uint32_t)(dk0 >> 32);
+            const uint32_t v_lo = (uint32_t)dv0, v_hi = (uint32_t)(dv0 >> 32);
+            constexpr uint32_t kTileStep = kTileBytes >> 4;
             uint32_t sslot = 0, sph = 0, qrph = 0, kst = 0, kph = 0, vst = 0, vph = 0, pph = 0;
-            auto issue_s = [=](uint32_t t, uint32_t kstage, int ncols) {
+            auto issue_s = [&](uint32_t t, uint32_t kstage, int ncols) {
                 const uint32_t idesc = idesc_f16(0, 0, 0, (uint32_t)ncols);
-                const uint64_t dq = dq0 + t * kTileStep, dk = dk0 + kstage * kTileStep;
+                const uint32_t qa = q_lo + t * kTileStep, kb_ = k_lo + kstage * kTileStep;
+                const uint32_t d = tmem + 128u * t;
 #pragma unroll
                 for (uint32_t kk = 0; kk < kHD / 16; ++kk) {
-                    const uint64_t off = (kk >> 2) * (kHalfTile >> 4) + (kk & 3) * 2;
-                    mma_ss(tmem + 128u * t, dq + off, dk + off, idesc, kk > 0);
+                    const uint32_t off = (kk >> 2) * (kHalfTile >> 4) + (kk & 3) * 2;
+                    mma_ss_w(d, qa + off, q_hi, kb_ + off, k_hi, idesc, kk > 0 ? 1u : 0u);
                 }
             };
-            auto issue_pv = [=](uint32_t t, uint32_t vstage, int ncols, bool acc) {
-                const uint64_t dv = dv0 + vstage * kTileStep;
+            auto issue_pv = [&](uint32_t t, uint32_t vstage, int ncols, bool acc) {
+                const uint32_t vb = v_lo + vstage * kTileStep;
+                const uint32_t d = tmem + 256u + 128u * t, pa = tmem + 128u * t;
                 const int nk = ncols >> 4;
-                for (int kk = 0; kk < nk; ++kk)
-                    mma_ts(tmem + 256u + 128u * t, tmem + 128u * t + 8u * kk,
-                           dv + (uint64_t)kk * (2048 >> 4), idesc_pv, (acc || kk > 0) ? 1u : 0u);
+                mma_ts_w(d, pa, vb, v_hi, idesc_pv, acc ? 1u : 0u);
+#pragma unroll
+                for (int kk = 1; kk < 8; ++kk)
+                    if (kk < nk) mma_ts_w(d, pa + 8u * kk, vb + kk * (2048 >> 4), v_hi, idesc_pv, 1u);
             };
             for (;;) {
                 if (!mbar_wait(bar(B_SCHED_FULL + sslot), sph, abort_flag, status)) break;
