@@ -20,6 +20,7 @@ __global__ void attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q,
                                 const __grid_constant__ CUtensorMap tm_k,
                                 const __grid_constant__ CUtensorMap tm_v, const AttnParams p);
 extern const unsigned kAttnSmemBytes;
+extern const unsigned kAttnThreads;
 }  // namespace flint
 
 using namespace flint;
@@ -245,7 +246,7 @@ flint_status_t run(int stages, const void* q, const void* k, const void* v, cons
     ap.eps = eps;
     const int max_units = L.max_items * kHKV;
     const int grid = max_units < sms ? max_units : sms;
-    attn_fwd_kernel<<<grid, 384, kAttnSmemBytes, s>>>(tm_q, tm_k, tm_v, ap);
+    attn_fwd_kernel<<<grid, kAttnThreads, kAttnSmemBytes, s>>>(tm_q, tm_k, tm_v, ap);
     e = cudaGetLastError();
     if (e != cudaSuccess) return fail(FLINT_ERR_CUDA, "attention launch: %s", cudaGetErrorString(e));
     return FLINT_OK;

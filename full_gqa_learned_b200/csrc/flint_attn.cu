@@ -15,8 +15,10 @@
 //   warp 1      TMEM owner; lane 0 issues every tcgen05.mma and commit
 //   warp 2      TMA producer of V chunks
 //   warp 3      TMA producer of raw Q tiles
-//   warps 4-7   softmax warpgroup (one thread per row)
-//   warps 8-11  tile warpgroup: Q prologue of the next item, epilogue of the
+//   warps 4-7   softmax warpgroup A: columns 0-63 of every S chunk
+//   warps 8-11  softmax warpgroup B: columns 64-127 (same rows; the two
+//               exchange row maxima once per chunk)
+//   warps 12-15 tile warpgroup: Q prologue of the next item, epilogue of the
 //               previous one
 // A work item is one tile of 128 MMA rows = 16 tokens x the 8 query heads of
 // one KV group, so every K/V chunk in shared memory serves 8 heads.
@@ -37,14 +39,14 @@
 
 namespace flint {
 
-constexpr int kThreads = 384;
-// Registers: launched with 384 x 168 = 64512; the control warpgroup drops to
-// 72, the softmax warpgroup rises to 232, the tile warpgroup drops to 160:
-// 128 * (72 + 232 + 160) = 59392.
-constexpr uint32_t kRegsControl = 72;
-constexpr uint32_t kRegsSoftmax = 232;
-constexpr uint32_t kRegsTile = 160;
-static_assert(128 * (kRegsControl + kRegsSoftmax + kRegsTile) <= 384 * 168, "register split");
+constexpr int kThreads = 512;
+// Registers: launched with 512 x 128 = 65536; the control warpgroup drops to
+// 64, the two softmax warpgroups rise to 160, the tile warpgroup stays at
+// 128: 128 * (64 + 2 * 160 + 128) = 65536.
+constexpr uint32_t kRegsControl = 64;
+constexpr uint32_t kRegsSoftmax = 160;
+constexpr uint32_t kRegsTile = 128;
+static_assert(128 * (kRegsControl + 2 * kRegsSoftmax + kRegsTile) <= 512 * 128, "register split");
 
 constexpr uint32_t kTileBytes = 128 * kHD * 2;       // 32 KiB: 128 rows x 128 x 16-bit
 constexpr uint32_t kHalfTile = kTileBytes / 2;       // one 64-column swizzled half
@@ -58,8 +60,9 @@ constexpr uint32_t kOffK = kOffQraw + kTileBytes;                  // K stages (
 constexpr uint32_t kOffV = kOffK + kKStages * kTileBytes;          // V stages (BF16)
 constexpr uint32_t kOffRope = kOffV + kVStages * kTileBytes;       // [16][64] float2
 constexpr uint32_t kRopeBytes = kTokPerTile * 64 * 8;
-constexpr uint32_t kOffStats = kOffRope + kRopeBytes;              // [2][128] float2 (m, l)
-constexpr uint32_t kOffW = kOffStats + 2 * 128 * 8;                // q_norm_w [128] f32
+constexpr uint32_t kOffStats = kOffRope + kRopeBytes;              // [2][128] float4 (m, lA, lB)
+constexpr uint32_t kOffPmax = kOffStats + 2 * 128 * 16;            // [2][2][128] f32 partial maxima
+constexpr uint32_t kOffW = kOffPmax + 2 * 2 * 128 * 4;             // q_norm_w [128] f32
 constexpr uint32_t kOffInv = kOffW + kHD * 4;                      // inv_freq [64] f64
 constexpr uint32_t kOffBar = kOffInv + 64 * 8;                     // mbarriers
 constexpr uint32_t kNumBars = 40;
@@ -190,6 +193,21 @@ __device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
 __device__ __forceinline__ float bf16_lo(uint32_t u) { return __uint_as_float(u << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t u) { return __uint_as_float(u & 0xffff0000u); }
 
+// AND of a per-thread flag over the `count` threads of named barrier `id`;
+// also orders their shared-memory accesses.
+__device__ __forceinline__ bool block_and(uint32_t id, uint32_t count, bool ok) {
+    uint32_t res;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "bar.red.and.pred q, %2, %3, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(res)
+        : "r"((uint32_t)ok), "r"(id), "r"(count)
+        : "memory");
+    return res != 0;
+}
+
 __device__ __forceinline__ int chunk_cols(int ks, int ke) {
     int n = ke - ks;
     n = n > kKeyChunk ? kKeyChunk : n;
@@ -233,7 +251,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     Misc* misc = reinterpret_cast<Misc*>(smem + kOffMisc);
     float* s_wq = reinterpret_cast<float*>(smem + kOffW);
     double* s_inv = reinterpret_cast<double*>(smem + kOffInv);
-    float2* s_stats = reinterpret_cast<float2*>(smem + kOffStats);
+    float4* s_stats = reinterpret_cast<float4*>(smem + kOffStats);
+    float* s_pmax = reinterpret_cast<float*>(smem + kOffPmax);
     int4* s_fifo = reinterpret_cast<int4*>(smem + kOffFifo);
     volatile int* abort_flag = &misc->abort_flag;
 
@@ -248,8 +267,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     if (tid == 0) {
         for (int s = 0; s < kSchedSlots; ++s) {
             mbar_init(bar(B_SCHED_FULL + s), 1);
-            // MMA thread, Q and V producers, lane 0 of the 4 softmax and 4 tile warps
-            mbar_init(bar(B_SCHED_EMPTY + s), 1 + 2 + 4 + 4);
+            // MMA thread, Q and V producers, lane 0 of the 8 softmax and 4 tile warps
+            mbar_init(bar(B_SCHED_EMPTY + s), 1 + 2 + 8 + 4);
         }
         mbar_init(bar(B_QRAW_FULL), 1);
         mbar_init(bar(B_QRAW_EMPTY), 4);
@@ -257,9 +276,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             mbar_init(bar(B_Q_READY + b), 128);
             mbar_init(bar(B_Q_FREE + b), 1);
             mbar_init(bar(B_S_FULL + b), 1);
-            mbar_init(bar(B_P_FULL + b), 128);
+            mbar_init(bar(B_P_FULL + b), 256);
             mbar_init(bar(B_PV_DONE + b), 1);
-            mbar_init(bar(B_STATS_FULL + b), 128);
+            mbar_init(bar(B_STATS_FULL + b), 256);
             mbar_init(bar(B_STATS_EMPTY + b), 128);
         }
         for (int s = 0; s < kKStages; ++s) {
@@ -509,21 +528,30 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             mbar_wait(bar(B_DRAIN), 0, &never, nullptr, 100ull * 1000ull * 1000ull);
         }
       }
-    } else if (warp < 8) {
+    } else if (warp < 12) {
         regs_inc<kRegsSoftmax>();
         // ============================================================ softmax
-        const int r = tid - 128;                     // row = TMEM lane, 0..127
+        // Two warpgroups share every row: w = 0 takes columns 0-63 of each S
+        // chunk, w = 1 columns 64-127.  Their partial row maxima meet in
+        // shared memory behind one 256-thread barrier per chunk, which also
+        // makes every abort decision common to both.
+        const int w = (warp - 4) >> 2;               // column half
+        const int r = (tid - 128) & 127;             // row = TMEM lane, 0..127
         const int tl = r >> 3, hl = r & 7;           // token within tile, head within group
         const uint32_t lane_base = (uint32_t)(warp & 3) * 32u;
         const uint32_t t_row = tmem + (lane_base << 16);
-        const uint32_t t_o = t_row + kTmemO;
+        const uint32_t t_o = t_row + kTmemO + 64u * w;     // this half's O columns
         const float C = misc->logit_scale;
         SchedCursor sc;
         uint32_t gchunk = 0, n = 0;
+        // `good` is warp-uniform; every exit goes through a 256-thread AND so
+        // both warpgroups leave together and no named barrier is left waiting.
+        bool good = true;
         for (;;) {
             bool ok = __all_sync(0xffffffffu, mbar_wait(bar(B_SCHED_FULL + sc.slot), sc.phase, abort_flag, status));
-            if (!ok) break;
-            const int u = misc->sched[sc.slot];
+            const int u = ok ? misc->sched[sc.slot] : -1;
+            good = block_and(1, 256, good && ok);
+            if (!good) break;
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(B_SCHED_EMPTY + sc.slot));
             sc.advance();
@@ -533,65 +561,69 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             const int i = it.q0 + tl;
             const float sink = p.sinks[h];
             float m = sink * 1.4426950408889634f;      // log2 domain
-            float l = (sink == -INFINITY) ? 0.f : 1.f;
+            float l = (w == 0 && sink != -INFINITY) ? 1.f : 0.f;   // the sink column counts once
             const int lo = p.window > 0 ? i - p.window + 1 : -(1 << 30);
-            bool alive = true;
             for (int c = 0; c < it.nch; ++c, ++gchunk) {
                 const int ks = it.kb + kKeyChunk * c;
                 const int nc = chunk_cols(ks, it.ke);
-                const int nblk = (nc + 31) >> 5;
+                const int mycols = min(max(nc - 64 * w, 0), 64);
+                const int nblk = (mycols + 31) >> 5;   // 0, 1 or 2 blocks of 32 columns
                 const uint32_t b = gchunk & 1;
                 const uint32_t t_s = t_row + kTmemS + 128u * b;
                 ok = __all_sync(0xffffffffu, mbar_wait(bar(B_S_FULL + b), (gchunk >> 1) & 1, abort_flag, status));
-                if (!ok) { alive = false; break; }
-                tc_fence_after();
-                uint32_t sv[128];
-#pragma unroll
-                for (int bb = 0; bb < 4; ++bb)
-                    if (bb < nblk) tmem_ld32(t_s + 32u * bb, sv + 32 * bb);
-                tmem_wait_ld();
+                ok = ok && good;
                 const bool boundary = (c == it.nch - 1) || (ks + nc - 1 > it.q0) ||
                                       (p.window > 0 && ks < it.q0 + kTokPerTile - p.window);
-                // row max over visible keys: 3-input max, 8 independent chains
-                float mxp[8];
+                uint32_t sv[64];
+                float mxp[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+                if (ok) {
+                    tc_fence_after();
 #pragma unroll
-                for (int k8 = 0; k8 < 8; ++k8) mxp[k8] = -INFINITY;
-                if (boundary) {
-                    const int jlo = lo - ks, jhi = i - ks;
+                    for (int bb = 0; bb < 2; ++bb)
+                        if (bb < nblk) tmem_ld32(t_s + 64u * w + 32u * bb, sv + 32 * bb);
+                    tmem_wait_ld();
+                    if (boundary) {
+                        const int jlo = lo - ks - 64 * w, jhi = i - ks - 64 * w;
 #pragma unroll
-                    for (int bb = 0; bb < 4; ++bb) {
-                        if (bb < nblk) {
+                        for (int bb = 0; bb < 2; ++bb) {
+                            if (bb < nblk) {
 #pragma unroll
-                            for (int j = 32 * bb; j < 32 * bb + 32; j += 2) {
-                                const float x0 = ((j >= jlo) && (j <= jhi)) ? __uint_as_float(sv[j]) : -INFINITY;
-                                const float x1 = ((j + 1 >= jlo) && (j + 1 <= jhi)) ? __uint_as_float(sv[j + 1]) : -INFINITY;
-                                sv[j] = __float_as_uint(x0);
-                                sv[j + 1] = __float_as_uint(x1);
-                                mxp[(j >> 1) & 7] = max3(mxp[(j >> 1) & 7], x0, x1);
+                                for (int j = 32 * bb; j < 32 * bb + 32; j += 2) {
+                                    const float x0 = ((j >= jlo) && (j <= jhi)) ? __uint_as_float(sv[j]) : -INFINITY;
+                                    const float x1 = ((j + 1 >= jlo) && (j + 1 <= jhi)) ? __uint_as_float(sv[j + 1]) : -INFINITY;
+                                    sv[j] = __float_as_uint(x0);
+                                    sv[j + 1] = __float_as_uint(x1);
+                                    mxp[(j >> 1) & 3] = max3(mxp[(j >> 1) & 3], x0, x1);
+                                }
                             }
                         }
-                    }
-                } else {
+                    } else {
 #pragma unroll
-                    for (int j = 0; j < 128; j += 2)
-                        mxp[(j >> 1) & 7] = max3(mxp[(j >> 1) & 7], __uint_as_float(sv[j]), __uint_as_float(sv[j + 1]));
+                        for (int j = 0; j < 64; j += 2)
+                            mxp[(j >> 1) & 3] = max3(mxp[(j >> 1) & 3], __uint_as_float(sv[j]), __uint_as_float(sv[j + 1]));
+                    }
                 }
-                const float mx = max3(max3(mxp[0], mxp[1], mxp[2]), max3(mxp[3], mxp[4], mxp[5]),
-                                      fmaxf(mxp[6], mxp[7]));
+                const float pm = fmaxf(max3(mxp[0], mxp[1], mxp[2]), mxp[3]);
+                float* px = s_pmax + (b * 2) * 128;
+                px[w * 128 + r] = pm;
+                good = block_and(1, 256, ok);
+                if (!good) break;
+                const float mx = fmaxf(pm, px[(1 - w) * 128 + r]);
+                // both halves take the same decisions from the same maxima
                 const float m_new = fmaxf(m, mx * C);
                 float m_use = m;
                 if (c == 0 ? (m_new > m) : (m_new > m + 8.f)) m_use = m_new;
                 const float alpha = (m_use == m) ? 1.f : ex2(m - m_use);
                 l *= alpha;
-                // rescale O in TMEM once the previous chunk's PV has landed
-                // (warp-uniform: tcgen05.ld/st are .sync.aligned)
+                // rescale this half of O in TMEM once the previous chunk's PV
+                // has landed (warp-uniform: tcgen05.ld/st are .sync.aligned)
                 if (c > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
                     const uint32_t pg = gchunk - 1;
-                    ok = __all_sync(0xffffffffu, mbar_wait(bar(B_PV_DONE + (pg & 1)), (pg >> 1) & 1, abort_flag, status));
-                    if (!ok) { alive = false; break; }
+                    good = __all_sync(0xffffffffu, mbar_wait(bar(B_PV_DONE + (pg & 1)), (pg >> 1) & 1, abort_flag, status));
+                    if (!good) continue;     // leaves at the next 256-thread AND
                     tc_fence_after();
 #pragma unroll 1
-                    for (int bb = 0; bb < 8; ++bb) {
+                    for (int bb = 0; bb < 4; ++bb) {
                         uint32_t v[16];
                         tmem_ld16(t_o + 16u * bb, v);
                         tmem_wait_ld();
@@ -608,12 +640,13 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 for (int k4 = 0; k4 < 4; ++k4) lp[k4] = 0ull;   // (+0.0f, +0.0f)
                 // Part of the pairs of an unmasked chunk go through the
                 // polynomial; masked chunks and infinite maxima keep ex2 so
-                // -inf maps to exactly 0.
+                // -inf maps to exactly 0.  P of key k goes to column k/2.
+                const uint32_t t_p = t_s + 32u * w;
                 const bool use_poly =
                     __all_sync(0xffffffffu, !boundary && m > -INFINITY && m < INFINITY);
                 if (use_poly) {
 #pragma unroll
-                    for (int bb = 0; bb < 4; ++bb) {
+                    for (int bb = 0; bb < 2; ++bb) {
                         uint32_t pk[16];
 #pragma unroll
                         for (int j = 0; j < 16; ++j) {
@@ -625,11 +658,11 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                             lp[j & 3] = f2_add(lp[j & 3], pp);
                             pk[j] = pack_bf16(f2_lo(pp), f2_hi(pp));
                         }
-                        tmem_st16(t_s + 16u * bb, pk);
+                        tmem_st16(t_p + 16u * bb, pk);
                     }
                 } else {
 #pragma unroll
-                    for (int bb = 0; bb < 4; ++bb) {
+                    for (int bb = 0; bb < 2; ++bb) {
                         if (bb < nblk) {
                             uint32_t pk[16];
 #pragma unroll
@@ -640,7 +673,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                                 lp[j & 3] = f2_add(lp[j & 3], pp);
                                 pk[j] = pack_bf16(f2_lo(pp), f2_hi(pp));
                             }
-                            tmem_st16(t_s + 16u * bb, pk);
+                            tmem_st16(t_p + 16u * bb, pk);
                         }
                     }
                 }
@@ -650,11 +683,13 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 tc_fence_before();
                 mbar_arrive(bar(B_P_FULL + b));
             }
-            if (!alive) break;
-            // final (m, l) of this item's rows for the epilogue
-            ok = __all_sync(0xffffffffu, mbar_wait(bar(B_STATS_EMPTY + (n & 1)), ((n >> 1) & 1) ^ 1, abort_flag, status));
-            if (!ok) break;
-            s_stats[(n & 1) * 128 + r] = make_float2(m, l);
+            good = block_and(1, 256, good);
+            if (!good) break;
+            // final (m, partial l) of this item's rows for the epilogue
+            good = __all_sync(0xffffffffu, mbar_wait(bar(B_STATS_EMPTY + (n & 1)), ((n >> 1) & 1) ^ 1, abort_flag, status));
+            if (!good) continue;             // leaves at the next 256-thread AND
+            float* st = reinterpret_cast<float*>(s_stats + (n & 1) * 128 + r);
+            if (w == 0) { st[0] = m; st[1] = l; } else { st[2] = l; }
             mbar_arrive(bar(B_STATS_FULL + (n & 1)));
             ++n;
         }
@@ -662,7 +697,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         regs_dec<kRegsTile>();
         // ============================================================ tile warpgroup:
         // Q prologue of the next item, epilogue of the previous one
-        const int r = tid - 256;                     // row = TMEM lane, 0..127
+        const int r = tid - 384;                     // row = TMEM lane, 0..127
         const int tl = r >> 3, hl = r & 7;
         const uint32_t lane_base = (uint32_t)(warp & 3) * 32u;
         const uint32_t t_row = tmem + (lane_base << 16);
@@ -678,9 +713,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             tc_fence_after();
             ok = __all_sync(0xffffffffu, mbar_wait(bar(B_STATS_FULL + (j & 1)), (j >> 1) & 1, abort_flag, status));
             if (!ok) return false;
-            const float2 st = s_stats[(j & 1) * 128 + r];
+            const float4 st = s_stats[(j & 1) * 128 + r];
             mbar_arrive(bar(B_STATS_EMPTY + (j & 1)));
-            const float m = st.x, l = st.y;
+            const float m = st.x, l = st.y + st.z;
             const int i = e.x + tl;
             const int h = kGroup * e.z + hl;
             const bool row_valid = tl < e.y;
@@ -822,5 +857,6 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 }
 
 extern const unsigned kAttnSmemBytes = kSmemBytes;
+extern const unsigned kAttnThreads = kThreads;
 
 }  // namespace flint
