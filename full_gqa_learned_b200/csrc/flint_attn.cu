@@ -177,7 +177,10 @@ __device__ __forceinline__ uint64_t exp2_poly2(uint64_t x) {
 }
 
 // Pairs j of each 16-pair block with (j % 8) < kPolyPairs take the polynomial.
-constexpr int kPolyPairs = 3;
+// Measured costs per warp instruction and scheduler on B200: ex2 8 cycles,
+// fma/add.f32x2 2, cvt.rn.bf16x2.f32 ~4.5; the polynomial pair costs ~20 on
+// the FMA/ALU pipes, so MUFU and the FMA/ALU pipes balance near 1/8.
+constexpr int kPolyPairs = 1;
 
 // Two FP32 values -> packed 16-bit pair, `lo` in the low half.
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
@@ -611,13 +614,15 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 const float mx = fmaxf(pm, px[(1 - w) * 128 + r]);
                 // both halves take the same decisions from the same maxima
                 const float m_new = fmaxf(m, mx * C);
-                float m_use = m;
-                if (c == 0 ? (m_new > m) : (m_new > m + 8.f)) m_use = m_new;
-                const float alpha = (m_use == m) ? 1.f : ex2(m - m_use);
-                l *= alpha;
+                const bool raise = (c == 0) ? (m_new > m) : (m_new > m + 8.f);
+                float alpha = 1.f;
+                if (raise) {
+                    alpha = ex2(m - m_new);
+                    l *= alpha;
+                }
                 // rescale this half of O in TMEM once the previous chunk's PV
                 // has landed (warp-uniform: tcgen05.ld/st are .sync.aligned)
-                if (c > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+                if (c > 0 && __any_sync(0xffffffffu, raise)) {
                     const uint32_t pg = gchunk - 1;
                     good = __all_sync(0xffffffffu, mbar_wait(bar(B_PV_DONE + (pg & 1)), (pg >> 1) & 1, abort_flag, status));
                     if (!good) continue;     // leaves at the next 256-thread AND
@@ -632,7 +637,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                         tmem_st16(t_o + 16u * bb, v);
                     }
                 }
-                m = m_use;
+                if (raise) m = m_new;
                 const float negm = (m == -INFINITY) ? 0.f : -m;
                 const uint64_t C2 = f2(C, C), negm2 = f2(negm, negm);
                 uint64_t lp[4];
