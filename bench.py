@@ -69,6 +69,25 @@ def row_flops(w, rows):
     return 4.0 * 128 * 32 * float(n.sum())
 
 
+def max_over_ranks(values, device=None):
+    """Element-wise maximum of per-rank timings (ms) across all ranks of the
+    default process group (any backend); identity on a single process."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64,
+                     device=device if device is not None else "cpu")
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.cpu()]
+
+
+def whole_job_tflops(flops_per_rank_step, steps, world, max_total_ms):
+    """Throughput of the whole job: every rank processes its own replica, so
+    the units done are world x steps x flops per step, over the slowest
+    rank's time."""
+    return world * flops_per_rank_step * steps / (max_total_ms * 1e-3) / 1e12
+
+
 # ---------------------------------------------------------------- clocks
 
 class ClockSampler:
@@ -248,10 +267,7 @@ def run_flint(args, rank, world, local_rank):
     e2e_ms /= e2e_steps
 
     # max over ranks
-    vals = torch.tensor([total_ms, attn_avg, e2e_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
-    total_ms, attn_avg, e2e_ms = [float(x) for x in vals.cpu()]
+    total_ms, attn_avg, e2e_ms = max_over_ranks([total_ms, attn_avg, e2e_ms], device=dev)
     return dict(w=w, total_ms=total_ms, attn_avg=attn_avg, prep_avg=sum(prep_ms) / len(prep_ms),
                 e2e_ms=e2e_ms, h2d=h2d, d2h=d2h, clocks=clocks, launches=2 * args.steps)
 
@@ -336,7 +352,7 @@ def main():
     w = r["w"]
     peaks, src = load_peaks()
     flops = w.flops()
-    value = world * flops * args.steps / (r["total_ms"] * 1e-3) / 1e12
+    value = whole_job_tflops(flops, args.steps, world, r["total_ms"])
     attn_tflops = flops / (r["attn_avg"] * 1e-3) / 1e12
     peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     line = dict(
@@ -353,7 +369,7 @@ def main():
                       kernel="flint::attn_fwd_kernel", peak_source="%s bf16_tflops (burst)" % src,
                       flops_per_launch=flops,
                       kernel_ms=round(r["attn_avg"], 5), prep_kernel_ms=round(r["prep_avg"], 5)),
-        e2e=dict(value=round(world * flops / (r["e2e_ms"] * 1e-3) / 1e12, 3), unit=UNIT,
+        e2e=dict(value=round(whole_job_tflops(flops, 1, world, r["e2e_ms"]), 3), unit=UNIT,
                  h2d_bytes_per_step=r["h2d"], d2h_bytes_per_step=r["d2h"],
                  ms_per_step=round(r["e2e_ms"], 4)),
         gpu_launches=r["launches"], clocks=r["clocks"],
