@@ -16,12 +16,13 @@ import os
 import threading
 from typing import Optional, Tuple
 
-__all__ = ["attn_fwd", "workspace_bytes", "device_status", "load_library", "FlintError",
-           "LIB_PATH", "HQ", "HKV", "HEAD_DIM", "STATUS"]
+__all__ = ["attn_fwd", "attn_fwd_static", "workspace_bytes", "device_status", "load_library",
+           "FlintError", "LIB_PATH", "HQ", "HKV", "HEAD_DIM", "STATUS", "STATIC_SCRATCH_BYTES"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libflint_attn.so")
 HQ, HKV, HEAD_DIM = 32, 4, 128
+STATIC_SCRATCH_BYTES = 16 << 20     # FLINT_STATIC_SCRATCH_BYTES
 STATUS = {0: "FLINT_OK", 1: "FLINT_ERR_INVALID_ARG", 2: "FLINT_ERR_UNSUPPORTED",
           3: "FLINT_ERR_CUDA", 4: "FLINT_ERR_TIMEOUT", 5: "FLINT_ERR_WORKSPACE"}
 
@@ -55,6 +56,8 @@ def load_library() -> ctypes.CDLL:
         for name in ("flint_attn_fwd", "flint_attn_prepare", "flint_attn_attend"):
             getattr(lib, name).restype = ctypes.c_int
             getattr(lib, name).argtypes = fwd_args
+        lib.flint_attn_fwd_static.restype = ctypes.c_int
+        lib.flint_attn_fwd_static.argtypes = fwd_args[:19] + [P]
         lib.flint_attn_device_status.restype = ctypes.c_int
         lib.flint_attn_device_status.argtypes = [P, P]
         lib.flint_attn_last_error.restype = ctypes.c_char_p
@@ -162,3 +165,46 @@ def device_status(workspace, stream=None) -> int:
         stream = torch.cuda.current_stream(workspace.device)
     sptr = stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
     return int(lib.flint_attn_device_status(_ptr(workspace), sptr))
+
+
+def attn_fwd_static(q, k, v, q_norm_w, k_norm_w, sinks, out, lse, *, pos_ids=None,
+                    cu_seqlens=None, pad_mask=None, window: int = 513, use_rope: bool = True,
+                    rope_theta: float = 10000.0, eps: float = 1e-6, stream=None) -> None:
+    """flint_attn_fwd_static: the forward for callers that cannot allocate
+    device memory when they run the layer.  The caller passes every buffer,
+    outputs included; the kernels' scratch is a fixed device array inside the
+    library (STATIC_SCRATCH_BYTES, about 16,000 tokens), shared by all calls,
+    so calls that may overlap on the GPU must be serialised.  Nothing is
+    allocated here."""
+    import torch
+    lib = load_library()
+    T = int(q.shape[0])
+    _check(q, "q", torch.bfloat16, (T, HQ, HEAD_DIM))
+    _check(k, "k", torch.bfloat16, (T, HKV, HEAD_DIM))
+    _check(v, "v", torch.bfloat16, (T, HKV, HEAD_DIM))
+    _check(q_norm_w, "q_norm_w", torch.float32, (HEAD_DIM,))
+    _check(k_norm_w, "k_norm_w", torch.float32, (HEAD_DIM,))
+    _check(sinks, "sinks", torch.float32, (HQ,))
+    _check(out, "out", torch.bfloat16, (T, HQ * HEAD_DIM))
+    if lse is not None:
+        _check(lse, "lse", torch.float32, (HQ, T))
+    num_docs, batch, seqlen = 0, 0, 0
+    if pos_ids is not None:
+        _check(pos_ids, "pos_ids", torch.int32, (T,))
+    if cu_seqlens is not None:
+        _check(cu_seqlens, "cu_seqlens", torch.int32)
+        num_docs = int(cu_seqlens.numel()) - 1
+    if pad_mask is not None:
+        _check(pad_mask, "pad_mask", torch.uint8)
+        batch, seqlen = int(pad_mask.shape[0]), int(pad_mask.shape[1])
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device)
+    sptr = stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+    with torch.cuda.device(q.device):
+        st = lib.flint_attn_fwd_static(
+            _ptr(q), _ptr(k), _ptr(v), _ptr(q_norm_w), _ptr(k_norm_w), _ptr(sinks),
+            _ptr(pos_ids), _ptr(cu_seqlens), num_docs, _ptr(pad_mask), batch, seqlen, T,
+            int(window), int(bool(use_rope)), float(rope_theta), float(eps), _ptr(out),
+            _ptr(lse), sptr)
+    if st != 0:
+        raise FlintError(st, lib.flint_attn_last_error().decode())

@@ -132,11 +132,9 @@ const char* flint_attn_status_string(flint_status_t s) {
 
 }  // extern "C"
 
-namespace {
+namespace flint {
 
-enum Stage : int { kStagePrepare = 1, kStageAttend = 2, kStageBoth = 3 };
-
-flint_status_t run(int stages, const void* q, const void* k, const void* v, const float* q_norm_w,
+flint_status_t run_stages(int stages, const void* q, const void* k, const void* v, const float* q_norm_w,
                    const float* k_norm_w, const float* sinks, const int32_t* pos_ids,
                    const int32_t* cu_seqlens, int32_t num_docs, const uint8_t* pad_mask,
                    int32_t batch, int32_t seqlen, int32_t T, int32_t window, int32_t use_rope,
@@ -252,7 +250,9 @@ flint_status_t run(int stages, const void* q, const void* k, const void* v, cons
     return FLINT_OK;
 }
 
-}  // namespace
+flint_status_t set_error(flint_status_t s, const char* msg) { return fail(s, "%s", msg); }
+
+}  // namespace flint
 
 extern "C" {
 
@@ -266,9 +266,9 @@ extern "C" {
     q, k, v, q_norm_w, k_norm_w, sinks, pos_ids, cu_seqlens, num_docs, pad_mask, batch, seqlen, \
         T, window, use_rope, rope_theta, eps, out, lse, workspace, workspace_bytes, stream
 
-flint_status_t flint_attn_fwd(FLINT_ARGS) { return run(kStageBoth, FLINT_FWD_ARGS); }
-flint_status_t flint_attn_prepare(FLINT_ARGS) { return run(kStagePrepare, FLINT_FWD_ARGS); }
-flint_status_t flint_attn_attend(FLINT_ARGS) { return run(kStageAttend, FLINT_FWD_ARGS); }
+flint_status_t flint_attn_fwd(FLINT_ARGS) { return run_stages(kStageBoth, FLINT_FWD_ARGS); }
+flint_status_t flint_attn_prepare(FLINT_ARGS) { return run_stages(kStagePrepare, FLINT_FWD_ARGS); }
+flint_status_t flint_attn_attend(FLINT_ARGS) { return run_stages(kStageAttend, FLINT_FWD_ARGS); }
 
 flint_status_t flint_attn_device_status(const void* workspace, void* stream) {
     if (!workspace) return fail(FLINT_ERR_WORKSPACE, "workspace is null");

@@ -104,6 +104,9 @@ __device__ __forceinline__ void rope_cos_sin(int pos, double inv_freq, float* c,
     __sincosf((float)r, s, c);
 }
 
+// Stages of one forward call (host side).
+enum Stage : int { kStagePrepare = 1, kStageAttend = 2, kStageBoth = 3 };
+
 // Kernel parameter blocks (passed by value).
 struct PrepParams {
     const __nv_bfloat16* k;

@@ -166,6 +166,47 @@ FLINT_API flint_status_t flint_attn_attend(const void* q, const void* k, const v
  */
 FLINT_API flint_status_t flint_attn_device_status(const void* workspace, void* stream);
 
+/*
+ * Size in bytes of the scratch array behind flint_attn_fwd_static: 16 MiB,
+ * enough for about 16,000 tokens (1 KiB of normalised keys per token plus the
+ * work plan).
+ */
+#define FLINT_STATIC_SCRATCH_BYTES (16u << 20)
+
+/*
+ * flint_attn_fwd_static - the same forward as flint_attn_fwd, for callers
+ * that cannot allocate device memory when they run the layer (an allocator
+ * that must not be re-entered from a callback, a memory budget fixed up front,
+ * a host that only hands out its own buffers).  The pages have no counterpart
+ * of this entry point; it exists for those callers.
+ *
+ * Arguments are those of flint_attn_fwd without workspace and
+ * workspace_bytes; the caller still provides inputs and outputs.  The
+ * kernels' scratch (work plan, normalised keys) lives in a file-scope device
+ * array of FLINT_STATIC_SCRATCH_BYTES that every GPU loading the library
+ * keeps until the process exits.  No cudaMalloc, cudaFree or allocating
+ * library call is made.
+ *  - A problem whose scratch would exceed FLINT_STATIC_SCRATCH_BYTES
+ *    (flint_attn_workspace_bytes(T, n) larger than it) is rejected with
+ *    FLINT_ERR_WORKSPACE before any launch.
+ *  - The first call on a device looks up the array's device address
+ *    (cudaGetSymbolAddress) with that device current; make that first call
+ *    before any stream capture.
+ *  - Every call shares the one array and it keeps the last call's contents
+ *    (the kernels initialise what they read); calls that may overlap on the
+ *    GPU race on it, so serialise them (one stream, or events).
+ *  - Device-side status is not readable for this entry point.
+ */
+FLINT_API flint_status_t flint_attn_fwd_static(const void* q, const void* k, const void* v,
+                              const float* q_norm_w, const float* k_norm_w,
+                              const float* sinks, const int32_t* pos_ids,
+                              const int32_t* cu_seqlens, int32_t num_docs,
+                              const uint8_t* pad_mask, int32_t batch, int32_t seqlen,
+                              int32_t T, int32_t window, int32_t use_rope,
+                              float rope_theta, float eps,
+                              void* out, float* lse,
+                              void* stream);
+
 /* Text of the last error raised on the calling host thread ("" if none). */
 FLINT_API const char* flint_attn_last_error(void);
 
