@@ -17,10 +17,10 @@ constexpr int kHD = 128;
 constexpr int kGroup = kHQ / kHKV;          // query heads per KV head (8)
 
 // Tiling.  One MMA tile of 128 rows packs 16 tokens x the 8 query heads of a
-// KV group; a work item is one tile (16 consecutive tokens of one document)
+// KV group; a work item is 32 consecutive tokens of one document (two tiles)
 // for one KV group; keys are streamed in chunks of 128.
 constexpr int kTokPerTile = 16;
-constexpr int kTokPerItem = 16;
+constexpr int kTokPerItem = 32;
 constexpr int kKeyChunk = 128;
 
 // Device status codes (mirror flint_status_t).
