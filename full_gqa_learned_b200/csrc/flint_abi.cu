@@ -189,7 +189,9 @@ flint_status_t run_stages(int stages, const void* q, const void* k, const void* 
     if (st != FLINT_OK) return st;
     char* ws = static_cast<char*>(workspace);
     CUtensorMap tm_q, tm_k, tm_v;
-    st = make_map(enc, &tm_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, q, kHQ, T, kGroup, kTokPerTile);
+    // Q operand: the FP16 normalised queries that the preparation kernel
+    // left in the output rows
+    st = make_map(enc, &tm_q, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, out, kHQ, T, kGroup, kTokPerTile);
     if (st != FLINT_OK) return st;
     st = make_map(enc, &tm_k, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, ws + L.kn, kHKV, T, 1, kKeyChunk);
     if (st != FLINT_OK) return st;
@@ -199,7 +201,9 @@ flint_status_t run_stages(int stages, const void* q, const void* k, const void* 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     cudaError_t e = cudaSuccess;
     PrepParams pp;
+    pp.q = static_cast<const __nv_bfloat16*>(q);
     pp.k = static_cast<const __nv_bfloat16*>(k);
+    pp.q_norm_w = q_norm_w;
     pp.k_norm_w = k_norm_w;
     pp.sinks = sinks;
     pp.pos_ids = pos_ids;

@@ -8,7 +8,9 @@
 // RMSNorm and, on sliding layers, NeoX RoPE (FlintAttention.forward and
 // _apply_rope on the NeMo AutoModel "flint.layers" API page; the sink as an
 // extra zero-value softmax column in natural-logit units: HF discussion #26 on
-// RecursiveSI/flint).  k~ was prepared by the preparation kernel.
+// RecursiveSI/flint).  q~ and k~ (FP16, scaled by powers of two) were
+// prepared by the preparation kernel; q~ sits in the output rows of its own
+// token, which each tile reads through TMA before it writes its result there.
 //
 // Layout of one CTA (one per SM, persistent, 384 threads):
 //   warp 0      dynamic scheduler + TMA producer (Q tiles, K/V chunks)
@@ -41,11 +43,7 @@ constexpr uint32_t kHalfTile = kTileBytes / 2;       // one 64-column swizzled h
 constexpr uint32_t kOffQ = 0;                        // 2 Q tiles
 constexpr uint32_t kOffK = kOffQ + 2 * kTileBytes;   // 2 K stages
 constexpr uint32_t kOffV = kOffK + 2 * kTileBytes;   // 2 V stages
-constexpr uint32_t kOffRope = kOffV + 2 * kTileBytes;        // 2 x [16][64] float2
-constexpr uint32_t kRopeBytes = kTokPerTile * 64 * 8;
-constexpr uint32_t kOffW = kOffRope + 2 * kRopeBytes;        // q_norm_w [128] f32
-constexpr uint32_t kOffInv = kOffW + kHD * 4;                // inv_freq [64] f64
-constexpr uint32_t kOffBar = kOffInv + 64 * 8;               // mbarriers
+constexpr uint32_t kOffBar = kOffV + 2 * kTileBytes;         // mbarriers
 constexpr uint32_t kNumBars = 32;
 constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
 constexpr uint32_t kSmemUsed = kOffMisc + 64;
@@ -54,7 +52,7 @@ constexpr uint32_t kSmemBytes = kSmemUsed + 1024;            // + alignment slac
 // barrier indices
 enum : uint32_t {
     B_SCHED_FULL = 0, B_SCHED_EMPTY = 2,
-    B_Q_FULL = 4, B_Q_READY = 6, B_Q_EMPTY = 8,
+    B_Q_FULL = 4, B_Q_EMPTY = 8,
     B_K_FULL = 10, B_K_EMPTY = 12, B_V_FULL = 14, B_V_EMPTY = 16,
     B_S_FULL = 18, B_P_FULL = 20, B_O_FULL = 22, B_DRAIN = 24
 };
@@ -63,7 +61,6 @@ struct Misc {
     int sched[2];
     uint32_t tmem_base;
     int abort_flag;
-    float q_scale;       // 2^eq
     float logit_scale;   // log2(e)/sqrt(128) * 2^-(eq+ek)
 };
 
@@ -143,19 +140,12 @@ __device__ __forceinline__ uint64_t exp2_poly2(uint64_t x) {
 // the FMA/ALU pipes, so MUFU and the FMA/ALU pipes balance near 1/8.
 constexpr int kPolyPairs = 1;
 
-// Two FP32 values -> packed 16-bit pair, `lo` in the low half.
+// Two FP32 values -> packed BF16 pair, `lo` in the low half.
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     uint32_t r;
     asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
     return r;
 }
-__device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
-    uint32_t r;
-    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
-    return r;
-}
-__device__ __forceinline__ float bf16_lo(uint32_t u) { return __uint_as_float(u << 16); }
-__device__ __forceinline__ float bf16_hi(uint32_t u) { return __uint_as_float(u & 0xffff0000u); }
 
 __device__ __forceinline__ int chunk_cols(int ks, int ke) {
     int n = ke - ks;
@@ -173,8 +163,6 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const uint32_t bar0 = sbase + kOffBar;
     auto bar = [&](uint32_t i) { return bar0 + 8u * i; };
     Misc* misc = reinterpret_cast<Misc*>(smem + kOffMisc);
-    float* s_wq = reinterpret_cast<float*>(smem + kOffW);
-    double* s_inv = reinterpret_cast<double*>(smem + kOffInv);
     volatile int* abort_flag = &misc->abort_flag;
 
     const WsLayout L = ws_layout(p.T, p.nseg);
@@ -193,7 +181,6 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         mbar_init(bar(B_SCHED_EMPTY + 1), 1 + 8);
         for (int t = 0; t < 2; ++t) {
             mbar_init(bar(B_Q_FULL + t), 1);
-            mbar_init(bar(B_Q_READY + t), 128);     // every softmax thread of tile t
             mbar_init(bar(B_Q_EMPTY + t), 1);
             mbar_init(bar(B_K_FULL + t), 1);
             mbar_init(bar(B_K_EMPTY + t), 1);
@@ -216,14 +203,11 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         tmem_alloc(smem_u32(&misc->tmem_base), 512);
         tmem_relinquish();
     }
-    if (tid < kHD) s_wq[tid] = p.q_norm_w[tid];
-    if (tid >= 128 && tid < 192) s_inv[tid - 128] = exp2(-(double)(tid - 128) / 64.0 * log2((double)p.rope_theta));
     if (warp == 2) {
         const float mq = warp_max_abs128(p.q_norm_w);
         const float mk = warp_max_abs128(p.k_norm_w);
         if (lane == 0) {
             const int eq = prescale_exponent(mq), ek = prescale_exponent(mk);
-            misc->q_scale = ldexpf(1.f, eq);
             misc->logit_scale = ldexpf(1.4426950408889634f * 0.08838834764831845f, -(eq + ek));
         }
     }
@@ -348,16 +332,16 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 const int q0 = it.x, nq = it.y, ds = it.z, nch = it.w;
                 const int ke = q0 + nq;
                 const int kb = p.window > 0 ? max(ds, q0 - p.window + 1) : ds;
-                if (!mbar_wait(bar(B_Q_READY + 0), qrph, abort_flag, status)) break;
-                if (!mbar_wait(bar(B_Q_READY + 1), qrph, abort_flag, status)) break;
-                qrph ^= 1;
-                tc_fence_after();
-                // S for chunk 0
+                // S for chunk 0, each tile as soon as its Q tile has landed
                 if (!mbar_wait(bar(B_K_FULL + kst), kph, abort_flag, status)) break;
+                if (!mbar_wait(bar(B_Q_FULL + 0), qrph, abort_flag, status)) break;
                 tc_fence_after();
                 int ncol = chunk_cols(kb, ke);
                 issue_s(0, kst, ncol);
                 mma_commit(bar(B_S_FULL + 0));
+                if (!mbar_wait(bar(B_Q_FULL + 1), qrph, abort_flag, status)) break;
+                tc_fence_after();
+                qrph ^= 1;
                 issue_s(1, kst, ncol);
                 mma_commit(bar(B_S_FULL + 1));
                 if (nch == 1) {
@@ -422,13 +406,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         const uint32_t lane_base = (uint32_t)(warp & 3) * 32u;
         const uint32_t t_s = tmem + (lane_base << 16) + 128u * t;
         const uint32_t t_o = tmem + (lane_base << 16) + 256u + 128u * t;
-        const uint32_t q_tile = sbase + kOffQ + t * kTileBytes;
-        uint8_t* q_tile_ptr = smem + kOffQ + t * kTileBytes;
-        float2* rope_tab = reinterpret_cast<float2*>(smem + kOffRope + t * kRopeBytes);
         const float C = misc->logit_scale;
-        const float qs = misc->q_scale;
-        uint32_t sslot = 0, sph = 0, qph = 0, s_ph = 0, oph = 0;
-        (void)q_tile;
+        uint32_t sslot = 0, sph = 0, s_ph = 0, oph = 0;
         for (;;) {
             // Warps of the warpgroup run without block-level barriers; every
             // wait's outcome is made warp-uniform (tcgen05.ld/st are
@@ -449,79 +428,6 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             const bool row_valid = (kTokPerTile * t + tl) < nq;
             const int ke = q0 + nq;
             const int kb = p.window > 0 ? max(ds, q0 - p.window + 1) : ds;
-
-            // ---- rope table for this tile's 16 tokens: thread r fills token
-            // tl, pair indices 8*hl .. 8*hl+7.  The 8 threads of a token are
-            // lanes of one warp, so a warp barrier publishes the entries.
-            __syncwarp();
-            if (p.use_rope) {
-                int pos = 0;
-                const int tok = min(i, p.T - 1);
-                pos = p.pos_ids ? p.pos_ids[tok] : (i - ds);
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    float c, s;
-                    rope_cos_sin(pos, s_inv[8 * hl + e], &c, &s);
-                    rope_tab[tl * 64 + 8 * hl + e] = make_float2(c, s);
-                }
-            }
-            __syncwarp();
-            ok = __all_sync(0xffffffffu, mbar_wait(bar(B_Q_FULL + t), qph, abort_flag, status));
-            if (!ok) break;
-            qph ^= 1;
-
-            // ---- Q prologue, in place: RMSNorm (weight form), RoPE, x 2^eq, FP16.
-            // Thread r owns row r; chunk c of each 64-channel half sits at the
-            // 128-byte-swizzled position (c ^ (r & 7)).  Two passes over shared
-            // memory keep the row out of registers.
-            {
-                const int sw = r & 7;
-                float ss = 0.f;
-#pragma unroll 2
-                for (int c = 0; c < 8; ++c) {
-                    const int off = r * 128 + ((c ^ sw) << 4);
-                    const uint4 ua = *reinterpret_cast<const uint4*>(q_tile_ptr + off);
-                    const uint4 ub = *reinterpret_cast<const uint4*>(q_tile_ptr + kHalfTile + off);
-                    const uint32_t w8[8] = {ua.x, ua.y, ua.z, ua.w, ub.x, ub.y, ub.z, ub.w};
-#pragma unroll
-                    for (int j = 0; j < 8; ++j) {
-                        const float x0 = bf16_lo(w8[j]), x1 = bf16_hi(w8[j]);
-                        ss = fmaf(x0, x0, ss);
-                        ss = fmaf(x1, x1, ss);
-                    }
-                }
-                const float rn = rsqrtf(ss * (1.f / kHD) + p.eps) * qs;
-#pragma unroll 1
-                for (int c = 0; c < 8; ++c) {
-                    const int off = r * 128 + ((c ^ sw) << 4);
-                    const uint4 ua = *reinterpret_cast<const uint4*>(q_tile_ptr + off);
-                    const uint4 ub = *reinterpret_cast<const uint4*>(q_tile_ptr + kHalfTile + off);
-                    const uint32_t wa4[4] = {ua.x, ua.y, ua.z, ua.w};
-                    const uint32_t wb4[4] = {ub.x, ub.y, ub.z, ub.w};
-                    uint32_t oa[4], ob[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int d0 = 8 * c + 2 * e;          // channels d0, d0+1 and 64+d0, 65+d0
-                        float a0 = bf16_lo(wa4[e]) * rn * s_wq[d0];
-                        float a1 = bf16_hi(wa4[e]) * rn * s_wq[d0 + 1];
-                        float b0 = bf16_lo(wb4[e]) * rn * s_wq[64 + d0];
-                        float b1 = bf16_hi(wb4[e]) * rn * s_wq[65 + d0];
-                        if (p.use_rope) {
-                            const float2 cs0 = rope_tab[tl * 64 + d0];
-                            const float2 cs1 = rope_tab[tl * 64 + d0 + 1];
-                            const float y0 = a0 * cs0.x - b0 * cs0.y, z0 = b0 * cs0.x + a0 * cs0.y;
-                            const float y1 = a1 * cs1.x - b1 * cs1.y, z1 = b1 * cs1.x + a1 * cs1.y;
-                            a0 = y0; b0 = z0; a1 = y1; b1 = z1;
-                        }
-                        oa[e] = pack_f16(a0, a1);
-                        ob[e] = pack_f16(b0, b1);
-                    }
-                    *reinterpret_cast<uint4*>(q_tile_ptr + off) = make_uint4(oa[0], oa[1], oa[2], oa[3]);
-                    *reinterpret_cast<uint4*>(q_tile_ptr + kHalfTile + off) = make_uint4(ob[0], ob[1], ob[2], ob[3]);
-                }
-            }
-            fence_proxy_async_smem();
-            mbar_arrive(bar(B_Q_READY + t));
 
             // ---- online softmax over the key chunks
             const float sink = p.sinks[h];
@@ -652,19 +558,25 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
             __nv_bfloat16* orow = p.out + ((size_t)i * kHQ + h) * kHD;
 #pragma unroll
-            for (int b = 0; b < 4; ++b) {
-                uint32_t v[32];
-                tmem_ld32(t_o + 32u * b, v);
+            for (int hb = 0; hb < 2; ++hb) {
+                // two TMEM loads of 32 columns in flight per wait
+                uint32_t v[64];
+                tmem_ld32(t_o + 64u * hb, v);
+                tmem_ld32(t_o + 64u * hb + 32u, v + 32);
                 tmem_wait_ld();
-                uint32_t w[16];
 #pragma unroll
-                for (int j = 0; j < 16; ++j)
-                    w[j] = pack_bf16(__uint_as_float(v[2 * j]) * inv_l, __uint_as_float(v[2 * j + 1]) * inv_l);
-                if (row_valid) {
-                    uint4* dst = reinterpret_cast<uint4*>(orow + 32 * b);
+                for (int b = 0; b < 2; ++b) {
+                    uint32_t w[16];
 #pragma unroll
-                    for (int j = 0; j < 4; ++j)
-                        dst[j] = make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+                    for (int j = 0; j < 16; ++j)
+                        w[j] = pack_bf16(__uint_as_float(v[32 * b + 2 * j]) * inv_l,
+                                         __uint_as_float(v[32 * b + 2 * j + 1]) * inv_l);
+                    if (row_valid) {
+                        uint4* dst = reinterpret_cast<uint4*>(orow + 64 * hb + 32 * b);
+#pragma unroll
+                        for (int j = 0; j < 4; ++j)
+                            dst[j] = make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+                    }
                 }
             }
             if (row_valid && p.lse) p.lse[(size_t)h * p.T + i] = m * 0.6931471805599453f + logf(l);

@@ -109,7 +109,9 @@ enum Stage : int { kStagePrepare = 1, kStageAttend = 2, kStageBoth = 3 };
 
 // Kernel parameter blocks (passed by value).
 struct PrepParams {
+    const __nv_bfloat16* q;
     const __nv_bfloat16* k;
+    const float* q_norm_w;
     const float* k_norm_w;
     const float* sinks;
     const int* pos_ids;

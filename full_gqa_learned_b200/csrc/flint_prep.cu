@@ -6,13 +6,15 @@
 // their number of 128-key chunks, longest first, so the attention kernel's
 // dynamic scheduler hands out the largest items first.
 //
-// The other blocks prepare the keys once per token instead of once per use:
-// per-head RMSNorm with k_norm_w (weight form; HF discussion #26 on
-// RecursiveSI/flint), then on sliding layers NeoX RoPE at the document-local
-// position (FlintAttention._apply_rope), scaled by a power of two and rounded
-// to FP16 into the workspace.  They also write the outputs of padded query
-// tokens: zeros and lse = sink (FlintAttention.forward, attention_mask: the
-// sink remains valid for padded queries).
+// The other blocks prepare the keys and queries once per token instead of
+// once per use: per-head RMSNorm with k_norm_w / q_norm_w (weight form; HF
+// discussion #26 on RecursiveSI/flint), then on sliding layers NeoX RoPE at
+// the document-local position (FlintAttention._apply_rope), scaled by a power
+// of two and rounded to FP16.  Keys go to the workspace; queries go to the
+// output rows of their own token, which the attention kernel reads back as
+// its Q operand before it writes the result over them.  Padded query tokens
+// get their final outputs here: zeros and lse = sink (FlintAttention.forward,
+// attention_mask: the sink remains valid for padded queries).
 #include "flint_common.cuh"
 
 namespace flint {
@@ -188,112 +190,144 @@ __device__ __forceinline__ int thd_segment_start(const int* cu, int ndocs, int t
     return cu[lo];
 }
 
-__device__ void prepare_keys(const PrepParams& p) {
+// Normalise one 128-channel head row held by 8 lanes (lane sub owns channels
+// 8*sub .. 8*sub+7 of each 64-channel half): RMSNorm in weight form, optional
+// NeoX rotation with the lane's 8 (cos, sin) pairs, x scale, FP16.
+__device__ __forceinline__ void norm_rope_row(const __nv_bfloat16* src, __half* dst, const float* w,
+                                              float eps, float scale, int sub, bool rope,
+                                              const float* cc, const float* sn) {
+    const uint4 a = *reinterpret_cast<const uint4*>(src + 8 * sub);
+    const uint4 b = *reinterpret_cast<const uint4*>(src + 64 + 8 * sub);
+    float x0[8], x1[8];
+    {
+        const __nv_bfloat162* pa = reinterpret_cast<const __nv_bfloat162*>(&a);
+        const __nv_bfloat162* pb = reinterpret_cast<const __nv_bfloat162*>(&b);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const float2 fa = __bfloat1622float2(pa[e]);
+            const float2 fb = __bfloat1622float2(pb[e]);
+            x0[2 * e] = fa.x; x0[2 * e + 1] = fa.y;
+            x1[2 * e] = fb.x; x1[2 * e + 1] = fb.y;
+        }
+    }
+    float ss = 0.f;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) ss = fmaf(x0[e], x0[e], fmaf(x1[e], x1[e], ss));
+    ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+    ss += __shfl_xor_sync(0xffffffffu, ss, 2);
+    ss += __shfl_xor_sync(0xffffffffu, ss, 4);
+    const float r = rsqrtf(ss * (1.f / kHD) + eps) * scale;
+    float n0[8], n1[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+        n0[e] = x0[e] * r * w[8 * sub + e];
+        n1[e] = x1[e] * r * w[64 + 8 * sub + e];
+    }
+    if (rope) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            const float y0 = n0[e] * cc[e] - n1[e] * sn[e];
+            const float y1 = n1[e] * cc[e] + n0[e] * sn[e];
+            n0[e] = y0; n1[e] = y1;
+        }
+    }
+    uint4 oa, ob;
+    {
+        __half2* ha = reinterpret_cast<__half2*>(&oa);
+        __half2* hb = reinterpret_cast<__half2*>(&ob);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            ha[e] = __floats2half2_rn(n0[2 * e], n0[2 * e + 1]);
+            hb[e] = __floats2half2_rn(n1[2 * e], n1[2 * e + 1]);
+        }
+    }
+    *reinterpret_cast<uint4*>(dst + 8 * sub) = oa;
+    *reinterpret_cast<uint4*>(dst + 64 + 8 * sub) = ob;
+}
+
+__device__ void prepare_tokens(const PrepParams& p) {
     __shared__ double s_inv_freq[64];
-    __shared__ float s_w[kHD];
-    __shared__ float s_scale;
+    __shared__ float s_wk[kHD], s_wq[kHD];
+    __shared__ float s_kscale, s_qscale;
     __shared__ int s_thd_end;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const WsLayout L = ws_layout(p.T, p.nseg);
     __half* kn = reinterpret_cast<__half*>(p.ws + L.kn);
 
     if (tid < 64) s_inv_freq[tid] = exp2(-(double)tid / 64.0 * log2((double)p.rope_theta));
-    if (tid < kHD) s_w[tid] = p.k_norm_w[tid];
+    if (tid < kHD) s_wk[tid] = p.k_norm_w[tid];
+    if (tid >= kHD && tid < 2 * kHD) s_wq[tid - kHD] = p.q_norm_w[tid - kHD];
     if (warp == 0) {
-        float m = warp_max_abs128(p.k_norm_w);
-        if (lane == 0) s_scale = ldexpf(1.f, prescale_exponent(m));
+        const float m = warp_max_abs128(p.k_norm_w);
+        if (lane == 0) s_kscale = ldexpf(1.f, prescale_exponent(m));
+    }
+    if (warp == 1) {
+        const float m = warp_max_abs128(p.q_norm_w);
+        if (lane == 0) s_qscale = ldexpf(1.f, prescale_exponent(m));
     }
     if (tid == 0) s_thd_end = (p.mode == kMaskThd) ? p.cu_seqlens[p.nseg] : p.T;
     __syncthreads();
 
     const int head = lane >> 3, sub = lane & 7;
     const int nwarps_total = (gridDim.x - 1) * (blockDim.x >> 5);
-    const float scale = s_scale;
+    const float kscale = s_kscale, qscale = s_qscale;
+    const bool rope = p.use_rope != 0;
     for (int t = (blockIdx.x - 1) * (blockDim.x >> 5) + warp; t < p.T; t += nwarps_total) {
-        // ---- normalise (and rotate) the 4 key heads of token t
-        const __nv_bfloat16* row = p.k + ((size_t)t * kHKV + head) * kHD;
-        uint4 a = *reinterpret_cast<const uint4*>(row + 8 * sub);
-        uint4 b = *reinterpret_cast<const uint4*>(row + 64 + 8 * sub);
-        float x0[8], x1[8];
-        {
-            const __nv_bfloat162* pa = reinterpret_cast<const __nv_bfloat162*>(&a);
-            const __nv_bfloat162* pb = reinterpret_cast<const __nv_bfloat162*>(&b);
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                float2 fa = __bfloat1622float2(pa[e]);
-                float2 fb = __bfloat1622float2(pb[e]);
-                x0[2 * e] = fa.x; x0[2 * e + 1] = fa.y;
-                x1[2 * e] = fb.x; x1[2 * e + 1] = fb.y;
-            }
-        }
-        float ss = 0.f;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) ss = fmaf(x0[e], x0[e], fmaf(x1[e], x1[e], ss));
-        ss += __shfl_xor_sync(0xffffffffu, ss, 1);
-        ss += __shfl_xor_sync(0xffffffffu, ss, 2);
-        ss += __shfl_xor_sync(0xffffffffu, ss, 4);
-        const float r = rsqrtf(ss * (1.f / kHD) + p.eps) * scale;
-        float n0[8], n1[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-            n0[e] = x0[e] * r * s_w[8 * sub + e];
-            n1[e] = x1[e] * r * s_w[64 + 8 * sub + e];
-        }
-        if (p.use_rope) {
+        // ---- the lane's 8 (cos, sin) pairs f = 8*sub + e at the token's
+        // document-local position, shared by its 4 key and 32 query heads
+        float cc[8], sn[8];
+        if (rope) {
             int pos;
             if (p.pos_ids) pos = p.pos_ids[t];
             else if (p.mode == kMaskThd) pos = t - (t < s_thd_end ? thd_segment_start(p.cu_seqlens, p.nseg, t) : s_thd_end);
             else if (p.mode == kMaskPad) pos = t % p.seqlen;
             else pos = t;
-            // lane computes the pairs f = 2*lane and 2*lane + 1
+            // lane computes the pairs 2*lane and 2*lane + 1
             float c0, s0, c1, s1;
             rope_cos_sin(pos, s_inv_freq[2 * lane], &c0, &s0);
             rope_cos_sin(pos, s_inv_freq[2 * lane + 1], &c1, &s1);
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
-                const int f = 8 * sub + e;             // pair index of this element
-                const int src = f >> 1;
-                float cc = __shfl_sync(0xffffffffu, (f & 1) ? c1 : c0, src);
-                float sn = __shfl_sync(0xffffffffu, (f & 1) ? s1 : s0, src);
+                const int f = 8 * sub + e;
                 // (e & 1) is uniform across the warp for a given e, so the
                 // selected register is the same in every lane
-                float y0 = n0[e] * cc - n1[e] * sn;
-                float y1 = n1[e] * cc + n0[e] * sn;
-                n0[e] = y0; n1[e] = y1;
+                cc[e] = __shfl_sync(0xffffffffu, (e & 1) ? c1 : c0, f >> 1);
+                sn[e] = __shfl_sync(0xffffffffu, (e & 1) ? s1 : s0, f >> 1);
             }
         }
-        uint4 oa, ob;
-        {
-            __half2* ha = reinterpret_cast<__half2*>(&oa);
-            __half2* hb = reinterpret_cast<__half2*>(&ob);
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                ha[e] = __floats2half2_rn(n0[2 * e], n0[2 * e + 1]);
-                hb[e] = __floats2half2_rn(n1[2 * e], n1[2 * e + 1]);
-            }
-        }
-        __half* dst = kn + ((size_t)t * kHKV + head) * kHD;
-        *reinterpret_cast<uint4*>(dst + 8 * sub) = oa;
-        *reinterpret_cast<uint4*>(dst + 64 + 8 * sub) = ob;
+        // ---- the 4 key heads (head = lane / 8)
+        norm_rope_row(p.k + ((size_t)t * kHKV + head) * kHD, kn + ((size_t)t * kHKV + head) * kHD,
+                      s_wk, p.eps, kscale, sub, rope, cc, sn);
 
-        // ---- padded query token: zero output row, lse = sink
         bool padded;
         if (p.mode == kMaskThd) padded = t >= s_thd_end;
         else if (p.mode == kMaskPad) padded = p.pad_mask[t] == 0;
         else padded = false;
         if (padded) {
+            // ---- padded query token: zero output row, lse = sink
             uint4 z = make_uint4(0, 0, 0, 0);
             uint4* o = reinterpret_cast<uint4*>(p.out + (size_t)t * kHQ * kHD);
 #pragma unroll 4
             for (int i = lane; i < kHQ * kHD / 8; i += 32) o[i] = z;
             if (p.lse) p.lse[(size_t)lane * p.T + t] = p.sinks[lane];
+        } else {
+            // ---- the 32 query heads, 4 per pass, into the output rows of
+            // the token: the attention kernel reads them back as its FP16
+            // Q operand and overwrites them with the result
+            const __nv_bfloat16* qrow = p.q + (size_t)t * kHQ * kHD;
+            __half* qdst = reinterpret_cast<__half*>(p.out + (size_t)t * kHQ * kHD);
+#pragma unroll 2
+            for (int hq = 0; hq < kHQ / kHKV; ++hq) {
+                const int hh = kHKV * hq + head;
+                norm_rope_row(qrow + hh * kHD, qdst + hh * kHD, s_wq, p.eps, qscale, sub, rope, cc, sn);
+            }
         }
     }
 }
 
 __global__ void __launch_bounds__(1024, 1) prep_kernel(PrepParams p) {
     if (blockIdx.x == 0) build_plan(p);
-    else prepare_keys(p);
+    else prepare_tokens(p);
 }
 
 }  // namespace flint
