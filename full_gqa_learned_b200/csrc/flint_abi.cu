@@ -18,7 +18,9 @@ namespace flint {
 __global__ void prep_kernel(PrepParams p);
 __global__ void attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q,
                                 const __grid_constant__ CUtensorMap tm_k,
-                                const __grid_constant__ CUtensorMap tm_v, const AttnParams p);
+                                const __grid_constant__ CUtensorMap tm_v,
+                                const __grid_constant__ CUtensorMap tm_o,
+                                const __grid_constant__ CUtensorMap tm_o1, const AttnParams p);
 extern const unsigned kAttnSmemBytes;
 extern const unsigned kAttnThreads;
 }  // namespace flint
@@ -188,12 +190,18 @@ flint_status_t run_stages(int stages, const void* q, const void* k, const void* 
     st = get_encoder(&enc);
     if (st != FLINT_OK) return st;
     char* ws = static_cast<char*>(workspace);
-    CUtensorMap tm_q, tm_k, tm_v;
+    CUtensorMap tm_q, tm_k, tm_v, tm_o, tm_o1;
     // Q operand: the FP16 normalised queries that the preparation kernel
     // left in the output rows
     st = make_map(enc, &tm_q, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, out, kHQ, T, kGroup, kTokPerTile);
     if (st != FLINT_OK) return st;
     st = make_map(enc, &tm_k, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, ws + L.kn, kHKV, T, 1, kKeyChunk);
+    if (st != FLINT_OK) return st;
+    // result: 4 tokens (the rows of one softmax warp), and single tokens
+    // where a document ends inside a warp's 4
+    st = make_map(enc, &tm_o, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, out, kHQ, T, kGroup, 4);
+    if (st != FLINT_OK) return st;
+    st = make_map(enc, &tm_o1, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, out, kHQ, T, kGroup, 1);
     if (st != FLINT_OK) return st;
     st = make_map(enc, &tm_v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, v, kHKV, T, 1, kKeyChunk);
     if (st != FLINT_OK) return st;
@@ -248,7 +256,7 @@ flint_status_t run_stages(int stages, const void* q, const void* k, const void* 
     ap.eps = eps;
     const int max_units = L.max_items * kHKV;
     const int grid = max_units < sms ? max_units : sms;
-    attn_fwd_kernel<<<grid, kAttnThreads, kAttnSmemBytes, s>>>(tm_q, tm_k, tm_v, ap);
+    attn_fwd_kernel<<<grid, kAttnThreads, kAttnSmemBytes, s>>>(tm_q, tm_k, tm_v, tm_o, tm_o1, ap);
     e = cudaGetLastError();
     if (e != cudaSuccess) return fail(FLINT_ERR_CUDA, "attention launch: %s", cudaGetErrorString(e));
     return FLINT_OK;

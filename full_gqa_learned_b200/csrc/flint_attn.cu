@@ -43,7 +43,9 @@ constexpr uint32_t kHalfTile = kTileBytes / 2;       // one 64-column swizzled h
 constexpr uint32_t kOffQ = 0;                        // 2 Q tiles
 constexpr uint32_t kOffK = kOffQ + 2 * kTileBytes;   // 2 K stages
 constexpr uint32_t kOffV = kOffK + 2 * kTileBytes;   // 2 V stages
-constexpr uint32_t kOffBar = kOffV + 2 * kTileBytes;         // mbarriers
+constexpr uint32_t kOffStage = kOffV + 2 * kTileBytes;       // output staging, 4 KiB per softmax warp
+constexpr uint32_t kStageBytes = 32 * 128;                   // 32 rows x 64 channels x BF16
+constexpr uint32_t kOffBar = kOffStage + 8 * kStageBytes;    // mbarriers
 constexpr uint32_t kNumBars = 32;
 constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
 constexpr uint32_t kSmemUsed = kOffMisc + 64;
@@ -155,7 +157,8 @@ __device__ __forceinline__ int chunk_cols(int ks, int ke) {
 
 __global__ void __launch_bounds__(kThreads, 1)
 attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
+                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+                const __grid_constant__ CUtensorMap tm_o1, const AttnParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~uintptr_t(1023));
@@ -408,6 +411,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         const uint32_t t_o = tmem + (lane_base << 16) + 256u + 128u * t;
         const float C = misc->logit_scale;
         uint32_t sslot = 0, sph = 0, s_ph = 0, oph = 0;
+        // this warp's output staging: its 32 rows = tokens 4*(warp&3) .. +3
+        // of the tile, 64 channels at a time
+        uint8_t* stg = smem + kOffStage + (warp - 4) * kStageBytes;
+        const uint32_t stg_s = sbase + kOffStage + (warp - 4) * kStageBytes;
         for (;;) {
             // Warps of the warpgroup run without block-level barriers; every
             // wait's outcome is made warp-uniform (tcgen05.ld/st are
@@ -556,27 +563,55 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             oph ^= 1;
             tc_fence_after();
             const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
-            __nv_bfloat16* orow = p.out + ((size_t)i * kHQ + h) * kHD;
-#pragma unroll
-            for (int hb = 0; hb < 2; ++hb) {
-                // two TMEM loads of 32 columns in flight per wait
+            // Valid tokens of this warp's 4: where a document ends inside the
+            // tile, rows of other documents must not be written.
+            const int wt0 = kTokPerTile * t + 4 * (warp & 3);       // first token of the warp, in the item
+            const int nvw = max(0, min(4, nq - wt0));
+            const int sw = lane & 7;
+            // One 64-channel half at a time: O / l -> BF16 into the warp's
+            // staging block in the 128-byte-swizzled layout of the output
+            // tensor map, then lane 0 stores it with TMA (one 4-token box, or
+            // one box per valid token).  The TMEM load of the second half
+            // overlaps the store of the first.
+            uint32_t pk[32];
+            {
                 uint32_t v[64];
-                tmem_ld32(t_o + 64u * hb, v);
-                tmem_ld32(t_o + 64u * hb + 32u, v + 32);
+                tmem_ld32(t_o, v);
+                tmem_ld32(t_o + 32u, v + 32);
                 tmem_wait_ld();
 #pragma unroll
-                for (int b = 0; b < 2; ++b) {
-                    uint32_t w[16];
+                for (int j = 0; j < 32; ++j)
+                    pk[j] = pack_bf16(__uint_as_float(v[2 * j]) * inv_l, __uint_as_float(v[2 * j + 1]) * inv_l);
+            }
+#pragma unroll 1
+            for (int hb = 0; hb < 2; ++hb) {
+                // the staging block is free once lane 0's earlier stores have read it
+                if (lane == 0) bulk_wait_group_read0();
+                __syncwarp();
 #pragma unroll
-                    for (int j = 0; j < 16; ++j)
-                        w[j] = pack_bf16(__uint_as_float(v[32 * b + 2 * j]) * inv_l,
-                                         __uint_as_float(v[32 * b + 2 * j + 1]) * inv_l);
-                    if (row_valid) {
-                        uint4* dst = reinterpret_cast<uint4*>(orow + 64 * hb + 32 * b);
-#pragma unroll
-                        for (int j = 0; j < 4; ++j)
-                            dst[j] = make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+                for (int c = 0; c < 8; ++c)
+                    *reinterpret_cast<uint4*>(stg + lane * 128 + ((c ^ sw) << 4)) =
+                        make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0 && nvw > 0) {
+                    if (nvw == 4) {
+                        tma_store_3d(&tm_o, stg_s, 64 * hb, kGroup * g, q0 + wt0);
+                    } else {
+                        for (int k = 0; k < nvw; ++k)
+                            tma_store_3d(&tm_o1, stg_s + 1024u * k, 64 * hb, kGroup * g, q0 + wt0 + k);
                     }
+                    bulk_commit_group();
+                }
+                if (hb == 0) {
+                    uint32_t v[64];
+                    tmem_ld32(t_o + 64u, v);
+                    tmem_ld32(t_o + 96u, v + 32);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int j = 0; j < 32; ++j)
+                        pk[j] = pack_bf16(__uint_as_float(v[2 * j]) * inv_l,
+                                          __uint_as_float(v[2 * j + 1]) * inv_l);
                 }
             }
             if (row_valid && p.lse) p.lse[(size_t)h * p.T + i] = m * 0.6931471805599453f + logf(l);
@@ -585,6 +620,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     }
 
     // ---------------------------------------------------------------- teardown
+    if (warp >= 4 && lane == 0) bulk_wait_group0();
     tc_fence_before();
     __syncthreads();
     if (warp == 1) {

@@ -244,3 +244,27 @@ def test_bad_cu_seqlens_reports_invalid():
     fa.attn_fwd(t["q"], t["k"], t["v"], t["q_norm_w"], t["k_norm_w"], t["sinks"],
                 cu_seqlens=cu, window=0, use_rope=False)
     assert fa.device_status(fa.attn_fwd.last_workspace) == 1
+
+
+@pytest.mark.parametrize("packed", [False, True])
+def test_out_may_alias_q(packed):
+    """The call uses out as scratch for the normalised queries; out = q (in
+    place) must give the same bits as a separate output buffer."""
+    import torch
+    import full_gqa_learned_b200 as fa
+    if packed:
+        cu = np.array([0, 70, 70, 231], np.int32)
+        w = W.make_small(240, seed=16, window=129, use_rope=True, cu_seqlens=cu)
+    else:
+        w = W.make_small(240, seed=17, window=0, use_rope=False)
+    t = to_device(w)
+    kw = dict(cu_seqlens=t["cu_seqlens"], window=w.window, use_rope=w.use_rope,
+              rope_theta=w.rope_theta, eps=w.eps)
+    args = (t["k"], t["v"], t["q_norm_w"], t["k_norm_w"], t["sinks"])
+    o1, l1 = fa.attn_fwd(t["q"], *args, **kw)
+    q2 = t["q"].clone()
+    o2, l2 = fa.attn_fwd(q2, *args, out=q2.view(w.T, 32 * 128), **kw)
+    assert fa.device_status(fa.attn_fwd.last_workspace) == 0
+    torch.cuda.synchronize()
+    assert torch.equal(o1.view(torch.int16), o2.view(torch.int16))
+    assert torch.equal(l1, l2)
