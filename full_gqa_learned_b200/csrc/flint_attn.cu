@@ -459,97 +459,129 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 tmem_wait_ld();
                 const bool boundary = (c == nch - 1) || (ks + nc - 1 > tok0) ||
                                       (p.window > 0 && ks < tok0 + kTokPerTile - p.window);
-                // row max over visible keys: 3-input max, 8 independent chains
-                float mxp[8];
+                // row max over the S columns: 3-input max, 8 independent
+                // chains; masked columns become -inf in sv
+                auto row_max = [&](bool masked) -> float {
+                    float mxp[8];
 #pragma unroll
-                for (int k8 = 0; k8 < 8; ++k8) mxp[k8] = -INFINITY;
-                if (boundary) {
-                    const int jlo = lo - ks, jhi = i - ks;
+                    for (int k8 = 0; k8 < 8; ++k8) mxp[k8] = -INFINITY;
+                    if (masked) {
+                        const int jlo = lo - ks, jhi = i - ks;
 #pragma unroll
-                    for (int b = 0; b < 4; ++b) {
-                        if (b < nblk) {
+                        for (int b = 0; b < 4; ++b) {
+                            if (b < nblk) {
 #pragma unroll
-                            for (int j = 32 * b; j < 32 * b + 32; j += 2) {
-                                const float x0 = ((j >= jlo) && (j <= jhi)) ? __uint_as_float(sv[j]) : -INFINITY;
-                                const float x1 = ((j + 1 >= jlo) && (j + 1 <= jhi)) ? __uint_as_float(sv[j + 1]) : -INFINITY;
-                                sv[j] = __float_as_uint(x0);
-                                sv[j + 1] = __float_as_uint(x1);
-                                mxp[(j >> 1) & 7] = max3(mxp[(j >> 1) & 7], x0, x1);
+                                for (int j = 32 * b; j < 32 * b + 32; j += 2) {
+                                    const float x0 = ((j >= jlo) && (j <= jhi)) ? __uint_as_float(sv[j]) : -INFINITY;
+                                    const float x1 = ((j + 1 >= jlo) && (j + 1 <= jhi)) ? __uint_as_float(sv[j + 1]) : -INFINITY;
+                                    sv[j] = __float_as_uint(x0);
+                                    sv[j + 1] = __float_as_uint(x1);
+                                    mxp[(j >> 1) & 7] = max3(mxp[(j >> 1) & 7], x0, x1);
+                                }
                             }
                         }
-                    }
-                } else {
+                    } else {
 #pragma unroll
-                    for (int j = 0; j < 128; j += 2)
-                        mxp[(j >> 1) & 7] = max3(mxp[(j >> 1) & 7], __uint_as_float(sv[j]), __uint_as_float(sv[j + 1]));
-                }
-                const float mx = max3(max3(mxp[0], mxp[1], mxp[2]), max3(mxp[3], mxp[4], mxp[5]),
-                                      fmaxf(mxp[6], mxp[7]));
-                const float m_new = fmaxf(m, mx * C);
-                const bool raise = (c == 0) ? (m_new > m) : (m_new > m + 8.f);
-                float alpha = 1.f;
-                if (raise) {
-                    alpha = ex2(m - m_new);
-                    l *= alpha;
-                }
-                // rescale O in TMEM (warp-uniform: tcgen05.ld/st are .sync.aligned)
-                if (c > 0 && __any_sync(0xffffffffu, raise)) {
+                        for (int j = 0; j < 128; j += 2)
+                            mxp[(j >> 1) & 7] = max3(mxp[(j >> 1) & 7], __uint_as_float(sv[j]), __uint_as_float(sv[j + 1]));
+                    }
+                    return max3(max3(mxp[0], mxp[1], mxp[2]), max3(mxp[3], mxp[4], mxp[5]), fmaxf(mxp[6], mxp[7]));
+                };
+                // Raise the running max to cover mx (always on the first
+                // chunk, where m still holds the sink; later only when it grew
+                // by more than 2^8) and rescale l and O.  Returns whether any
+                // row of the warp raised.
+                auto raise_to = [&](float mx) -> bool {
+                    const float m_new = fmaxf(m, mx * C);
+                    const bool raise = (c == 0) ? (m_new > m) : (m_new > m + 8.f);
+                    float alpha = 1.f;
+                    if (raise) {
+                        alpha = ex2(m - m_new);
+                        l *= alpha;
+                    }
+                    const bool any = __any_sync(0xffffffffu, raise);
+                    // rescale O in TMEM (warp-uniform: tcgen05.ld/st are .sync.aligned)
+                    if (c > 0 && any) {
 #pragma unroll 1
-                    for (int b = 0; b < 8; ++b) {
-                        uint32_t v[16];
-                        tmem_ld16(t_o + 16u * b, v);
-                        tmem_wait_ld();
+                        for (int b = 0; b < 8; ++b) {
+                            uint32_t v[16];
+                            tmem_ld16(t_o + 16u * b, v);
+                            tmem_wait_ld();
 #pragma unroll
-                        for (int j = 0; j < 16; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) * alpha);
-                        tmem_st16(t_o + 16u * b, v);
-                    }
-                }
-                if (raise) m = m_new;
-                const float negm = (m == -INFINITY) ? 0.f : -m;
-                const uint64_t C2 = f2(C, C), negm2 = f2(negm, negm);
-                uint64_t lp[4];
-#pragma unroll
-                for (int k4 = 0; k4 < 4; ++k4) lp[k4] = 0ull;   // (+0.0f, +0.0f)
-                // Part of the pairs of an unmasked chunk go through the
-                // polynomial; masked chunks and infinite maxima keep ex2 so
-                // -inf maps to exactly 0.
-                const bool use_poly =
-                    __all_sync(0xffffffffu, !boundary && m > -INFINITY && m < INFINITY);
-                if (use_poly) {
-#pragma unroll
-                    for (int b = 0; b < 4; ++b) {
-                        uint32_t pk[16];
-#pragma unroll
-                        for (int j = 0; j < 16; ++j) {
-                            const uint64_t x = f2_fma(f2(__uint_as_float(sv[32 * b + 2 * j]),
-                                                         __uint_as_float(sv[32 * b + 2 * j + 1])), C2, negm2);
-                            uint64_t pp;
-                            if ((j & 7) < kPolyPairs) pp = exp2_poly2(x);
-                            else pp = f2(ex2(f2_lo(x)), ex2(f2_hi(x)));
-                            lp[j & 3] = f2_add(lp[j & 3], pp);
-                            pk[j] = pack_bf16(f2_lo(pp), f2_hi(pp));
+                            for (int j = 0; j < 16; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) * alpha);
+                            tmem_st16(t_o + 16u * b, v);
                         }
-                        tmem_st16(t_s + 16u * b, pk);
                     }
-                } else {
+                    if (raise) m = m_new;
+                    return any;
+                };
+                // P = 2^(s*C - m) -> BF16 into the first 64 columns of S;
+                // returns the row sum.  With `poly`, part of the pairs go
+                // through the polynomial (unmasked chunks and finite m only:
+                // ex2 keeps -inf -> exactly 0).
+                auto exp_chunk = [&](bool poly) -> float {
+                    const float negm = (m == -INFINITY) ? 0.f : -m;
+                    const uint64_t C2 = f2(C, C), negm2 = f2(negm, negm);
+                    uint64_t lp[4];
 #pragma unroll
-                    for (int b = 0; b < 4; ++b) {
-                        if (b < nblk) {
+                    for (int k4 = 0; k4 < 4; ++k4) lp[k4] = 0ull;   // (+0.0f, +0.0f)
+                    if (poly) {
+#pragma unroll
+                        for (int b = 0; b < 4; ++b) {
                             uint32_t pk[16];
 #pragma unroll
                             for (int j = 0; j < 16; ++j) {
                                 const uint64_t x = f2_fma(f2(__uint_as_float(sv[32 * b + 2 * j]),
                                                              __uint_as_float(sv[32 * b + 2 * j + 1])), C2, negm2);
-                                const uint64_t pp = f2(ex2(f2_lo(x)), ex2(f2_hi(x)));
+                                uint64_t pp;
+                                if ((j & 7) < kPolyPairs) pp = exp2_poly2(x);
+                                else pp = f2(ex2(f2_lo(x)), ex2(f2_hi(x)));
                                 lp[j & 3] = f2_add(lp[j & 3], pp);
                                 pk[j] = pack_bf16(f2_lo(pp), f2_hi(pp));
                             }
                             tmem_st16(t_s + 16u * b, pk);
                         }
+                    } else {
+#pragma unroll
+                        for (int b = 0; b < 4; ++b) {
+                            if (b < nblk) {
+                                uint32_t pk[16];
+#pragma unroll
+                                for (int j = 0; j < 16; ++j) {
+                                    const uint64_t x = f2_fma(f2(__uint_as_float(sv[32 * b + 2 * j]),
+                                                                 __uint_as_float(sv[32 * b + 2 * j + 1])), C2, negm2);
+                                    const uint64_t pp = f2(ex2(f2_lo(x)), ex2(f2_hi(x)));
+                                    lp[j & 3] = f2_add(lp[j & 3], pp);
+                                    pk[j] = pack_bf16(f2_lo(pp), f2_hi(pp));
+                                }
+                                tmem_st16(t_s + 16u * b, pk);
+                            }
+                        }
                     }
+                    const uint64_t ls = f2_add(f2_add(lp[0], lp[1]), f2_add(lp[2], lp[3]));
+                    return f2_lo(ls) + f2_hi(ls);
+                };
+                // Interior chunks after the first start without a row max:
+                // exponentials against the current m.  Every term is at most
+                // the row sum, so a sum within 2^8 keeps each term inside the
+                // lazy-rescale bound.  A larger sum (rare) takes a second
+                // pass with the exact max, which recomputes the chunk only if
+                // some row's max moved by more than 2^8.
+                bool need_max = !(c > 0 && __all_sync(0xffffffffu, !boundary && m > -INFINITY && m < INFINITY));
+                bool second = false;
+                float lsum = 0.f;
+#pragma unroll 1
+                for (;;) {
+                    if (need_max) {
+                        const bool any = raise_to(row_max(boundary));
+                        if (second && !any) break;             // first pass's P and sum stand
+                        if (second) tmem_wait_st();            // its P stores land before the new ones
+                    }
+                    lsum = exp_chunk(__all_sync(0xffffffffu, !boundary && m > -INFINITY && m < INFINITY));
+                    if (need_max || !__any_sync(0xffffffffu, !(lsum <= 256.f))) break;
+                    need_max = true;
+                    second = true;
                 }
-                const uint64_t ls = f2_add(f2_add(lp[0], lp[1]), f2_add(lp[2], lp[3]));
-                const float lsum = f2_lo(ls) + f2_hi(ls);
                 l += lsum;
                 tmem_wait_st();
                 tc_fence_before();
