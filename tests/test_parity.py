@@ -268,3 +268,22 @@ def test_out_may_alias_q(packed):
     torch.cuda.synchronize()
     assert torch.equal(o1.view(torch.int16), o2.view(torch.int16))
     assert torch.equal(l1, l2)
+
+
+@pytest.mark.parametrize("mix", [1.0, 0.35])
+def test_later_chunk_raises_the_max(mix):
+    """Keys 256..300 are aligned with query token 400 (mix = 1: the row max
+    jumps by far more than 2^8 in an interior chunk; mix = 0.35: the chunk's
+    terms sum past 2^8 while the max moves less), so the softmax's exact-max
+    second pass runs on interior chunks."""
+    T = 512
+    w = W.make_small(T, seed=18, window=0, use_rope=False)
+    q = W.bf16_to_f64(w.q)
+    k = W.bf16_to_f64(w.k)
+    rng = np.random.default_rng(19)
+    for g in range(4):
+        k[256:301, g] = mix * q[400, 8 * g] + (1.0 - mix) * rng.standard_normal((45, 128))
+    w.k = W.bf16_bits(k.astype(np.float32))
+    o, l = run_gpu(w)
+    rows = np.unique(np.concatenate([np.arange(380, 420), np.arange(0, 512, 7)]))
+    compare(w, o, l, rows=rows, tol=TOL_EDGE)
