@@ -459,31 +459,55 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 tmem_wait_ld();
                 const bool boundary = (c == nch - 1) || (ks + nc - 1 > tok0) ||
                                       (p.window > 0 && ks < tok0 + kTokPerTile - p.window);
+                // Row r sees columns jlo .. jhi of the chunk.  Each block of 32
+                // columns is, for the whole warp, either full (no mask),
+                // empty (P = 0, nothing to compute) or partial (masked per
+                // element); interior chunks are full.
+                const int jlo = lo - ks, jhi = min(i - ks, nc - 1);
+                uint32_t fullm = 0xFu, emptym = 0u;
+                if (boundary) {
+                    const int lo_max = __reduce_max_sync(0xffffffffu, jlo);
+                    const int lo_min = __reduce_min_sync(0xffffffffu, jlo);
+                    const int hi_max = __reduce_max_sync(0xffffffffu, jhi);
+                    const int hi_min = __reduce_min_sync(0xffffffffu, jhi);
+                    fullm = 0u;
+#pragma unroll
+                    for (int b = 0; b < 4; ++b) {
+                        if (lo_max <= 32 * b && hi_min >= 32 * b + 31) fullm |= 1u << b;
+                        else if (hi_max < 32 * b || lo_min > 32 * b + 31) emptym |= 1u << b;
+                    }
+                }
                 // row max over the S columns: 3-input max, 8 independent
                 // chains; masked columns become -inf in sv
-                auto row_max = [&](bool masked) -> float {
+                auto row_max_full = [&]() -> float {
                     float mxp[8];
 #pragma unroll
                     for (int k8 = 0; k8 < 8; ++k8) mxp[k8] = -INFINITY;
-                    if (masked) {
-                        const int jlo = lo - ks, jhi = i - ks;
 #pragma unroll
-                        for (int b = 0; b < 4; ++b) {
-                            if (b < nblk) {
+                    for (int j = 0; j < 128; j += 2)
+                        mxp[(j >> 1) & 7] = max3(mxp[(j >> 1) & 7], __uint_as_float(sv[j]), __uint_as_float(sv[j + 1]));
+                    return max3(max3(mxp[0], mxp[1], mxp[2]), max3(mxp[3], mxp[4], mxp[5]), fmaxf(mxp[6], mxp[7]));
+                };
+                auto row_max = [&]() -> float {
+                    float mxp[8];
 #pragma unroll
-                                for (int j = 32 * b; j < 32 * b + 32; j += 2) {
-                                    const float x0 = ((j >= jlo) && (j <= jhi)) ? __uint_as_float(sv[j]) : -INFINITY;
-                                    const float x1 = ((j + 1 >= jlo) && (j + 1 <= jhi)) ? __uint_as_float(sv[j + 1]) : -INFINITY;
-                                    sv[j] = __float_as_uint(x0);
-                                    sv[j + 1] = __float_as_uint(x1);
-                                    mxp[(j >> 1) & 7] = max3(mxp[(j >> 1) & 7], x0, x1);
-                                }
+                    for (int k8 = 0; k8 < 8; ++k8) mxp[k8] = -INFINITY;
+#pragma unroll
+                    for (int b = 0; b < 4; ++b) {
+                        if (fullm & (1u << b)) {
+#pragma unroll
+                            for (int j = 32 * b; j < 32 * b + 32; j += 2)
+                                mxp[(j >> 1) & 7] = max3(mxp[(j >> 1) & 7], __uint_as_float(sv[j]), __uint_as_float(sv[j + 1]));
+                        } else if (!(emptym & (1u << b))) {
+#pragma unroll
+                            for (int j = 32 * b; j < 32 * b + 32; j += 2) {
+                                const float x0 = ((j >= jlo) && (j <= jhi)) ? __uint_as_float(sv[j]) : -INFINITY;
+                                const float x1 = ((j + 1 >= jlo) && (j + 1 <= jhi)) ? __uint_as_float(sv[j + 1]) : -INFINITY;
+                                sv[j] = __float_as_uint(x0);
+                                sv[j + 1] = __float_as_uint(x1);
+                                mxp[(j >> 1) & 7] = max3(mxp[(j >> 1) & 7], x0, x1);
                             }
                         }
-                    } else {
-#pragma unroll
-                        for (int j = 0; j < 128; j += 2)
-                            mxp[(j >> 1) & 7] = max3(mxp[(j >> 1) & 7], __uint_as_float(sv[j]), __uint_as_float(sv[j + 1]));
                     }
                     return max3(max3(mxp[0], mxp[1], mxp[2]), max3(mxp[3], mxp[4], mxp[5]), fmaxf(mxp[6], mxp[7]));
                 };
@@ -516,10 +540,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     return any;
                 };
                 // P = 2^(s*C - m) -> BF16 into the first 64 columns of S;
-                // returns the row sum.  With `poly`, part of the pairs go
-                // through the polynomial (unmasked chunks and finite m only:
-                // ex2 keeps -inf -> exactly 0).
-                auto exp_chunk = [&](bool poly) -> float {
+                // returns the row sum.  Interior chunks: all 128 columns, and
+                // with `poly` (finite m) part of the pairs go through the
+                // polynomial.
+                auto exp_full = [&](bool poly) -> float {
                     const float negm = (m == -INFINITY) ? 0.f : -m;
                     const uint64_t C2 = f2(C, C), negm2 = f2(negm, negm);
                     uint64_t lp[4];
@@ -544,43 +568,75 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     } else {
 #pragma unroll
                         for (int b = 0; b < 4; ++b) {
-                            if (b < nblk) {
-                                uint32_t pk[16];
+                            uint32_t pk[16];
 #pragma unroll
-                                for (int j = 0; j < 16; ++j) {
-                                    const uint64_t x = f2_fma(f2(__uint_as_float(sv[32 * b + 2 * j]),
-                                                                 __uint_as_float(sv[32 * b + 2 * j + 1])), C2, negm2);
-                                    const uint64_t pp = f2(ex2(f2_lo(x)), ex2(f2_hi(x)));
-                                    lp[j & 3] = f2_add(lp[j & 3], pp);
-                                    pk[j] = pack_bf16(f2_lo(pp), f2_hi(pp));
-                                }
-                                tmem_st16(t_s + 16u * b, pk);
+                            for (int j = 0; j < 16; ++j) {
+                                const uint64_t x = f2_fma(f2(__uint_as_float(sv[32 * b + 2 * j]),
+                                                             __uint_as_float(sv[32 * b + 2 * j + 1])), C2, negm2);
+                                const uint64_t pp = f2(ex2(f2_lo(x)), ex2(f2_hi(x)));
+                                lp[j & 3] = f2_add(lp[j & 3], pp);
+                                pk[j] = pack_bf16(f2_lo(pp), f2_hi(pp));
                             }
+                            tmem_st16(t_s + 16u * b, pk);
                         }
                     }
                     const uint64_t ls = f2_add(f2_add(lp[0], lp[1]), f2_add(lp[2], lp[3]));
                     return f2_lo(ls) + f2_hi(ls);
                 };
-                // Interior chunks after the first start without a row max:
-                // exponentials against the current m.  Every term is at most
-                // the row sum, so a sum within 2^8 keeps each term inside the
-                // lazy-rescale bound.  A larger sum (rare) takes a second
-                // pass with the exact max, which recomputes the chunk only if
-                // some row's max moved by more than 2^8.
-                bool need_max = !(c > 0 && __all_sync(0xffffffffu, !boundary && m > -INFINITY && m < INFINITY));
-                bool second = false;
-                float lsum = 0.f;
-#pragma unroll 1
-                for (;;) {
-                    if (need_max) {
-                        const bool any = raise_to(row_max(boundary));
-                        if (second && !any) break;             // first pass's P and sum stand
-                        if (second) tmem_wait_st();            // its P stores land before the new ones
+                // Masked chunks: full blocks as above, partial blocks with ex2
+                // (the masked -inf maps to exactly 0), empty blocks store zeros.
+                auto exp_blocks = [&]() -> float {
+                    const float negm = (m == -INFINITY) ? 0.f : -m;
+                    const uint64_t C2 = f2(C, C), negm2 = f2(negm, negm);
+                    uint64_t lp[4];
+#pragma unroll
+                    for (int k4 = 0; k4 < 4; ++k4) lp[k4] = 0ull;   // (+0.0f, +0.0f)
+#pragma unroll
+                    for (int b = 0; b < 4; ++b) {
+                        uint32_t pk[16];
+                        if (emptym & (1u << b)) {
+#pragma unroll
+                            for (int j = 0; j < 16; ++j) pk[j] = 0u;
+                        } else {
+#pragma unroll
+                            for (int j = 0; j < 16; ++j) {
+                                const uint64_t x = f2_fma(f2(__uint_as_float(sv[32 * b + 2 * j]),
+                                                             __uint_as_float(sv[32 * b + 2 * j + 1])), C2, negm2);
+                                const uint64_t pp = f2(ex2(f2_lo(x)), ex2(f2_hi(x)));
+                                lp[j & 3] = f2_add(lp[j & 3], pp);
+                                pk[j] = pack_bf16(f2_lo(pp), f2_hi(pp));
+                            }
+                        }
+                        if (b < nblk) tmem_st16(t_s + 16u * b, pk);
                     }
-                    lsum = exp_chunk(__all_sync(0xffffffffu, !boundary && m > -INFINITY && m < INFINITY));
-                    if (need_max || !__any_sync(0xffffffffu, !(lsum <= 256.f))) break;
-                    need_max = true;
-                    second = true;
+                    const uint64_t ls = f2_add(f2_add(lp[0], lp[1]), f2_add(lp[2], lp[3]));
+                    return f2_lo(ls) + f2_hi(ls);
+                };
+                float lsum = 0.f;
+                if (!boundary) {
+                    // Interior chunks after the first start without a row
+                    // max: exponentials against the current m.  Every term is
+                    // at most the row sum, so a sum within 2^8 keeps each term
+                    // inside the lazy-rescale bound.  A larger sum (rare)
+                    // takes a second pass with the exact max, which recomputes
+                    // the chunk only if some row's max moved by more than 2^8.
+                    bool need_max = !(c > 0 && __all_sync(0xffffffffu, m > -INFINITY && m < INFINITY));
+                    bool second = false;
+#pragma unroll 1
+                    for (;;) {
+                        if (need_max) {
+                            const bool any = raise_to(row_max_full());
+                            if (second && !any) break;         // first pass's P and sum stand
+                            if (second) tmem_wait_st();        // its P stores land before the new ones
+                        }
+                        lsum = exp_full(__all_sync(0xffffffffu, m > -INFINITY && m < INFINITY));
+                        if (need_max || !__any_sync(0xffffffffu, !(lsum <= 256.f))) break;
+                        need_max = true;
+                        second = true;
+                    }
+                } else {
+                    raise_to(row_max());
+                    lsum = exp_blocks();
                 }
                 l += lsum;
                 tmem_wait_st();
