@@ -450,15 +450,22 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 if (!ok) { alive = false; break; }
                 s_ph ^= 1;
                 tc_fence_after();
-                // all S columns of this chunk: one TMEM load per 32 columns,
-                // a single wait
-                uint32_t sv[128];
-#pragma unroll
-                for (int b = 0; b < 4; ++b)
-                    if (b < nblk) tmem_ld32(t_s + 32u * b, sv + 32 * b);
-                tmem_wait_ld();
                 const bool boundary = (c == nch - 1) || (ks + nc - 1 > tok0) ||
                                       (p.window > 0 && ks < tok0 + kTokPerTile - p.window);
+                // Interior chunks after the first with a finite running max
+                // take the fast path below (no row max).
+                const bool fastp =
+                    !boundary && c > 0 && __all_sync(0xffffffffu, m > -INFINITY && m < INFINITY);
+                // S columns of this chunk, one TMEM load per 32 columns.  On
+                // the fast path the exponentials of columns 0..63 overlap the
+                // load of columns 64..127.
+                uint32_t sv[128];
+                tmem_ld32(t_s, sv);
+                if (nblk > 1) tmem_ld32(t_s + 32u, sv + 32);
+                if (fastp) tmem_wait_ld();
+                if (nblk > 2) tmem_ld32(t_s + 64u, sv + 64);
+                if (nblk > 3) tmem_ld32(t_s + 96u, sv + 96);
+                if (!fastp) tmem_wait_ld();
                 // Row r sees columns jlo .. jhi of the chunk.  Each block of 32
                 // columns is, for the whole warp, either full (no mask),
                 // empty (P = 0, nothing to compute) or partial (masked per
@@ -583,6 +590,30 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     const uint64_t ls = f2_add(f2_add(lp[0], lp[1]), f2_add(lp[2], lp[3]));
                     return f2_lo(ls) + f2_hi(ls);
                 };
+                // Blocks b0 .. b1-1 with the polynomial share (unmasked, finite m).
+                auto exp_part = [&](const int b0, const int b1) -> float {
+                    const uint64_t C2 = f2(C, C), negm2 = f2(-m, -m);
+                    uint64_t lp[4];
+#pragma unroll
+                    for (int k4 = 0; k4 < 4; ++k4) lp[k4] = 0ull;   // (+0.0f, +0.0f)
+#pragma unroll
+                    for (int b = b0; b < b1; ++b) {
+                        uint32_t pk[16];
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) {
+                            const uint64_t x = f2_fma(f2(__uint_as_float(sv[32 * b + 2 * j]),
+                                                         __uint_as_float(sv[32 * b + 2 * j + 1])), C2, negm2);
+                            uint64_t pp;
+                            if ((j & 7) < kPolyPairs) pp = exp2_poly2(x);
+                            else pp = f2(ex2(f2_lo(x)), ex2(f2_hi(x)));
+                            lp[j & 3] = f2_add(lp[j & 3], pp);
+                            pk[j] = pack_bf16(f2_lo(pp), f2_hi(pp));
+                        }
+                        tmem_st16(t_s + 16u * b, pk);
+                    }
+                    const uint64_t ls = f2_add(f2_add(lp[0], lp[1]), f2_add(lp[2], lp[3]));
+                    return f2_lo(ls) + f2_hi(ls);
+                };
                 // Masked chunks: full blocks as above, partial blocks with ex2
                 // (the masked -inf maps to exactly 0), empty blocks store zeros.
                 auto exp_blocks = [&]() -> float {
@@ -613,27 +644,25 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     return f2_lo(ls) + f2_hi(ls);
                 };
                 float lsum = 0.f;
-                if (!boundary) {
-                    // Interior chunks after the first start without a row
-                    // max: exponentials against the current m.  Every term is
-                    // at most the row sum, so a sum within 2^8 keeps each term
-                    // inside the lazy-rescale bound.  A larger sum (rare)
-                    // takes a second pass with the exact max, which recomputes
-                    // the chunk only if some row's max moved by more than 2^8.
-                    bool need_max = !(c > 0 && __all_sync(0xffffffffu, m > -INFINITY && m < INFINITY));
-                    bool second = false;
+                if (fastp) {
+                    // Exponentials against the current m without a row max.
+                    // Every term is at most the row sum, so a sum within 2^8
+                    // keeps each term inside the lazy-rescale bound.  A larger
+                    // sum (rare) takes the exact max and, if some row's max
+                    // moved by more than 2^8, rescales and recomputes.
 #pragma unroll 1
-                    for (;;) {
-                        if (need_max) {
-                            const bool any = raise_to(row_max_full());
-                            if (second && !any) break;         // first pass's P and sum stand
-                            if (second) tmem_wait_st();        // its P stores land before the new ones
-                        }
-                        lsum = exp_full(__all_sync(0xffffffffu, m > -INFINITY && m < INFINITY));
-                        if (need_max || !__any_sync(0xffffffffu, !(lsum <= 256.f))) break;
-                        need_max = true;
-                        second = true;
+                    for (int attempt = 0; attempt < 2; ++attempt) {
+                        lsum = exp_part(0, 2);
+                        tmem_wait_ld();                    // columns 64..127 (no-op when recomputing)
+                        lsum += exp_part(2, 4);
+                        if (attempt == 1 || !__any_sync(0xffffffffu, !(lsum <= 256.f))) break;
+                        if (!raise_to(row_max_full())) break;   // first attempt stands
+                        tmem_wait_st();                    // its P stores land before the new ones
                     }
+                } else if (!boundary) {
+                    // first chunk (m still holds the sink) or infinite max
+                    raise_to(row_max_full());
+                    lsum = exp_full(__all_sync(0xffffffffu, m > -INFINITY && m < INFINITY));
                 } else {
                     raise_to(row_max());
                     lsum = exp_blocks();
