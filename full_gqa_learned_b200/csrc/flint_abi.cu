@@ -256,8 +256,24 @@ flint_status_t run_stages(int stages, const void* q, const void* k, const void* 
     ap.eps = eps;
     const int max_units = L.max_items * kHKV;
     const int grid = max_units < sms ? max_units : sms;
-    attn_fwd_kernel<<<grid, kAttnThreads, kAttnSmemBytes, s>>>(tm_q, tm_k, tm_v, tm_o, tm_o1, ap);
-    e = cudaGetLastError();
+    if (stages & kStagePrepare) {
+        // launched right behind the preparation kernel: a programmatic
+        // dependent, so its setup overlaps the preparation kernel's tail
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(grid);
+        cfg.blockDim = dim3(kAttnThreads);
+        cfg.dynamicSmemBytes = kAttnSmemBytes;
+        cfg.stream = s;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        e = cudaLaunchKernelEx(&cfg, attn_fwd_kernel, tm_q, tm_k, tm_v, tm_o, tm_o1, ap);
+    } else {
+        attn_fwd_kernel<<<grid, kAttnThreads, kAttnSmemBytes, s>>>(tm_q, tm_k, tm_v, tm_o, tm_o1, ap);
+        e = cudaGetLastError();
+    }
     if (e != cudaSuccess) return fail(FLINT_ERR_CUDA, "attention launch: %s", cudaGetErrorString(e));
     return FLINT_OK;
 }

@@ -214,6 +214,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             misc->logit_scale = ldexpf(1.4426950408889634f * 0.08838834764831845f, -(eq + ek));
         }
     }
+    // everything above overlaps the tail of the preparation kernel; the work
+    // plan and the prepared keys and queries are read only after it completed
+    griddep_wait();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();

@@ -16,6 +16,7 @@
 // get their final outputs here: zeros and lse = sink (FlintAttention.forward,
 // attention_mask: the sink remains valid for padded queries).
 #include "flint_common.cuh"
+#include "sm100.cuh"
 
 namespace flint {
 
@@ -326,6 +327,12 @@ __device__ void prepare_tokens(const PrepParams& p) {
 }
 
 __global__ void __launch_bounds__(1024, 1) prep_kernel(PrepParams p) {
+    // The attention kernel may be scheduled as soon as every block of this
+    // grid has started (it is launched as a programmatic dependent and waits
+    // for this grid's completion before it reads anything written here).
+    // Blocks trigger on entry, so by the time the attention kernel can take
+    // an SM, no block of this grid is still waiting for one.
+    griddep_launch_dependents();
     if (blockIdx.x == 0) build_plan(p);
     else prepare_tokens(p);
 }
