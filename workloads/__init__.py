@@ -288,3 +288,79 @@ def make_small(T, seed, *, window=0, use_rope=False, cu_seqlens=None,
     return Workload(name, q, k, v, wq, wk, s, pos_ids=pos_ids,
                     cu_seqlens=None if cu_seqlens is None else np.asarray(cu_seqlens, np.int32),
                     pad_mask=pad_mask, window=window, use_rope=use_rope, seed=seed)
+
+
+@dataclasses.dataclass
+class DecodeWorkload:
+    """One decode step for B sequences: the new token's projections and a
+    key/value cache of capacity cap (position j in slot j mod cap).  Cached
+    keys stand in for normalised, rotated keys (N(0,1) BF16); values are
+    N(0,1) BF16 like v."""
+    name: str
+    q: np.ndarray          # uint16 [B,32,128]
+    k: np.ndarray          # uint16 [B,4,128]
+    v: np.ndarray          # uint16 [B,4,128]
+    k_cache: np.ndarray    # uint16 [B,cap,4,128]
+    v_cache: np.ndarray    # uint16 [B,cap,4,128]
+    cache_len: np.ndarray  # int32 [B]: position of the new token
+    q_norm_w: np.ndarray
+    k_norm_w: np.ndarray
+    sinks: np.ndarray
+    window: int
+    use_rope: bool
+    rope_theta: float = ROPE_THETA
+    eps: float = EPS
+
+    @property
+    def B(self) -> int:
+        return int(self.q.shape[0])
+
+    @property
+    def cap(self) -> int:
+        return int(self.k_cache.shape[1])
+
+    def keys_per_sequence(self) -> np.ndarray:
+        """Keys each new token attends to (its window, itself included)."""
+        n = self.cache_len.astype(np.int64) + 1
+        return np.minimum(n, self.window) if self.window > 0 else n
+
+    def flops(self) -> float:
+        return float(4 * D * HQ * self.keys_per_sequence().sum())
+
+    def algorithmic_bytes(self) -> float:
+        """Window keys and values read once per KV head, the new token's q, k,
+        v read, its cache slot, out and lse written."""
+        kv = 2 * HKV * D * 2 * self.keys_per_sequence().sum()
+        return float(kv + self.B * (HQ * D * 2 + 2 * HKV * D * 2 + 2 * HKV * D * 2 + HQ * D * 2 + HQ * 4))
+
+
+def make_decode(B, cap, seed, *, window, use_rope, max_len, min_len=0, name="decode",
+                sinks=None) -> DecodeWorkload:
+    """Seeded decode step: cache lengths uniform in [min_len, max_len)."""
+    rng = np.random.default_rng(seed)
+    q = bf16_bits(_normal(rng, (B, HQ, D), 1.0))
+    k = bf16_bits(_normal(rng, (B, HKV, D), 1.0))
+    v = bf16_bits(_normal(rng, (B, HKV, D), 1.0))
+    wq = (1.0 + 0.1 * rng.standard_normal(D)).astype(np.float32)
+    wk = (1.0 + 0.1 * rng.standard_normal(D)).astype(np.float32)
+    s = rng.standard_normal(HQ).astype(np.float32)
+    if sinks is not None:
+        s = np.broadcast_to(np.asarray(sinks, dtype=np.float32), (HQ,)).copy()
+    kc = bf16_bits(_normal(rng, (B, cap, HKV, D), 1.0))
+    vc = bf16_bits(_normal(rng, (B, cap, HKV, D), 1.0))
+    cache_len = rng.integers(min_len, max_len, size=B).astype(np.int32)
+    return DecodeWorkload(name, q, k, v, kc, vc, cache_len, wq, wk, s, window=window, use_rope=use_rope)
+
+
+# decode steps: a batch of sequences deep into a 262,144-token context on a
+# sliding layer (ring cache of 513), and a full layer with a 4,096-token cache
+DECODE_CONFIGS = {
+    "decode_sliding_b128": dict(B=128, cap=513, seed=5, window=513, use_rope=True,
+                                max_len=262144, min_len=513),
+    "decode_full_b64_s4096": dict(B=64, cap=4096, seed=6, window=0, use_rope=False,
+                                  max_len=4096, min_len=1),
+}
+
+
+def make_decode_named(name: str) -> DecodeWorkload:
+    return make_decode(name=name, **DECODE_CONFIGS[name])
