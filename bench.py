@@ -340,12 +340,110 @@ def cpu_baseline(w, budget_s, nthreads=0):
                 (len(rows), w.T, w.name, dt))
 
 
+DECODE_METRIC = "decode step: algorithmic HBM bytes per second (window keys and values once)"
+
+
+def run_decode(args, rank, world, local_rank):
+    """One decode step per timed step (flint_attn_decode), L2 flushed before
+    each; the step rewrites the same cache slot with the same values, so
+    repeating it is idempotent."""
+    import torch
+    import full_gqa_learned_b200 as fa
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    d = W.make_decode_named(args.workload)
+
+    def bf(x):
+        return torch.from_numpy(np.ascontiguousarray(x)).view(torch.bfloat16).to(dev)
+    t = dict(q=bf(d.q), k=bf(d.k), v=bf(d.v), k_cache=bf(d.k_cache), v_cache=bf(d.v_cache),
+             cache_len=torch.from_numpy(d.cache_len).to(dev), q_norm_w=torch.from_numpy(d.q_norm_w).to(dev),
+             k_norm_w=torch.from_numpy(d.k_norm_w).to(dev),
+             sinks=torch.from_numpy(np.ascontiguousarray(d.sinks, np.float32)).to(dev))
+    out = torch.empty((d.B, 4096), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((32, d.B), dtype=torch.float32, device=dev)
+    ws = torch.empty(fa.decode_workspace_bytes(d.B, d.cap, d.window), dtype=torch.uint8, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        fa.attn_decode(t["q"], t["k"], t["v"], t["q_norm_w"], t["k_norm_w"], t["sinks"], t["k_cache"],
+                       t["v_cache"], t["cache_len"], window=d.window, use_rope=d.use_rope,
+                       rope_theta=d.rope_theta, eps=d.eps, out=out, lse=lse, workspace=ws, stream=stream)
+    for _ in range(args.warmup):
+        flush.fill_(1)
+        step()
+    st = fa.device_status(ws)
+    if st != 0:
+        raise RuntimeError("device status %s" % fa.STATUS.get(st, st))
+    sampler = ClockSampler(local_rank if "CUDA_VISIBLE_DEVICES" not in os.environ else
+                           os.environ["CUDA_VISIBLE_DEVICES"].split(",")[local_rank])
+    sampler.start()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    for i in range(args.steps):
+        flush.fill_(i & 0xFF)
+        evs[i][0].record(stream)
+        step()
+        evs[i][1].record(stream)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+    total_ms = sum(e[0].elapsed_time(e[1]) for e in evs)
+    (total_ms,) = max_over_ranks([total_ms], device=dev)
+    return d, total_ms, clocks
+
+
+def decode_cpu_baseline(d, budget_s):
+    """The decode oracle, as it stands, on the first sequences of the step
+    (about budget_s seconds of single-threaded numpy): algorithmic bytes of
+    those sequences per second."""
+    import oracle.decode as OD
+    t0 = time.time()
+    n = 0
+    for b in range(d.B):
+        OD.decode_step(d.q[b:b + 1], d.k[b:b + 1], d.v[b:b + 1], d.k_cache[b:b + 1], d.v_cache[b:b + 1],
+                       d.cache_len[b:b + 1], d.q_norm_w, d.k_norm_w, d.sinks, window=d.window,
+                       use_rope=d.use_rope)
+        n = b + 1
+        if time.time() - t0 > budget_s:
+            break
+    dt = time.time() - t0
+    frac = n / d.B
+    return dict(value=d.algorithmic_bytes() * frac / dt / 1e9, unit="GB/s", cores=1, kind="oracle",
+                sample="%d of %d sequences of %s, %.1f s" % (n, d.B, d.name, dt))
+
+
+def decode_line(args, world, d, total_ms, clocks):
+    peaks, src = load_peaks()
+    peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    nbytes = d.algorithmic_bytes()
+    step_ms = total_ms / args.steps
+    gbs = nbytes / (step_ms * 1e-3) / 1e9
+    return dict(
+        metric=DECODE_METRIC, value=round(gbs * world, 3), unit="GB/s", n_gpus=world, steps=args.steps,
+        warmup=args.warmup, ms_per_step=round(step_ms, 5), higher_is_better=True, scaling="weak",
+        vs_baseline=None, dtype="f32", data="synthetic (seeded N(0,1) BF16 q/k/v and caches)",
+        config=dict(workload=d.name, B=d.B, cap=d.cap, window=d.window, use_rope=bool(d.use_rope),
+                    keys=int(d.keys_per_sequence().sum()), l2="flushed before every timed step (256 MiB write)",
+                    per_rank="independent replica"),
+        roofline=dict(bound="hbm", achieved=round(gbs, 3), peak=peak, unit="GB/s", frac=round(gbs / peak, 4),
+                      traffic=None, kernel="flint::decode_split_kernel + decode_combine_kernel (whole step)",
+                      peak_source="%s hbm_gbs" % src, bytes_per_step=nbytes),
+        gpu_launches=2 * args.steps, clocks=clocks)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=10)
-    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(W.CONFIGS))
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD,
+                    choices=sorted(W.CONFIGS) + sorted(W.DECODE_CONFIGS))
     ap.add_argument("--impl", default="flint", choices=["flint", "reference"])
     ap.add_argument("--soak", type=float, default=1.0, help="seconds of untimed load before timing")
     ap.add_argument("--cpu-budget", type=float, default=12.0)
@@ -364,6 +462,24 @@ def main():
 
     if args.impl == "reference":
         if rank != 0:
+            return 0
+        if args.workload in W.DECODE_CONFIGS:
+            d = W.make_decode_named(args.workload)
+            vals, cb = [], None
+            for i in range(args.warmup + args.steps):
+                cb = decode_cpu_baseline(d, budget_s=min(args.cpu_budget, 60.0 / max(1, args.steps + args.warmup)))
+                if i >= args.warmup:
+                    vals.append(cb["value"])
+            value = statistics.median(vals)
+            cb["value"] = value
+            print(json.dumps(dict(impl="reference", metric=DECODE_METRIC, value=value, unit="GB/s",
+                                  n_gpus=args.gpus, steps=args.steps, warmup=args.warmup, ms_per_step=None,
+                                  higher_is_better=True, scaling="weak", vs_baseline=None, dtype="f64",
+                                  data="synthetic", config=dict(workload=d.name, B=d.B, cap=d.cap,
+                                                                window=d.window, use_rope=d.use_rope),
+                                  cpu_baseline=cb,
+                                  e2e=dict(value=value, unit="GB/s", h2d_bytes_per_step=0,
+                                           d2h_bytes_per_step=0))))
             return 0
         w = W.make(args.workload)
         times, cb = [], None
@@ -391,10 +507,18 @@ def main():
         from datetime import timedelta
         dist.init_process_group("nccl", timeout=timedelta(seconds=120),
                                 device_id=torch.device("cuda", local_rank))
-    try:
-        r = run_flint(args, rank, world, local_rank)
-    finally:
-        pass
+    if args.workload in W.DECODE_CONFIGS:
+        d, total_ms, clocks = run_decode(args, rank, world, local_rank)
+        line = decode_line(args, world, d, total_ms, clocks)
+        if rank == 0 and world == 1 and not args.profile:
+            line["cpu_baseline"] = decode_cpu_baseline(d, budget_s=args.cpu_budget)
+        if world > 1:
+            dist.barrier()
+            dist.destroy_process_group()
+        if rank == 0:
+            print(json.dumps(line))
+        return 0
+    r = run_flint(args, rank, world, local_rank)
     w = r["w"]
     peaks, src = load_peaks()
     flops = w.flops()

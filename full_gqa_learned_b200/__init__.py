@@ -16,7 +16,8 @@ import os
 import threading
 from typing import Optional, Tuple
 
-__all__ = ["attn_fwd", "attn_fwd_static", "workspace_bytes", "device_status", "load_library",
+__all__ = ["attn_fwd", "attn_fwd_static", "attn_decode", "workspace_bytes", "decode_workspace_bytes",
+           "device_status", "load_library",
            "FlintError", "LIB_PATH", "HQ", "HKV", "HEAD_DIM", "STATUS", "STATIC_SCRATCH_BYTES"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -58,6 +59,11 @@ def load_library() -> ctypes.CDLL:
             getattr(lib, name).argtypes = fwd_args
         lib.flint_attn_fwd_static.restype = ctypes.c_int
         lib.flint_attn_fwd_static.argtypes = fwd_args[:19] + [P]
+        lib.flint_attn_decode_workspace_bytes.restype = ctypes.c_size_t
+        lib.flint_attn_decode_workspace_bytes.argtypes = [I32, I32, I32]
+        lib.flint_attn_decode.restype = ctypes.c_int
+        lib.flint_attn_decode.argtypes = [P, P, P, P, P, P, P, P, P, I32, I32, I32, I32, F32, F32,
+                                          P, P, P, ctypes.c_size_t, P]
         lib.flint_attn_device_status.restype = ctypes.c_int
         lib.flint_attn_device_status.argtypes = [P, P]
         lib.flint_attn_last_error.restype = ctypes.c_char_p
@@ -153,6 +159,61 @@ def attn_fwd(q, k, v, q_norm_w, k_norm_w, sinks, *, pos_ids=None, cu_seqlens=Non
     if st != 0:
         raise FlintError(st, lib.flint_attn_last_error().decode())
     attn_fwd.last_workspace = workspace
+    return out, lse
+
+
+def decode_workspace_bytes(B: int, cap: int, window: int) -> int:
+    return int(load_library().flint_attn_decode_workspace_bytes(int(B), int(cap), int(window)))
+
+
+def attn_decode(q, k, v, q_norm_w, k_norm_w, sinks, k_cache, v_cache, cache_len, *,
+                window: int = 513, use_rope: bool = True, rope_theta: float = 10000.0,
+                eps: float = 1e-6, out=None, lse=None, workspace=None, stream=None,
+                want_lse: bool = True) -> Tuple[object, object]:
+    """One decode step (see include/flint_attn.h, flint_attn_decode).
+
+    q [B,32,128], k/v [B,4,128] bf16: the new token of each sequence;
+    k_cache, v_cache [B,cap,4,128] bf16 (position j in slot j mod cap; the
+    step writes the new token into slot cache_len[b] mod cap); cache_len [B]
+    int32.  Returns (out [B,4096] bf16, lse [32,B] f32 or None).
+    """
+    import torch
+    lib = load_library()
+    B = int(q.shape[0]) if q.dim() >= 1 else 0
+    cap = int(k_cache.shape[1]) if k_cache.dim() >= 2 else 0
+    _check(q, "q", torch.bfloat16, (B, HQ, HEAD_DIM))
+    _check(k, "k", torch.bfloat16, (B, HKV, HEAD_DIM))
+    _check(v, "v", torch.bfloat16, (B, HKV, HEAD_DIM))
+    _check(q_norm_w, "q_norm_w", torch.float32, (HEAD_DIM,))
+    _check(k_norm_w, "k_norm_w", torch.float32, (HEAD_DIM,))
+    _check(sinks, "sinks", torch.float32, (HQ,))
+    _check(k_cache, "k_cache", torch.bfloat16, (B, cap, HKV, HEAD_DIM))
+    _check(v_cache, "v_cache", torch.bfloat16, (B, cap, HKV, HEAD_DIM))
+    _check(cache_len, "cache_len", torch.int32, (B,))
+    dev = q.device
+    if out is None:
+        out = torch.empty((B, HQ * HEAD_DIM), dtype=torch.bfloat16, device=dev)
+    _check(out, "out", torch.bfloat16, (B, HQ * HEAD_DIM))
+    if lse is None and want_lse:
+        lse = torch.empty((HQ, B), dtype=torch.float32, device=dev)
+    if lse is not None:
+        _check(lse, "lse", torch.float32, (HQ, B))
+    need = decode_workspace_bytes(B, max(cap, 1), window)
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
+    _check(workspace, "workspace", torch.uint8)
+    if stream is None:
+        stream = torch.cuda.current_stream(dev)
+    sptr = stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+    with torch.cuda.device(dev):
+        st = lib.flint_attn_decode(
+            _ptr(q), _ptr(k), _ptr(v), _ptr(q_norm_w), _ptr(k_norm_w), _ptr(sinks), _ptr(k_cache),
+            _ptr(v_cache), _ptr(cache_len), B, cap, int(window), int(bool(use_rope)),
+            float(rope_theta), float(eps), _ptr(out), _ptr(lse), _ptr(workspace),
+            int(workspace.numel()), sptr)
+    if st != 0:
+        raise FlintError(st, lib.flint_attn_last_error().decode())
+    attn_decode.last_workspace = workspace
     return out, lse
 
 

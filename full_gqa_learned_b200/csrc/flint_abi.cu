@@ -280,6 +280,13 @@ flint_status_t run_stages(int stages, const void* q, const void* k, const void* 
 
 flint_status_t set_error(flint_status_t s, const char* msg) { return fail(s, "%s", msg); }
 
+size_t decode_workspace_bytes(int B, int cap, int window);
+flint_status_t run_decode(const void* q, const void* k, const void* v, const float* q_norm_w,
+                          const float* k_norm_w, const float* sinks, void* k_cache, void* v_cache,
+                          const int32_t* cache_len, int32_t B, int32_t cap, int32_t window,
+                          int32_t use_rope, float rope_theta, float eps, void* out, float* lse,
+                          void* workspace, size_t workspace_bytes, void* stream);
+
 }  // namespace flint
 
 extern "C" {
@@ -297,6 +304,48 @@ extern "C" {
 flint_status_t flint_attn_fwd(FLINT_ARGS) { return run_stages(kStageBoth, FLINT_FWD_ARGS); }
 flint_status_t flint_attn_prepare(FLINT_ARGS) { return run_stages(kStagePrepare, FLINT_FWD_ARGS); }
 flint_status_t flint_attn_attend(FLINT_ARGS) { return run_stages(kStageAttend, FLINT_FWD_ARGS); }
+
+size_t flint_attn_decode_workspace_bytes(int32_t B, int32_t cap, int32_t window) {
+    if (B < 0 || B > FLINT_MAX_DECODE_BATCH || cap < 1 || cap > FLINT_MAX_TOKENS || window < 0) return 0;
+    return flint::decode_workspace_bytes(B, cap, window);
+}
+
+flint_status_t flint_attn_decode(const void* q, const void* k, const void* v, const float* q_norm_w,
+                                 const float* k_norm_w, const float* sinks, void* k_cache,
+                                 void* v_cache, const int32_t* cache_len, int32_t B, int32_t cap,
+                                 int32_t window, int32_t use_rope, float rope_theta, float eps,
+                                 void* out, float* lse, void* workspace, size_t workspace_bytes,
+                                 void* stream) {
+    g_err[0] = '\0';
+    if (B < 0 || B > FLINT_MAX_DECODE_BATCH)
+        return fail(FLINT_ERR_INVALID_ARG, "B=%d outside [0, %d]", B, FLINT_MAX_DECODE_BATCH);
+    if (cap < 1 || cap > FLINT_MAX_TOKENS) return fail(FLINT_ERR_INVALID_ARG, "cap=%d", cap);
+    if (window < 0) return fail(FLINT_ERR_INVALID_ARG, "window=%d < 0", window);
+    if (use_rope != 0 && use_rope != 1) return fail(FLINT_ERR_INVALID_ARG, "use_rope must be 0 or 1");
+    if (!(eps > 0.f) || !std::isfinite(eps)) return fail(FLINT_ERR_INVALID_ARG, "eps must be > 0");
+    if (use_rope && (!(rope_theta > 1.f) || !std::isfinite(rope_theta)))
+        return fail(FLINT_ERR_INVALID_ARG, "rope_theta must be > 1");
+    if (B == 0) return FLINT_OK;
+    if (!q || !k || !v || !q_norm_w || !k_norm_w || !sinks || !k_cache || !v_cache || !cache_len || !out)
+        return fail(FLINT_ERR_INVALID_ARG, "null tensor pointer");
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(k_cache, 16) ||
+        !aligned(v_cache, 16) || !aligned(out, 16))
+        return fail(FLINT_ERR_INVALID_ARG, "q, k, v, the caches and out must be 16-byte aligned");
+    if (!aligned(q_norm_w, 4) || !aligned(k_norm_w, 4) || !aligned(sinks, 4) || !aligned(cache_len, 4) ||
+        (lse && !aligned(lse, 4)))
+        return fail(FLINT_ERR_INVALID_ARG, "misaligned 32-bit array");
+    const size_t need = flint::decode_workspace_bytes(B, cap, window);
+    if (!workspace || !aligned(workspace, 256))
+        return fail(FLINT_ERR_WORKSPACE, "workspace missing or not 256-byte aligned");
+    if (workspace_bytes < need)
+        return fail(FLINT_ERR_WORKSPACE, "workspace too small: %zu < %zu bytes", workspace_bytes, need);
+    int sms = 0;
+    flint_status_t st = device_setup(&sms);
+    if (st != FLINT_OK) return st;
+    return flint::run_decode(q, k, v, q_norm_w, k_norm_w, sinks, k_cache, v_cache, cache_len, B, cap,
+                             window, use_rope, rope_theta, eps, out, lse, workspace, workspace_bytes,
+                             stream);
+}
 
 flint_status_t flint_attn_device_status(const void* workspace, void* stream) {
     if (!workspace) return fail(FLINT_ERR_WORKSPACE, "workspace is null");

@@ -1,0 +1,326 @@
+// One decode step of the sink-aware GQA attention against a key/value cache
+// (sm_100a, CUDA cores: the step reads each cached key and value once and is
+// bound by memory, not by the tensor cores).
+//
+// Sequence b's new token sits at position p = cache_len[b].  Its queries and
+// key get the prologue of FlintAttention.forward (NeMo AutoModel
+// "flint.layers" API page): per-head RMSNorm in weight form, then NeoX RoPE at
+// p on sliding layers.  It attends to the keys of positions lo .. p (lo =
+// max(0, p - W + 1) on a sliding layer, the window counting the current
+// token; 0 on a full layer) and to the learned sink, a zero-value softmax
+// column in natural-logit units (HF discussion #26 on RecursiveSI/flint).
+// Position j lives in cache slot j mod cap, so a cache of capacity >= W is a
+// ring on sliding layers (the "flint" model page: a hybrid KV cache must
+// honour per-layer window sizes).  The step appends the new token: its
+// normalised, rotated key (rounded to BF16) and its value go to slot p mod cap.
+//
+// Split-KV: CTA (s, g, b) takes keys lo + 128 s .. lo + 128 s + 127 of KV head
+// g and writes a partial (m, l, O) per query head in log2 units; the combine
+// kernel folds the partials and the sink:
+//   M = max(sink * log2e, max_s m_s)
+//   L = 2^(sink * log2e - M) + sum_s l_s 2^(m_s - M)
+//   out = sum_s O_s 2^(m_s - M) / L,  lse = (M ln 2 + ln L)
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+
+#include "../../include/flint_attn.h"
+#include "flint_common.cuh"
+#include "sm100.cuh"
+
+namespace flint {
+
+constexpr int kDecKeys = 128;          // keys per split = threads per CTA
+constexpr int kDecThreads = 128;
+
+__device__ __forceinline__ float dec_bf16(uint32_t bits16) { return __uint_as_float(bits16 << 16); }
+
+// Normalise (weight form) and, if rope, rotate one 128-channel row held by a
+// warp: lane l owns channels l, l+32, l+64, l+96 (the pairs (l, l+64) and
+// (l+32, l+96) rotate with frequencies l and l+32).  Returns the 4 values.
+__device__ __forceinline__ void dec_norm_rope_row(const __nv_bfloat16* row, const float* w, float eps,
+                                                  bool rope, int pos, const double* inv_freq, int lane,
+                                                  float y[4]) {
+    const uint16_t* r16 = reinterpret_cast<const uint16_t*>(row);
+    float x[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) x[i] = dec_bf16(r16[lane + 32 * i]);
+    float ss = x[0] * x[0] + x[1] * x[1] + x[2] * x[2] + x[3] * x[3];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    const float rn = rsqrtf(ss * (1.f / kHD) + eps);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) y[i] = x[i] * rn * w[lane + 32 * i];
+    if (rope) {
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+            float c, s;
+            rope_cos_sin(pos, inv_freq[lane + 32 * i], &c, &s);
+            const float a = y[i], b = y[i + 2];
+            y[i] = a * c - b * s;
+            y[i + 2] = b * c + a * s;
+        }
+    }
+}
+
+struct DecodeParams {
+    const __nv_bfloat16* q;      // [B,32,128]
+    const __nv_bfloat16* k;      // [B,4,128]
+    const __nv_bfloat16* v;      // [B,4,128]
+    const float* q_norm_w;
+    const float* k_norm_w;
+    const float* sinks;
+    __nv_bfloat16* k_cache;      // [B,cap,4,128]
+    __nv_bfloat16* v_cache;      // [B,cap,4,128]
+    const int* cache_len;        // [B]
+    __nv_bfloat16* out;          // [B,4096]
+    float* lse;                  // [32,B]
+    int* status;                 // device status word
+    float* part;                 // [B,4,nsplit,8,(2 + 128)]
+    int B, cap, window, use_rope, nsplit;
+    float rope_theta, eps;
+};
+
+constexpr int kPartFloats = 8 * (2 + kHD);   // m[8], l[8], O[8][128]
+
+__global__ void __launch_bounds__(kDecThreads)
+decode_split_kernel(const DecodeParams p) {
+    __shared__ float s_q[kHD][kGroup];         // q~ x log2(e)/sqrt(128), channel-major
+    __shared__ float s_knew[kHD];              // the new token's k~ (FP32)
+    __shared__ float s_p[kGroup][kDecKeys];    // scores, then probabilities
+    __shared__ float s_w[2][kHD];              // q_norm_w, k_norm_w
+    __shared__ double s_inv[64];
+    __shared__ float s_m[kGroup];
+
+    const int s = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int pos = p.cache_len[b];
+    const int lo = p.window > 0 ? max(0, pos - p.window + 1) : 0;
+    const int n = pos - lo + 1;
+    float* part = p.part + (((size_t)b * kHKV + g) * p.nsplit + s) * kPartFloats;
+    if (pos < 0 || pos >= FLINT_MAX_TOKENS || n > p.cap) {
+        if (tid == 0) atomicCAS(p.status, 0, 1 /* FLINT_ERR_INVALID_ARG */);
+        if (tid < kGroup) { part[tid] = -INFINITY; part[kGroup + tid] = 0.f; }
+        return;
+    }
+    const int k0 = lo + kDecKeys * s, k1 = min(lo + kDecKeys * (s + 1), pos + 1);
+    if (k0 >= k1) {                            // nothing in this split
+        if (tid < kGroup) { part[tid] = -INFINITY; part[kGroup + tid] = 0.f; }
+        return;
+    }
+    const bool has_new = (k1 == pos + 1);      // this split holds the new token
+
+    s_w[0][tid] = p.q_norm_w[tid];
+    s_w[1][tid] = p.k_norm_w[tid];
+    if (tid < 64) s_inv[tid] = exp2(-(double)tid / 64.0 * log2((double)p.rope_theta));
+    __syncthreads();
+
+    // ---- q~ for the 8 heads of group g (warp w: heads 2w, 2w+1); k~ of the new token
+    const float qscale = 1.4426950408889634f * 0.08838834764831845f;   // log2(e) / sqrt(128)
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+        const int h = 2 * warp + hh;
+        float y[4];
+        dec_norm_rope_row(p.q + ((size_t)b * kHQ + kGroup * g + h) * kHD, s_w[0], p.eps, p.use_rope != 0,
+                          pos, s_inv, lane, y);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) s_q[lane + 32 * i][h] = y[i] * qscale;
+    }
+    if (has_new && warp == 0) {
+        float y[4];
+        dec_norm_rope_row(p.k + ((size_t)b * kHKV + g) * kHD, s_w[1], p.eps, p.use_rope != 0, pos, s_inv,
+                          lane, y);
+        const size_t slot = (size_t)(pos % p.cap);
+        __nv_bfloat16* kdst = p.k_cache + (((size_t)b * p.cap + slot) * kHKV + g) * kHD;
+        __nv_bfloat16* vdst = p.v_cache + (((size_t)b * p.cap + slot) * kHKV + g) * kHD;
+        const __nv_bfloat16* vsrc = p.v + ((size_t)b * kHKV + g) * kHD;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            s_knew[lane + 32 * i] = y[i];
+            kdst[lane + 32 * i] = __float2bfloat16_rn(y[i]);
+            vdst[lane + 32 * i] = vsrc[lane + 32 * i];
+        }
+    }
+    __syncthreads();
+
+    // ---- scores: thread j takes key k0 + j, all 8 heads
+    const int j = tid, kj = k0 + j;
+    if (kj < k1) {
+        float acc[kGroup];
+#pragma unroll
+        for (int h = 0; h < kGroup; ++h) acc[h] = 0.f;
+        if (kj == pos) {
+#pragma unroll 4
+            for (int c = 0; c < kHD; ++c) {
+                const float kc = s_knew[c];
+#pragma unroll
+                for (int h = 0; h < kGroup; ++h) acc[h] = fmaf(s_q[c][h], kc, acc[h]);
+            }
+        } else {
+            const uint4* krow = reinterpret_cast<const uint4*>(
+                p.k_cache + (((size_t)b * p.cap + (size_t)(kj % p.cap)) * kHKV + g) * kHD);
+#pragma unroll 2
+            for (int c8 = 0; c8 < kHD / 8; ++c8) {
+                const uint4 u = krow[c8];
+                const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float ka = __uint_as_float(w4[e] << 16), kb = __uint_as_float(w4[e] & 0xffff0000u);
+                    const int c = 8 * c8 + 2 * e;
+#pragma unroll
+                    for (int h = 0; h < kGroup; ++h) acc[h] = fmaf(s_q[c + 1][h], kb, fmaf(s_q[c][h], ka, acc[h]));
+                }
+            }
+        }
+#pragma unroll
+        for (int h = 0; h < kGroup; ++h) s_p[h][j] = acc[h];
+    } else {
+#pragma unroll
+        for (int h = 0; h < kGroup; ++h) s_p[h][j] = -INFINITY;
+    }
+    __syncthreads();
+
+    // ---- per head: max over the split, probabilities, sum (warp w: heads 2w, 2w+1)
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+        const int h = 2 * warp + hh;
+        float x[4], mx = -INFINITY;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) { x[i] = s_p[h][lane + 32 * i]; mx = fmaxf(mx, x[i]); }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        float sum = 0.f;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float e = exp2f(x[i] - mx);        // masked keys: 2^-inf = 0
+            s_p[h][lane + 32 * i] = e;
+            sum += e;
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+        if (lane == 0) { s_m[h] = mx; part[h] = mx; part[kGroup + h] = sum; }
+    }
+    __syncthreads();
+
+    // ---- O_h[c] = sum_j p_h[j] V_j[c]: thread c, keys of the split in order
+    {
+        const int c = tid;
+        float o[kGroup];
+#pragma unroll
+        for (int h = 0; h < kGroup; ++h) o[h] = 0.f;
+        const int nk = k1 - k0;
+#pragma unroll 8
+        for (int jj = 0; jj < nk; ++jj) {
+            const int kk = k0 + jj;
+            const __nv_bfloat16* vrow =
+                (kk == pos) ? p.v + ((size_t)b * kHKV + g) * kHD
+                            : p.v_cache + (((size_t)b * p.cap + (size_t)(kk % p.cap)) * kHKV + g) * kHD;
+            const float vc = __bfloat162float(vrow[c]);
+#pragma unroll
+            for (int h = 0; h < kGroup; ++h) o[h] = fmaf(s_p[h][jj], vc, o[h]);
+        }
+#pragma unroll
+        for (int h = 0; h < kGroup; ++h) part[2 * kGroup + h * kHD + c] = o[h];
+    }
+}
+
+// Folds the partials of (b, g) with the sinks of its 8 query heads.
+__global__ void __launch_bounds__(kDecThreads)
+decode_combine_kernel(const DecodeParams p) {
+    const int g = blockIdx.x, b = blockIdx.y, c = threadIdx.x;
+    griddep_wait();
+    const float* base = p.part + ((size_t)b * kHKV + g) * p.nsplit * kPartFloats;
+    for (int hh = 0; hh < kGroup; ++hh) {
+        const int h = kGroup * g + hh;
+        const float sink = p.sinks[h];
+        float acc = 0.f, L = 0.f, M;
+        if (sink == INFINITY) {
+            M = INFINITY;
+        } else {
+            M = sink * 1.4426950408889634f;
+            for (int s = 0; s < p.nsplit; ++s) M = fmaxf(M, base[s * kPartFloats + hh]);
+            if (M > -INFINITY) {
+                L = (sink > -INFINITY) ? exp2f(sink * 1.4426950408889634f - M) : 0.f;
+                for (int s = 0; s < p.nsplit; ++s) {
+                    const float* ps = base + s * kPartFloats;
+                    const float ms = ps[hh];
+                    if (ms == -INFINITY) continue;
+                    const float a = exp2f(ms - M);
+                    L += ps[kGroup + hh] * a;
+                    acc += ps[2 * kGroup + hh * kHD + c] * a;
+                }
+            }
+        }
+        const float o = (L > 0.f) ? acc / L : 0.f;
+        p.out[((size_t)b * kHQ + h) * kHD + c] = __float2bfloat16_rn(o);
+        if (c == 0 && p.lse) {
+            float v;
+            if (M == INFINITY) v = INFINITY;
+            else if (L > 0.f) v = M * 0.6931471805599453f + logf(L);
+            else v = -INFINITY;
+            p.lse[(size_t)h * p.B + b] = v;
+        }
+    }
+}
+
+flint_status_t set_error(flint_status_t s, const char* msg);
+
+size_t decode_nsplit(int cap, int window) {
+    const int nmax = window > 0 ? (window < cap ? window : cap) : cap;
+    return (size_t)((nmax + kDecKeys - 1) / kDecKeys);
+}
+
+size_t decode_workspace_bytes(int B, int cap, int window) {
+    return 256 + (size_t)B * kHKV * decode_nsplit(cap, window) * kPartFloats * sizeof(float);
+}
+
+flint_status_t run_decode(const void* q, const void* k, const void* v, const float* q_norm_w,
+                          const float* k_norm_w, const float* sinks, void* k_cache, void* v_cache,
+                          const int32_t* cache_len, int32_t B, int32_t cap, int32_t window,
+                          int32_t use_rope, float rope_theta, float eps, void* out, float* lse,
+                          void* workspace, size_t workspace_bytes, void* stream) {
+    DecodeParams dp;
+    dp.q = static_cast<const __nv_bfloat16*>(q);
+    dp.k = static_cast<const __nv_bfloat16*>(k);
+    dp.v = static_cast<const __nv_bfloat16*>(v);
+    dp.q_norm_w = q_norm_w;
+    dp.k_norm_w = k_norm_w;
+    dp.sinks = sinks;
+    dp.k_cache = static_cast<__nv_bfloat16*>(k_cache);
+    dp.v_cache = static_cast<__nv_bfloat16*>(v_cache);
+    dp.cache_len = cache_len;
+    dp.out = static_cast<__nv_bfloat16*>(out);
+    dp.lse = lse;
+    dp.status = static_cast<int*>(workspace);
+    dp.part = reinterpret_cast<float*>(static_cast<char*>(workspace) + 256);
+    dp.B = B;
+    dp.cap = cap;
+    dp.window = window;
+    dp.use_rope = use_rope;
+    dp.nsplit = (int)decode_nsplit(cap, window);
+    dp.rope_theta = rope_theta;
+    dp.eps = eps;
+    (void)workspace_bytes;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaMemsetAsync(workspace, 0, sizeof(int), s);
+    if (e != cudaSuccess) return set_error(FLINT_ERR_CUDA, "decode: status reset failed");
+    decode_split_kernel<<<dim3(dp.nsplit, kHKV, B), kDecThreads, 0, s>>>(dp);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return set_error(FLINT_ERR_CUDA, "decode: split launch failed");
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(kHKV, B);
+    cfg.blockDim = dim3(kDecThreads);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, decode_combine_kernel, dp);
+    if (e != cudaSuccess) return set_error(FLINT_ERR_CUDA, "decode: combine launch failed");
+    return FLINT_OK;
+}
+
+}  // namespace flint

@@ -166,8 +166,9 @@ FLINT_API flint_status_t flint_attn_attend(const void* q, const void* k, const v
 
 /*
  * Synchronises `stream`, then returns the status the kernels of the last
- * flint_attn_fwd on `workspace` recorded (FLINT_OK, FLINT_ERR_INVALID_ARG for
- * an ill-formed cu_seqlens, FLINT_ERR_UNSUPPORTED for a non-trailing mask,
+ * flint_attn_fwd or flint_attn_decode on `workspace` recorded (FLINT_OK,
+ * FLINT_ERR_INVALID_ARG for an ill-formed cu_seqlens or a decode window that
+ * does not fit its cache, FLINT_ERR_UNSUPPORTED for a non-trailing mask,
  * FLINT_ERR_TIMEOUT), or FLINT_ERR_CUDA if synchronising failed.
  */
 FLINT_API flint_status_t flint_attn_device_status(const void* workspace, void* stream);
@@ -212,6 +213,61 @@ FLINT_API flint_status_t flint_attn_fwd_static(const void* q, const void* k, con
                               float rope_theta, float eps,
                               void* out, float* lse,
                               void* stream);
+
+/* Largest batch of one decode step (sequences per call). */
+#define FLINT_MAX_DECODE_BATCH 65535
+
+/*
+ * One decode step: a new token per sequence attends to the keys and values
+ * cached for its earlier positions (FlintAttention.forward on the NeMo
+ * AutoModel "flint.layers" API page, applied to the last position only; the
+ * "flint" model page notes that the KV cache must honour the per-layer
+ * window sizes).  Sequence b's new token sits at position p = cache_len[b]:
+ * its queries and key get the prologue (per-head RMSNorm in weight form,
+ * then NeoX RoPE at p when use_rope), it attends to positions
+ * max(0, p - window + 1) .. p (window > 0, the window counting the token
+ * itself) or 0 .. p (window == 0) plus the learned sink, and the step
+ * appends it to the cache.
+ *
+ *  q          bf16 [B,32,128]: the new tokens' projected queries, before q_norm.
+ *  k, v       bf16 [B,4,128]: their projected keys (before k_norm) and values.
+ *  q_norm_w, k_norm_w, sinks   as for flint_attn_fwd.
+ *  k_cache    bf16 [B,cap,4,128]: normalised, rotated keys of earlier
+ *             positions; position j of sequence b lives in slot j mod cap, so
+ *             a cache of capacity >= window is a ring on sliding layers.
+ *  v_cache    bf16 [B,cap,4,128]: values, same slots.
+ *             The step writes the new token's key (normalised, rotated,
+ *             rounded to BF16) and value into slot p mod cap.  The window
+ *             must fit the cache (p - lo + 1 <= cap); otherwise the device
+ *             status becomes FLINT_ERR_INVALID_ARG and that sequence's output
+ *             is undefined.
+ *  cache_len  int32 [B]: positions already cached = position of the new token,
+ *             0 <= cache_len[b] < FLINT_MAX_TOKENS (else the device status
+ *             becomes FLINT_ERR_INVALID_ARG).
+ *  B          sequences, 0 <= B <= FLINT_MAX_DECODE_BATCH (0: no-op).
+ *  cap        cache capacity in positions, >= 1.
+ *  window     0 for a full layer, W > 0 for a sliding layer.
+ *  use_rope, rope_theta, eps   as for flint_attn_fwd.
+ *  out        bf16 [B,4096]: out[b, h*128 + c].
+ *  lse        fp32 [32,B] natural-log sum of exponentials including the sink;
+ *             may be NULL.
+ *  workspace  device buffer of at least flint_attn_decode_workspace_bytes(B,
+ *             cap, window) bytes, 256-byte aligned; holds the device status
+ *             (read with flint_attn_device_status) and the split partials.
+ *  stream     cudaStream_t as void*.
+ *
+ * Queries, keys and scores are computed in FP32 on CUDA cores; the key
+ * range of every (sequence, KV head) is split in blocks of 128 keys whose
+ * partial results a second kernel combines with the sink.
+ */
+FLINT_API size_t flint_attn_decode_workspace_bytes(int32_t B, int32_t cap, int32_t window);
+FLINT_API flint_status_t flint_attn_decode(const void* q, const void* k, const void* v,
+                              const float* q_norm_w, const float* k_norm_w,
+                              const float* sinks, void* k_cache, void* v_cache,
+                              const int32_t* cache_len, int32_t B, int32_t cap,
+                              int32_t window, int32_t use_rope, float rope_theta,
+                              float eps, void* out, float* lse,
+                              void* workspace, size_t workspace_bytes, void* stream);
 
 /* Text of the last error raised on the calling host thread ("" if none). */
 FLINT_API const char* flint_attn_last_error(void);
