@@ -14,7 +14,7 @@
 // honour per-layer window sizes).  The step appends the new token: its
 // normalised, rotated key (rounded to BF16) and its value go to slot p mod cap.
 //
-// Split-KV: CTA (s, g, b) takes keys lo + 128 s .. lo + 128 s + 127 of KV head
+// Split-KV: CTA (s, g, b) takes keys lo + 256 s .. lo + 256 s + 255 of KV head
 // g and writes a partial (m, l, O) per query head in log2 units; the combine
 // kernel folds the partials and the sink:
 //   M = max(sink * log2e, max_s m_s)
@@ -31,8 +31,8 @@
 
 namespace flint {
 
-constexpr int kDecKeys = 128;          // keys per split = threads per CTA
-constexpr int kDecThreads = 128;
+constexpr int kDecKeys = 256;          // keys per split
+constexpr int kDecThreads = 128;       // 2 keys per thread for the scores
 
 __device__ __forceinline__ float dec_bf16(uint32_t bits16) { return __uint_as_float(bits16 << 16); }
 
@@ -86,9 +86,10 @@ constexpr int kPartFloats = 8 * (2 + kHD);   // m[8], l[8], O[8][128]
 
 __global__ void __launch_bounds__(kDecThreads)
 decode_split_kernel(const DecodeParams p) {
-    __shared__ float s_q[kHD][kGroup];         // q~ x log2(e)/sqrt(128), channel-major
+    __shared__ __align__(16) float s_q[kHD][kGroup];   // q~ x log2(e)/sqrt(128), channel-major
     __shared__ float s_knew[kHD];              // the new token's k~ (FP32)
-    __shared__ float s_p[kGroup][kDecKeys];    // scores, then probabilities
+    __shared__ __align__(16) float s_p[kDecKeys][kGroup];   // scores, then probabilities, key-major
+    __shared__ __align__(16) float s_o[kDecThreads / 2][2 * kGroup];   // second key half's PV sums
     __shared__ float s_w[2][kHD];              // q_norm_w, k_norm_w
     __shared__ double s_inv[64];
     __shared__ float s_m[kGroup];
@@ -144,40 +145,51 @@ decode_split_kernel(const DecodeParams p) {
     }
     __syncthreads();
 
-    // ---- scores: thread j takes key k0 + j, all 8 heads
-    const int j = tid, kj = k0 + j;
-    if (kj < k1) {
+    // ---- scores: thread t takes keys k0 + t and k0 + t + 128, all 8 heads
+#pragma unroll 1
+    for (int half = 0; half < 2; ++half) {
+        const int j = tid + kDecThreads * half, kj = k0 + j;
         float acc[kGroup];
 #pragma unroll
-        for (int h = 0; h < kGroup; ++h) acc[h] = 0.f;
-        if (kj == pos) {
+        for (int h = 0; h < kGroup; ++h) acc[h] = (kj < k1) ? 0.f : -INFINITY;
+        if (kj < k1 && kj == pos) {
 #pragma unroll 4
             for (int c = 0; c < kHD; ++c) {
                 const float kc = s_knew[c];
-#pragma unroll
-                for (int h = 0; h < kGroup; ++h) acc[h] = fmaf(s_q[c][h], kc, acc[h]);
+                const float4 qa = *reinterpret_cast<const float4*>(&s_q[c][0]);
+                const float4 qb = *reinterpret_cast<const float4*>(&s_q[c][4]);
+                acc[0] = fmaf(qa.x, kc, acc[0]); acc[1] = fmaf(qa.y, kc, acc[1]);
+                acc[2] = fmaf(qa.z, kc, acc[2]); acc[3] = fmaf(qa.w, kc, acc[3]);
+                acc[4] = fmaf(qb.x, kc, acc[4]); acc[5] = fmaf(qb.y, kc, acc[5]);
+                acc[6] = fmaf(qb.z, kc, acc[6]); acc[7] = fmaf(qb.w, kc, acc[7]);
             }
-        } else {
+        } else if (kj < k1) {
             const uint4* krow = reinterpret_cast<const uint4*>(
                 p.k_cache + (((size_t)b * p.cap + (size_t)(kj % p.cap)) * kHKV + g) * kHD);
-#pragma unroll 2
+            // the whole 256-byte row in flight at once
+            uint4 kr[kHD / 8];
+#pragma unroll
+            for (int c8 = 0; c8 < kHD / 8; ++c8) kr[c8] = krow[c8];
+#pragma unroll
             for (int c8 = 0; c8 < kHD / 8; ++c8) {
-                const uint4 u = krow[c8];
+                const uint4 u = kr[c8];
                 const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float ka = __uint_as_float(w4[e] << 16), kb = __uint_as_float(w4[e] & 0xffff0000u);
-                    const int c = 8 * c8 + 2 * e;
-#pragma unroll
-                    for (int h = 0; h < kGroup; ++h) acc[h] = fmaf(s_q[c + 1][h], kb, fmaf(s_q[c][h], ka, acc[h]));
+                for (int e = 0; e < 8; ++e) {
+                    const float kc = (e & 1) ? __uint_as_float(w4[e >> 1] & 0xffff0000u)
+                                             : __uint_as_float(w4[e >> 1] << 16);
+                    const int c = 8 * c8 + e;
+                    const float4 qa = *reinterpret_cast<const float4*>(&s_q[c][0]);
+                    const float4 qb = *reinterpret_cast<const float4*>(&s_q[c][4]);
+                    acc[0] = fmaf(qa.x, kc, acc[0]); acc[1] = fmaf(qa.y, kc, acc[1]);
+                    acc[2] = fmaf(qa.z, kc, acc[2]); acc[3] = fmaf(qa.w, kc, acc[3]);
+                    acc[4] = fmaf(qb.x, kc, acc[4]); acc[5] = fmaf(qb.y, kc, acc[5]);
+                    acc[6] = fmaf(qb.z, kc, acc[6]); acc[7] = fmaf(qb.w, kc, acc[7]);
                 }
             }
         }
-#pragma unroll
-        for (int h = 0; h < kGroup; ++h) s_p[h][j] = acc[h];
-    } else {
-#pragma unroll
-        for (int h = 0; h < kGroup; ++h) s_p[h][j] = -INFINITY;
+        *reinterpret_cast<float4*>(&s_p[j][0]) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+        *reinterpret_cast<float4*>(&s_p[j][4]) = make_float4(acc[4], acc[5], acc[6], acc[7]);
     }
     __syncthreads();
 
@@ -185,16 +197,16 @@ decode_split_kernel(const DecodeParams p) {
 #pragma unroll
     for (int hh = 0; hh < 2; ++hh) {
         const int h = 2 * warp + hh;
-        float x[4], mx = -INFINITY;
+        float x[kDecKeys / 32], mx = -INFINITY;
 #pragma unroll
-        for (int i = 0; i < 4; ++i) { x[i] = s_p[h][lane + 32 * i]; mx = fmaxf(mx, x[i]); }
+        for (int i = 0; i < kDecKeys / 32; ++i) { x[i] = s_p[lane + 32 * i][h]; mx = fmaxf(mx, x[i]); }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
         float sum = 0.f;
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const float e = exp2f(x[i] - mx);        // masked keys: 2^-inf = 0
-            s_p[h][lane + 32 * i] = e;
+        for (int i = 0; i < kDecKeys / 32; ++i) {
+            const float e = exp2f(x[i] - mx);        // keys past the split: 2^-inf = 0
+            s_p[lane + 32 * i][h] = e;
             sum += e;
         }
 #pragma unroll
@@ -203,25 +215,46 @@ decode_split_kernel(const DecodeParams p) {
     }
     __syncthreads();
 
-    // ---- O_h[c] = sum_j p_h[j] V_j[c]: thread c, keys of the split in order
+    // ---- O_h[c] = sum_j p_h[j] V_j[c]: thread t takes channels 2(t % 64),
+    // +1 over half of the split's keys; the two halves meet in shared memory
     {
-        const int c = tid;
-        float o[kGroup];
+        const int cp = tid & 63, kh = tid >> 6;
+        float o[kGroup][2];
 #pragma unroll
-        for (int h = 0; h < kGroup; ++h) o[h] = 0.f;
+        for (int h = 0; h < kGroup; ++h) o[h][0] = o[h][1] = 0.f;
         const int nk = k1 - k0;
-#pragma unroll 8
-        for (int jj = 0; jj < nk; ++jj) {
+        const int jb = kh * (kDecKeys / 2), je = min(nk, jb + kDecKeys / 2);
+        const uint32_t* vnew = reinterpret_cast<const uint32_t*>(p.v + ((size_t)b * kHKV + g) * kHD) + cp;
+        const uint32_t* vbase = reinterpret_cast<const uint32_t*>(p.v_cache + ((size_t)b * p.cap * kHKV + g) * kHD) + cp;
+        const size_t slot_stride = (size_t)kHKV * kHD / 2;        // 32-bit words per cache slot
+        int slot = (k0 + jb) % p.cap;                             // advances by one per key
+#pragma unroll 16
+        for (int jj = jb; jj < je; ++jj) {
             const int kk = k0 + jj;
-            const __nv_bfloat16* vrow =
-                (kk == pos) ? p.v + ((size_t)b * kHKV + g) * kHD
-                            : p.v_cache + (((size_t)b * p.cap + (size_t)(kk % p.cap)) * kHKV + g) * kHD;
-            const float vc = __bfloat162float(vrow[c]);
+            const uint32_t v2 = (kk == pos) ? *vnew : vbase[(size_t)slot * slot_stride];
+            slot = (slot + 1 == p.cap) ? 0 : slot + 1;
+            const float v0 = __uint_as_float(v2 << 16), v1 = __uint_as_float(v2 & 0xffff0000u);
+            const float4 pa = *reinterpret_cast<const float4*>(&s_p[jj][0]);
+            const float4 pb = *reinterpret_cast<const float4*>(&s_p[jj][4]);
+            const float pr[8] = {pa.x, pa.y, pa.z, pa.w, pb.x, pb.y, pb.z, pb.w};
 #pragma unroll
-            for (int h = 0; h < kGroup; ++h) o[h] = fmaf(s_p[h][jj], vc, o[h]);
+            for (int h = 0; h < kGroup; ++h) {
+                o[h][0] = fmaf(pr[h], v0, o[h][0]);
+                o[h][1] = fmaf(pr[h], v1, o[h][1]);
+            }
         }
+        if (kh == 1) {
 #pragma unroll
-        for (int h = 0; h < kGroup; ++h) part[2 * kGroup + h * kHD + c] = o[h];
+            for (int h = 0; h < kGroup; ++h) { s_o[cp][2 * h] = o[h][0]; s_o[cp][2 * h + 1] = o[h][1]; }
+        }
+        __syncthreads();
+        if (kh == 0) {
+#pragma unroll
+            for (int h = 0; h < kGroup; ++h) {
+                const float2 r = make_float2(o[h][0] + s_o[cp][2 * h], o[h][1] + s_o[cp][2 * h + 1]);
+                *reinterpret_cast<float2*>(&part[2 * kGroup + h * kHD + 2 * cp]) = r;
+            }
+        }
     }
 }
 
