@@ -84,7 +84,8 @@ struct DecodeParams {
 
 constexpr int kPartFloats = 8 * (2 + kHD);   // m[8], l[8], O[8][128]
 
-__global__ void __launch_bounds__(kDecThreads)
+// 6 CTAs per SM (80 registers): more loads in flight than one CTA's worth
+__global__ void __launch_bounds__(kDecThreads, 6)
 decode_split_kernel(const DecodeParams p) {
     __shared__ __align__(16) float s_q[kHD][kGroup];   // q~ x log2(e)/sqrt(128), channel-major
     __shared__ float s_knew[kHD];              // the new token's k~ (FP32)
