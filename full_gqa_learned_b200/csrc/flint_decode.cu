@@ -32,7 +32,8 @@
 namespace flint {
 
 constexpr int kDecKeys = 256;          // keys per split
-constexpr int kDecThreads = 128;       // 2 keys per thread for the scores
+constexpr int kDecThreads = 128;       // split kernel: 2 keys per thread for the scores
+constexpr int kCombThreads = kHD;      // combine kernel: one thread per channel
 
 __device__ __forceinline__ float dec_bf16(uint32_t bits16) { return __uint_as_float(bits16 << 16); }
 
@@ -260,10 +261,11 @@ decode_split_kernel(const DecodeParams p) {
 }
 
 // Folds the partials of (b, g) with the sinks of its 8 query heads.
-__global__ void __launch_bounds__(kDecThreads)
+__global__ void __launch_bounds__(kCombThreads)
 decode_combine_kernel(const DecodeParams p) {
     const int g = blockIdx.x, b = blockIdx.y, c = threadIdx.x;
     griddep_wait();
+    if (c >= kHD) return;
     const float* base = p.part + ((size_t)b * kHKV + g) * p.nsplit * kPartFloats;
     for (int hh = 0; hh < kGroup; ++hh) {
         const int h = kGroup * g + hh;
@@ -344,7 +346,7 @@ flint_status_t run_decode(const void* q, const void* k, const void* v, const flo
     if (e != cudaSuccess) return set_error(FLINT_ERR_CUDA, "decode: split launch failed");
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(kHKV, B);
-    cfg.blockDim = dim3(kDecThreads);
+    cfg.blockDim = dim3(kCombThreads);
     cfg.dynamicSmemBytes = 0;
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
