@@ -123,3 +123,53 @@ def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     with pytest.raises(ImportError):
         fa.load_library()
     importlib.reload(fa)
+
+
+# ---------------------------------------------------------------- decode entry
+
+def call_decode(lib, **kw):
+    args = dict(q=A, k=A, v=A, wq=A, wk=A, sinks=A, kc=A, vc=A, lens=A, B=8, cap=513, window=513,
+                use_rope=1, theta=1e4, eps=1e-6, out=A, lse=A, ws=A, ws_bytes=1 << 40, stream=None)
+    args.update(kw)
+    return lib.flint_attn_decode(args["q"], args["k"], args["v"], args["wq"], args["wk"], args["sinks"],
+                                 args["kc"], args["vc"], args["lens"], args["B"], args["cap"],
+                                 args["window"], args["use_rope"], args["theta"], args["eps"],
+                                 args["out"], args["lse"], args["ws"], args["ws_bytes"], args["stream"])
+
+
+def test_decode_workspace_bytes(lib):
+    # status word + partials: 4 KV heads x splits of 128 keys x (8 x 130) floats
+    a = fa.decode_workspace_bytes(8, 513, 513)
+    assert a >= 256 + 8 * 4 * 2 * 8 * 130 * 4
+    assert fa.decode_workspace_bytes(8, 4096, 0) > a        # full layer: splits follow the capacity
+    assert fa.decode_workspace_bytes(8, 4096, 513) == a     # sliding: the window bounds the splits
+    assert fa.decode_workspace_bytes(-1, 513, 513) == 0
+    assert fa.decode_workspace_bytes(8, 0, 513) == 0
+    assert fa.decode_workspace_bytes(8, 513, -1) == 0
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(B=-1), 1),
+    (dict(B=70000), 1),
+    (dict(cap=0), 1),
+    (dict(window=-1), 1),
+    (dict(use_rope=3), 1),
+    (dict(eps=-1.0), 1),
+    (dict(theta=0.5), 1),
+    (dict(q=None), 1),
+    (dict(kc=None), 1),
+    (dict(lens=None), 1),
+    (dict(kc=A + 8), 1),
+    (dict(lens=A + 2), 1),
+    (dict(ws=None), 5),
+    (dict(ws=A + 16), 5),
+    (dict(ws_bytes=512), 5),
+])
+def test_decode_invalid_arguments_rejected_on_host(lib, kw, status):
+    assert call_decode(lib, **kw) == status
+    assert lib.flint_attn_last_error() != b""
+
+
+def test_decode_empty_batch_is_a_noop(lib):
+    assert call_decode(lib, B=0) == 0
+    assert call_decode(lib, B=0, q=None, kc=None, out=None, ws=None) == 0
