@@ -8,6 +8,7 @@
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 
@@ -254,6 +255,13 @@ flint_status_t run_stages(int stages, const void* q, const void* k, const void* 
     ap.use_rope = use_rope;
     ap.rope_theta = rope_theta;
     ap.eps = eps;
+    // test hook (not part of the ABI): FLINT_TEST_WAIT_TIMEOUT_MS=n makes the
+    // attention kernel's bounded waits run out after n ms
+    ap.test_wait_ns = 0;
+    if (const char* tw = std::getenv("FLINT_TEST_WAIT_TIMEOUT_MS")) {
+        const long ms = std::strtol(tw, nullptr, 10);
+        if (ms > 0 && ms <= 10000) ap.test_wait_ns = (unsigned long long)ms * 1000000ull;
+    }
     const int max_units = L.max_items * kHKV;
     const int grid = max_units < sms ? max_units : sms;
     if (stages & kStagePrepare) {

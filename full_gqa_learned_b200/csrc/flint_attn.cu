@@ -56,7 +56,8 @@ enum : uint32_t {
     B_SCHED_FULL = 0, B_SCHED_EMPTY = 2,
     B_Q_FULL = 4, B_Q_EMPTY = 8,
     B_K_FULL = 10, B_K_EMPTY = 12, B_V_FULL = 14, B_V_EMPTY = 16,
-    B_S_FULL = 18, B_P_FULL = 20, B_O_FULL = 22, B_DRAIN = 24
+    B_S_FULL = 18, B_P_FULL = 20, B_O_FULL = 22, B_DRAIN = 24,
+    B_TEST_WAIT = 26     // nothing arrives here: the timeout test hook waits on it
 };
 
 struct Misc {
@@ -194,6 +195,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             mbar_init(bar(B_O_FULL + t), 1);
         }
         mbar_init(bar(B_DRAIN), 1);
+        mbar_init(bar(B_TEST_WAIT), 1);
         misc->abort_flag = 0;
         fence_mbar_init();
     }
@@ -328,7 +330,11 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 for (int kk = 1; kk < 8; ++kk)
                     if (kk < nk) mma_ts_w(d, pa + 8u * kk, vb + kk * (2048 >> 4), v_hi, idesc_pv, 1u);
             };
-            for (;;) {
+            // test hook: a wait that runs out (FLINT_ERR_TIMEOUT and abort)
+            // before any MMA is issued
+            const bool stalled =
+                p.test_wait_ns > 0 && !mbar_wait(bar(B_TEST_WAIT), 0, abort_flag, status, p.test_wait_ns);
+            for (; !stalled;) {
                 if (!mbar_wait(bar(B_SCHED_FULL + sslot), sph, abort_flag, status)) break;
                 const int u = misc->sched[sslot];
                 mbar_arrive(bar(B_SCHED_EMPTY + sslot));

@@ -134,6 +134,10 @@ struct AttnParams {
     char* ws;
     int T, nseg, window, use_rope;
     float rope_theta, eps;
+    // > 0: test hook.  The MMA warp of every CTA first waits this many
+    // nanoseconds on a barrier nothing arrives on, so the bounded-wait
+    // timeout path (status FLINT_ERR_TIMEOUT, abort, drain) runs.
+    unsigned long long test_wait_ns;
 };
 
 }  // namespace flint

@@ -287,3 +287,20 @@ def test_later_chunk_raises_the_max(mix):
     o, l = run_gpu(w)
     rows = np.unique(np.concatenate([np.arange(380, 420), np.arange(0, 512, 7)]))
     compare(w, o, l, rows=rows, tol=TOL_EDGE)
+
+
+def test_bounded_wait_timeout_reports_status(monkeypatch):
+    """Failure detection without a fault: a test hook makes every CTA's MMA
+    warp wait 20 ms on a barrier nothing arrives on.  The bounded wait runs
+    out, the status reads FLINT_ERR_TIMEOUT, every warp unwinds (drains its
+    copies, frees TMEM) and the next call on the same context is correct."""
+    import full_gqa_learned_b200 as fa
+    w = W.make_small(300, seed=19, window=0, use_rope=False)
+    t = to_device(w)
+    monkeypatch.setenv("FLINT_TEST_WAIT_TIMEOUT_MS", "20")
+    fa.attn_fwd(t["q"], t["k"], t["v"], t["q_norm_w"], t["k_norm_w"], t["sinks"], window=0,
+                use_rope=False)
+    assert fa.device_status(fa.attn_fwd.last_workspace) == 4      # FLINT_ERR_TIMEOUT
+    monkeypatch.delenv("FLINT_TEST_WAIT_TIMEOUT_MS")
+    o, l = run_gpu(w)
+    compare(w, o, l, tol=TOL_EDGE)
