@@ -359,6 +359,9 @@ DECODE_CONFIGS = {
                                 max_len=262144, min_len=513),
     "decode_full_b64_s4096": dict(B=64, cap=4096, seed=6, window=0, use_rope=False,
                                   max_len=4096, min_len=1),
+    # a small batch of the sliding case, sized for profiler captures
+    "decode_sliding_b16": dict(B=16, cap=513, seed=5, window=513, use_rope=True,
+                               max_len=262144, min_len=513),
 }
 
 
