@@ -275,7 +275,8 @@ def run_flint(args, rank, world, local_rank):
 
     if args.profile:
         return dict(w=w, total_ms=total_ms, attn_avg=attn_avg, prep_avg=sum(prep_ms) / len(prep_ms),
-                    e2e_ms=float("nan"), h2d=0, d2h=0, clocks=clocks, launches=2 * args.steps)
+                    e2e_ms=float("nan"), h2d=0, d2h=0, clocks=clocks, launches=2 * args.steps,
+                    gpu=torch.cuda.get_device_name(dev))
 
     # end-to-end through the public API from pinned host buffers
     pinned = {k: v.pin_memory() for k, v in host.items()}
@@ -314,7 +315,8 @@ def run_flint(args, rank, world, local_rank):
     # max over ranks
     total_ms, attn_avg, e2e_ms = max_over_ranks([total_ms, attn_avg, e2e_ms], device=dev)
     return dict(w=w, total_ms=total_ms, attn_avg=attn_avg, prep_avg=sum(prep_ms) / len(prep_ms),
-                e2e_ms=e2e_ms, h2d=h2d, d2h=d2h, clocks=clocks, launches=2 * args.steps)
+                e2e_ms=e2e_ms, h2d=h2d, d2h=d2h, clocks=clocks, launches=2 * args.steps,
+                gpu=torch.cuda.get_device_name(dev))
 
 
 def cpu_baseline(w, budget_s, nthreads=0):
@@ -533,7 +535,7 @@ def main():
         config=dict(workload=w.name, T=w.T, window=w.window, use_rope=bool(w.use_rope),
                     q_heads=32, kv_heads=4, head_dim=128, qk_operands="fp16 (post-norm)",
                     pv_operands="bf16", l2="flushed before every timed step (256 MiB write)",
-                    per_rank="independent replica"),
+                    per_rank="independent replica", seed=w.seed, gpu=r["gpu"]),
         roofline=dict(bound="tensor", achieved=round(attn_tflops, 3), peak=peak, unit=UNIT,
                       frac=round(attn_tflops / peak, 4),
                       traffic=args.traffic if args.traffic is not None else recorded_traffic(w.name),

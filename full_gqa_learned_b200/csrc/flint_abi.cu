@@ -9,6 +9,8 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstdlib>
+
+#include <nvtx3/nvToolsExt.h>   // header-only NVTX v3: named ranges for profilers
 #include <cstring>
 #include <mutex>
 
@@ -309,9 +311,25 @@ extern "C" {
     q, k, v, q_norm_w, k_norm_w, sinks, pos_ids, cu_seqlens, num_docs, pad_mask, batch, seqlen, \
         T, window, use_rope, rope_theta, eps, out, lse, workspace, workspace_bytes, stream
 
-flint_status_t flint_attn_fwd(FLINT_ARGS) { return run_stages(kStageBoth, FLINT_FWD_ARGS); }
-flint_status_t flint_attn_prepare(FLINT_ARGS) { return run_stages(kStagePrepare, FLINT_FWD_ARGS); }
-flint_status_t flint_attn_attend(FLINT_ARGS) { return run_stages(kStageAttend, FLINT_FWD_ARGS); }
+// Each entry point is one NVTX range (host side: the enqueue), so a timeline
+// profiler shows which library call launched which kernels.
+struct NvtxRange {
+    explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
+};
+
+flint_status_t flint_attn_fwd(FLINT_ARGS) {
+    NvtxRange r("flint_attn_fwd");
+    return run_stages(kStageBoth, FLINT_FWD_ARGS);
+}
+flint_status_t flint_attn_prepare(FLINT_ARGS) {
+    NvtxRange r("flint_attn_prepare");
+    return run_stages(kStagePrepare, FLINT_FWD_ARGS);
+}
+flint_status_t flint_attn_attend(FLINT_ARGS) {
+    NvtxRange r("flint_attn_attend");
+    return run_stages(kStageAttend, FLINT_FWD_ARGS);
+}
 
 size_t flint_attn_decode_workspace_bytes(int32_t B, int32_t cap, int32_t window) {
     if (B < 0 || B > FLINT_MAX_DECODE_BATCH || cap < 1 || cap > FLINT_MAX_TOKENS || window < 0) return 0;
@@ -324,6 +342,7 @@ flint_status_t flint_attn_decode(const void* q, const void* k, const void* v, co
                                  int32_t window, int32_t use_rope, float rope_theta, float eps,
                                  void* out, float* lse, void* workspace, size_t workspace_bytes,
                                  void* stream) {
+    NvtxRange r("flint_attn_decode");
     g_err[0] = '\0';
     if (B < 0 || B > FLINT_MAX_DECODE_BATCH)
         return fail(FLINT_ERR_INVALID_ARG, "B=%d outside [0, %d]", B, FLINT_MAX_DECODE_BATCH);
