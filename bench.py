@@ -66,13 +66,42 @@ def recorded_traffic(workload):
                 vals[key.strip()] = val.strip()
     if "traffic_bytes_per_launch" not in vals or "kernel_source_sha256" not in vals:
         return None
-    h = hashlib.sha256()
-    for src in KERNEL_SOURCES:
-        with open(src, "rb") as f:
-            h.update(f.read())
-    if h.hexdigest() != vals["kernel_source_sha256"]:
+    if kernel_code_sha256() != vals["kernel_source_sha256"]:
         return None
     return float(vals["traffic_bytes_per_launch"])
+
+
+def strip_comments(text):
+    """C/C++ source without // and /* */ comments (string literals kept)."""
+    out, i, n = [], 0, len(text)
+    while i < n:
+        c = text[i]
+        if c == '"':
+            j = i + 1
+            while j < n and text[j] != '"':
+                j += 2 if text[j] == "\\" else 1
+            out.append(text[i:j + 1])
+            i = j + 1
+        elif text.startswith("//", i):
+            j = text.find("\n", i)
+            i = n if j < 0 else j
+        elif text.startswith("/*", i):
+            j = text.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+        else:
+            out.append(c)
+            i += 1
+    return "".join(out)
+
+
+def kernel_code_sha256():
+    """SHA-256 of the attention kernel's sources with comments removed: a
+    recorded profile stays valid across comment edits, not code edits."""
+    h = hashlib.sha256()
+    for src in KERNEL_SOURCES:
+        with open(src, encoding="utf-8") as f:
+            h.update(strip_comments(f.read()).encode("utf-8"))
+    return h.hexdigest()
 
 
 def load_peaks():

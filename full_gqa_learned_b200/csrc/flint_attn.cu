@@ -15,6 +15,7 @@
 // Layout of one CTA (one per SM, persistent, 384 threads):
 //   warp 0      dynamic scheduler + TMA producer (Q tiles, K/V chunks)
 //   warp 1      TMEM owner; lane 0 issues every tcgen05.mma and commit
+//   warps 2-3   idle (their registers go to the softmax warpgroups)
 //   warps 4-7   softmax warpgroup of tile 0 (tokens q0..q0+15)
 //   warps 8-11  softmax warpgroup of tile 1 (tokens q0+16..q0+31)
 // A tile is 128 MMA rows = 16 tokens x the 8 query heads of one KV group, so
@@ -25,6 +26,12 @@
 // from TMEM.  The online softmax starts from m = sink*log2(e), l = 1, which
 // is exactly the extra sink column; the running max is only raised (and O
 // rescaled) when it grows by more than 2^8, so the rescale is rare.
+// Interior chunks after the first skip the row max altogether while the row
+// sum of their terms stays within 2^8; masked chunks treat each 32-column
+// block as full, empty or partial.  Each softmax warp stores its 4 output
+// tokens through a swizzled staging block and TMA.  The kernel runs as a
+// programmatic dependent of the preparation kernel: its setup overlaps that
+// kernel's tail and it reads nothing prepared before griddepcontrol.wait.
 #include <cuda.h>
 #include <cmath>
 #include "flint_common.cuh"
@@ -138,9 +145,10 @@ __device__ __forceinline__ uint64_t exp2_poly2(uint64_t x) {
 }
 
 // Pairs j of each 16-pair block with (j % 8) < kPolyPairs take the polynomial.
-// Measured costs per warp instruction and scheduler on B200: ex2 8 cycles,
-// fma/add.f32x2 2, cvt.rn.bf16x2.f32 ~4.5; a polynomial pair costs ~20 on
-// the FMA/ALU pipes, so MUFU and the FMA/ALU pipes balance near 1/8.
+// Measured costs per warp instruction and scheduler on B200: ex2 8 cycles;
+// fma/add.f32x2, cvt.rn.bf16x2.f32 and 3-input max 2 each (cvt and max share
+// a pipe, ex2 overlaps all of them); a polynomial pair costs ~20 on the
+// FMA/ALU pipes.  Shares of 2/8 and 3/8 measured slower than 1/8.
 constexpr int kPolyPairs = 1;
 
 // Two FP32 values -> packed BF16 pair, `lo` in the low half.
