@@ -95,12 +95,14 @@ def strip_comments(text):
 
 
 def kernel_code_sha256():
-    """SHA-256 of the attention kernel's sources with comments removed: a
-    recorded profile stays valid across comment edits, not code edits."""
+    """SHA-256 of the attention kernel's sources with comments removed and
+    whitespace collapsed: a recorded profile stays valid across comment and
+    layout edits, not code edits."""
     h = hashlib.sha256()
     for src in KERNEL_SOURCES:
         with open(src, encoding="utf-8") as f:
-            h.update(strip_comments(f.read()).encode("utf-8"))
+            # whitespace runs collapsed: a removed comment leaves no trace
+            h.update(" ".join(strip_comments(f.read()).split()).encode("utf-8"))
     return h.hexdigest()
 
 
