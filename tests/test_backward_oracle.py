@@ -1,0 +1,190 @@
+"""Pins of the backward oracle (oracle/backward.py).  CPU only.
+
+The strongest pin is independent of the adjoint formulas: central finite
+differences of the C forward oracle (a separate code path) of the scalar
+loss sum(dO * out), checked entry by entry on q, k, v, both norm weights and
+the sinks, for full and sliding layers, with RoPE, documents, padding and the
+window.  Closed forms and invariants cover the rest.
+"""
+import numpy as np
+import pytest
+
+import oracle
+import workloads as W
+from oracle import backward as OB
+
+FD_STEP = 1e-5
+
+
+def _loss(w, dO, q=None, k=None, v=None, wq=None, wk=None, sinks=None):
+    out, _ = oracle.attn_fwd(w.q if q is None else q, w.k if k is None else k,
+                             w.v if v is None else v, w.q_norm_w if wq is None else wq,
+                             w.k_norm_w if wk is None else wk, w.sinks if sinks is None else sinks,
+                             pos_ids=w.pos_ids, cu_seqlens=w.cu_seqlens, pad_mask=w.pad_mask,
+                             window=w.window, use_rope=w.use_rope, rope_theta=w.rope_theta,
+                             eps=w.eps)
+    return float(np.sum(out * dO))
+
+
+def _fd(w, dO, name, idx):
+    """Central difference of the loss in one entry of input `name`."""
+    base = {"q": oracle._f64(w.q), "k": oracle._f64(w.k), "v": oracle._f64(w.v),
+            "wq": np.asarray(w.q_norm_w, np.float64), "wk": np.asarray(w.k_norm_w, np.float64),
+            "sinks": np.asarray(w.sinks, np.float64)}[name]
+    vals = []
+    for sgn in (1.0, -1.0):
+        x = base.copy()
+        x[idx] += sgn * FD_STEP
+        vals.append(_loss(w, dO, **{name: x}))
+    return (vals[0] - vals[1]) / (2 * FD_STEP)
+
+
+def _case(kind):
+    if kind == "full":
+        return W.make_small(20, seed=71, window=0, use_rope=False)
+    if kind == "sliding_thd":
+        return W.make_small(20, seed=72, window=5, use_rope=True, cu_seqlens=[0, 9, 17])
+    if kind == "padmask":
+        m = np.zeros((2, 10), np.uint8)
+        m[0, :10] = 1
+        m[1, :6] = 1
+        return W.make_small(20, seed=73, window=4, use_rope=True, pad_mask=m)
+    raise KeyError(kind)
+
+
+def _dout(T, seed):
+    return np.random.default_rng(seed).standard_normal((T, 32, 128))
+
+
+def _sample_indices(rng, shape, n, forced=()):
+    idx = [tuple(int(rng.integers(0, s)) for s in shape) for _ in range(n)]
+    return list(forced) + idx
+
+
+@pytest.mark.parametrize("kind", ["full", "sliding_thd", "padmask"])
+def test_gradient_matches_finite_differences(kind):
+    w = _case(kind)
+    T = w.T
+    dO = _dout(T, 100)
+    g = OB.attn_bwd_workload(w, dO)
+    rng = np.random.default_rng(7)
+    # forced entries: a padded token, the first and last valid tokens
+    last = T - 1
+    checks = []
+    for idx in _sample_indices(rng, (T, 32, 128), 10, [(0, 0, 0), (last, 5, 64), (8, 31, 127)]):
+        checks.append(("q", "dq", idx))
+    for idx in _sample_indices(rng, (T, 4, 128), 10, [(0, 0, 3), (last, 3, 100), (16, 1, 0)]):
+        checks.append(("k", "dk", idx))
+    for idx in _sample_indices(rng, (T, 4, 128), 8, [(last, 2, 7), (4, 0, 0)]):
+        checks.append(("v", "dv", idx))
+    for c in (0, 63, 64, 127):
+        checks.append(("wq", "dq_norm_w", (c,)))
+        checks.append(("wk", "dk_norm_w", (c,)))
+    for h in (0, 7, 8, 31):
+        checks.append(("sinks", "dsinks", (h,)))
+    for name, key, idx in checks:
+        fd = _fd(w, dO, name, idx)
+        an = g[key][idx]
+        assert abs(fd - an) <= 1e-6 * (1.0 + abs(an)), (kind, name, idx, fd, an)
+
+
+def test_padded_tokens_get_zero_gradient():
+    w = _case("sliding_thd")          # tokens 17..19 are padding
+    g = OB.attn_bwd_workload(w, _dout(w.T, 101))
+    for key in ("dq", "dk", "dv"):
+        assert np.all(g[key][17:] == 0.0), key
+        assert np.any(g[key][:17] != 0.0), key
+
+
+def test_forward_part_equals_the_c_oracle():
+    """The backward module's own norm/RoPE/softmax forward reproduces the C
+    oracle's out and lse."""
+    for kind in ("full", "sliding_thd", "padmask"):
+        w = _case(kind)
+        g = OB.attn_bwd_workload(w, _dout(w.T, 102))
+        out, lse = oracle.attn_fwd_workload(w, rows=None)
+        np.testing.assert_allclose(g["out"], out, rtol=0, atol=1e-12)
+        np.testing.assert_allclose(g["lse"], lse, rtol=0, atol=1e-12)
+
+
+def test_single_token_closed_form():
+    """One token, one key: out_h = sigma(s_h - sink_h) v_g, so
+    dv_g = sum_{h in g} sigma_h dO_h and dsink_h = -sigma_h (1 - sigma_h) dO_h . v_g."""
+    w = W.make_small(1, seed=74, window=0, use_rope=True)
+    dO = _dout(1, 103)
+    g = OB.attn_bwd_workload(w, dO)
+    _, lse = oracle.attn_fwd_workload(w, rows=None)
+    v = oracle._f64(w.v)[0]
+    sk = np.asarray(w.sinks, np.float64)
+    sig = 1.0 - np.exp(sk - lse[0])            # P of the one key = 1 - P_sink
+    for grp in range(4):
+        hs = range(8 * grp, 8 * grp + 8)
+        want = sum(sig[h] * dO[0, h] for h in hs)
+        np.testing.assert_allclose(g["dv"][0, grp], want, rtol=1e-12, atol=1e-12)
+    for h in range(32):
+        want = -sig[h] * (1 - sig[h]) * float(dO[0, h] @ v[h // 8])
+        assert abs(g["dsinks"][h] - want) <= 1e-12 * (1 + abs(want))
+
+
+def test_value_gradient_column_sum():
+    """sum_j dv_j = sum_i sum_{h in g} (1 - e^{sink_h - lse_ih}) dO_ih: each
+    row's key probabilities add up to one minus the sink's share."""
+    w = _case("sliding_thd")
+    dO = _dout(w.T, 104)
+    g = OB.attn_bwd_workload(w, dO)
+    _, lse = oracle.attn_fwd_workload(w, rows=None)
+    doc = oracle.doc_ids(w.T, w.cu_seqlens, None)
+    sk = np.asarray(w.sinks, np.float64)
+    for grp in range(4):
+        want = np.zeros(128)
+        for i in range(w.T):
+            if doc[i] < 0:
+                continue
+            for h in range(8 * grp, 8 * grp + 8):
+                want += (1.0 - np.exp(sk[h] - lse[i, h])) * dO[i, h]
+        np.testing.assert_allclose(g["dv"][:, grp].sum(axis=0), want, rtol=0, atol=1e-10)
+
+
+def test_norm_scale_invariance_makes_gradient_orthogonal():
+    """With eps = 0 the output is invariant to scaling a pre-norm row, so the
+    gradient of every q and k row is orthogonal to that row."""
+    w = W.make_small(12, seed=75, window=0, use_rope=True)
+    w.eps = 0.0
+    g = OB.attn_bwd_workload(w, _dout(12, 105))
+    q, k = oracle._f64(w.q), oracle._f64(w.k)
+    dots_q = np.sum(g["dq"] * q, axis=-1)
+    dots_k = np.sum(g["dk"] * k, axis=-1)
+    assert np.max(np.abs(dots_q)) < 1e-12 * max(1.0, np.max(np.abs(g["dq"])) * 128)
+    assert np.max(np.abs(dots_k)) < 1e-12 * max(1.0, np.max(np.abs(g["dk"])) * 128)
+    assert np.max(np.abs(g["dq"])) > 1e-3 and np.max(np.abs(g["dk"])) > 1e-3
+
+
+def test_packed_documents_equal_separate_runs():
+    """Gradients of a packed run are the per-document gradients side by side;
+    the shared weights' and sinks' gradients add up."""
+    w = W.make_small(20, seed=76, window=6, use_rope=True, cu_seqlens=[0, 11, 20])
+    dO = _dout(20, 106)
+    g = OB.attn_bwd_workload(w, dO)
+    acc = {"dq_norm_w": 0.0, "dk_norm_w": 0.0, "dsinks": 0.0}
+    for a, b in ((0, 11), (11, 20)):
+        gs = OB.attn_bwd(w.q[a:b], w.k[a:b], w.v[a:b], w.q_norm_w, w.k_norm_w, w.sinks, dO[a:b],
+                         pos_ids=w.pos_ids[a:b], window=6, use_rope=True)
+        for key in ("dq", "dk", "dv"):
+            np.testing.assert_allclose(g[key][a:b], gs[key], rtol=0, atol=1e-12)
+        for key in acc:
+            acc[key] = acc[key] + gs[key]
+    for key in acc:
+        np.testing.assert_allclose(g[key], acc[key], rtol=0, atol=1e-11)
+
+
+def test_infinite_sinks():
+    """sink = +inf: out = 0 whatever the inputs, so all gradients vanish;
+    sink = -inf: the sink column is absent and dsink = 0."""
+    w = W.make_small(6, seed=77, window=0, use_rope=False, sinks=np.inf)
+    g = OB.attn_bwd_workload(w, _dout(6, 107))
+    for key in ("dq", "dk", "dv", "dq_norm_w", "dk_norm_w", "dsinks"):
+        assert np.all(g[key] == 0.0), key
+    w = W.make_small(6, seed=78, window=0, use_rope=False, sinks=-np.inf)
+    g = OB.attn_bwd_workload(w, _dout(6, 108))
+    assert np.all(g["dsinks"] == 0.0)
+    assert np.all(np.isfinite(g["dq"])) and np.any(g["dq"] != 0.0)
