@@ -84,7 +84,8 @@ def attn_bwd(q, k, v, q_norm_w, k_norm_w, sinks, dout, *, pos_ids=None, cu_seqle
     """Gradients of sum(dout * out) for the forward with these arguments.
 
     q [T,32,128], k and v [T,4,128] (BF16 bit patterns or floats), weights
-    [128], sinks [32], dout [T,32,128] (or [T,4096]).  Returns a dict of
+    [128], sinks [32], dout [T,32,128] (or [T,4096]); pos_ids None means the
+    index of each token within its document.  Returns a dict of
     float64 arrays: dq [T,32,128], dk, dv [T,4,128], dq_norm_w, dk_norm_w
     [128], dsinks [32], and the forward's out [T,32,128] and lse [T,32].
     """
@@ -98,7 +99,12 @@ def attn_bwd(q, k, v, q_norm_w, k_norm_w, sinks, dout, *, pos_ids=None, cu_seqle
     wk = _f64(k_norm_w).reshape(D)
     sk = np.asarray(sinks, np.float64).reshape(HQ)
     doc = doc_ids(T, cu_seqlens, pad_mask)
-    pos = np.zeros(T, np.int64) if pos_ids is None else np.asarray(pos_ids, np.int64).reshape(T)
+    if pos_ids is None:                 # default: index of the token within its document
+        pos = np.zeros(T, np.int64)
+        for a, b in _segments(doc):
+            pos[a:b] = np.arange(b - a)
+    else:
+        pos = np.asarray(pos_ids, np.int64).reshape(T)
     scale = 1.0 / np.sqrt(D)
 
     # forward quantities

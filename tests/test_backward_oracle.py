@@ -107,6 +107,22 @@ def test_forward_part_equals_the_c_oracle():
         np.testing.assert_allclose(g["lse"], lse, rtol=0, atol=1e-12)
 
 
+def test_default_positions_are_document_local():
+    """pos_ids = None rotates each token by its index within its document,
+    as the C forward oracle does."""
+    w = W.make_small(20, seed=79, window=5, use_rope=True, cu_seqlens=[0, 7, 16])
+    dO = _dout(20, 109)
+    g = OB.attn_bwd(w.q, w.k, w.v, w.q_norm_w, w.k_norm_w, w.sinks, dO, cu_seqlens=w.cu_seqlens,
+                    window=5, use_rope=True)
+    out, lse = oracle.attn_fwd(w.q, w.k, w.v, w.q_norm_w, w.k_norm_w, w.sinks,
+                               cu_seqlens=w.cu_seqlens, window=5, use_rope=True)
+    np.testing.assert_allclose(g["out"], out, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(g["lse"], lse, rtol=0, atol=1e-12)
+    ge = OB.attn_bwd_workload(w, dO)
+    for key in ("dq", "dk", "dv", "dsinks"):
+        np.testing.assert_array_equal(g[key], ge[key])
+
+
 def test_single_token_closed_form():
     """One token, one key: out_h = sigma(s_h - sink_h) v_g, so
     dv_g = sum_{h in g} sigma_h dO_h and dsink_h = -sigma_h (1 - sigma_h) dO_h . v_g."""

@@ -40,6 +40,7 @@ PINS = [
     P.test_norm_scale_invariance_makes_gradient_orthogonal,
     P.test_packed_documents_equal_separate_runs,
     P.test_infinite_sinks,
+    P.test_default_positions_are_document_local,
 ]
 
 
