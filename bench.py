@@ -14,6 +14,9 @@ With --gpus N > 1 (launched by torch.distributed.run) every rank runs its own
 replica on its own GPU (weak scaling, no data-path collective); NCCL is only
 used for the barriers and the max-over-ranks of the timings.
 
+--workload bwd_<name> times the gradient (flint_attn_bwd) on workload <name>
+instead; decode_* workloads time one decode step.
+
 --impl reference times the FP64 CPU oracle on the host cores on a bounded
 sample of the same workload (rank 0 only).
 
@@ -470,13 +473,171 @@ def decode_line(args, world, d, total_ms, clocks):
         gpu_launches=2 * args.steps, clocks=clocks)
 
 
+# ---------------------------------------------------------------- backward leg
+
+BWD_PREFIX = "bwd_"
+BWD_METRIC = ("sink-attn backward TFLOP/s (window-aware algorithmic FLOPs: 2.5x the forward's, "
+              "five contractions per pair and head)")
+# FP32 FMA rate of the CUDA cores: 148 SMs x 128 lanes x 2 FLOPs x 1.965 GHz
+ALU_FP32_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+
+
+def bwd_flops(w):
+    return 2.5 * w.flops()
+
+
+def run_bwd(args, rank, world, local_rank):
+    """One flint_attn_bwd call per timed step on the forward's out and lse of
+    the named workload and a seeded N(0,1) BF16 upstream gradient; L2
+    flushed before each step."""
+    import torch
+    import full_gqa_learned_b200 as fa
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    w = W.make(args.workload[len(BWD_PREFIX):])
+    T = w.T
+
+    def bf(x):
+        return torch.from_numpy(np.ascontiguousarray(x)).view(torch.bfloat16)
+    host = dict(q=bf(w.q), k=bf(w.k), v=bf(w.v), q_norm_w=torch.from_numpy(w.q_norm_w),
+                k_norm_w=torch.from_numpy(w.k_norm_w),
+                sinks=torch.from_numpy(np.ascontiguousarray(w.sinks, np.float32)))
+    for name in ("pos_ids", "cu_seqlens", "pad_mask"):
+        if getattr(w, name) is not None:
+            host[name] = torch.from_numpy(getattr(w, name))
+    rng = np.random.default_rng(w.seed + 1000)
+    host["dout"] = bf(W.bf16_bits(rng.standard_normal((T, 4096), dtype=np.float32)))
+    d = {k: v.to(dev) for k, v in host.items()}
+    kw = dict(pos_ids=d.get("pos_ids"), cu_seqlens=d.get("cu_seqlens"), pad_mask=d.get("pad_mask"),
+              window=w.window, use_rope=w.use_rope, rope_theta=w.rope_theta, eps=w.eps)
+    out, lse = fa.attn_fwd(d["q"], d["k"], d["v"], d["q_norm_w"], d["k_norm_w"], d["sinks"], **kw)
+    host["out"], host["lse"] = out.cpu(), lse.cpu()
+    d["out"], d["lse"] = out, lse
+    shapes = {"dq": (T, 32, 128), "dk": (T, 4, 128), "dv": (T, 4, 128), "dq_norm_w": (128,),
+              "dk_norm_w": (128,), "dsinks": (32,)}
+    grads = {n: torch.empty(sh, dtype=torch.float32, device=dev) for n, sh in shapes.items()}
+    ws = torch.empty(fa.bwd_workspace_bytes(T), dtype=torch.uint8, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def call(dd, g):
+        fa.attn_bwd(dd["q"], dd["k"], dd["v"], dd["q_norm_w"], dd["k_norm_w"], dd["sinks"], dd["out"],
+                    dd["lse"], dd["dout"], pos_ids=dd.get("pos_ids"), cu_seqlens=dd.get("cu_seqlens"),
+                    pad_mask=dd.get("pad_mask"), window=w.window, use_rope=w.use_rope,
+                    rope_theta=w.rope_theta, eps=w.eps, grads=g, workspace=ws, stream=stream)
+
+    for _ in range(args.warmup):
+        flush.fill_(1)
+        call(d, grads)
+    st = fa.device_status(ws)
+    if st != 0:
+        raise RuntimeError("device status %s" % fa.STATUS.get(st, st))
+    sampler = ClockSampler(local_rank if "CUDA_VISIBLE_DEVICES" not in os.environ else
+                           os.environ["CUDA_VISIBLE_DEVICES"].split(",")[local_rank])
+    sampler.start()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    for i in range(args.steps):
+        flush.fill_(i & 0xFF)
+        evs[i][0].record(stream)
+        call(d, grads)
+        evs[i][1].record(stream)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+    total_ms = sum(e[0].elapsed_time(e[1]) for e in evs)
+
+    e2e_ms, h2d, d2h = float("nan"), 0, 0
+    if not args.profile:
+        # end to end: inputs from pinned host memory, gradients back to it
+        pinned = {k: v.pin_memory() for k, v in host.items()}
+        g_h = {n: torch.empty(sh, dtype=torch.float32).pin_memory() for n, sh in shapes.items()}
+        h2d = sum(v.numel() * v.element_size() for v in pinned.values())
+        d2h = sum(v.numel() * 4 for v in g_h.values())
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        n_e2e = max(3, min(args.steps, 10))
+        e2e_ms = 0.0
+        for _ in range(n_e2e):
+            flush.fill_(3)
+            e0.record(stream)
+            dd = {k: v.to(dev, non_blocking=True) for k, v in pinned.items()}
+            call(dd, grads)
+            for n in g_h:
+                g_h[n].copy_(grads[n], non_blocking=True)
+            e1.record(stream)
+            torch.cuda.synchronize(dev)
+            e2e_ms += e0.elapsed_time(e1)
+        e2e_ms /= n_e2e
+    total_ms, e2e_ms = max_over_ranks([total_ms, e2e_ms], device=dev)
+    return dict(w=w, total_ms=total_ms, e2e_ms=e2e_ms, h2d=h2d, d2h=d2h, clocks=clocks,
+                gpu=torch.cuda.get_device_name(dev))
+
+
+def bwd_cpu_baseline(w, budget_s):
+    """The backward oracle, as it stands, on a prefix of the workload's
+    tokens (a prefix of a causal layer is a self-contained problem), grown
+    until a run takes about budget_s seconds: algorithmic FLOPs per second."""
+    from threadpoolctl import threadpool_limits
+    from oracle import backward as OB
+    rng = np.random.default_rng(1)
+    n, dt = 32, 0.0
+    with threadpool_limits(limits=1):          # one BLAS thread: `cores` below is exact
+        return _bwd_cpu_sample(w, budget_s, OB, rng)
+
+
+def _bwd_cpu_sample(w, budget_s, OB, rng):
+    n, dt = 32, 0.0
+    while True:
+        sub = W.make_small(n, seed=w.seed, window=w.window, use_rope=w.use_rope)
+        sub.q, sub.k, sub.v = w.q[:n], w.k[:n], w.v[:n]
+        sub.q_norm_w, sub.k_norm_w, sub.sinks = w.q_norm_w, w.k_norm_w, w.sinks
+        dO = rng.standard_normal((n, 32, 128))
+        t0 = time.time()
+        OB.attn_bwd_workload(sub, dO)
+        dt = time.time() - t0
+        if dt > budget_s / 4 or 2 * n > w.T:
+            break
+        n *= 2
+    return dict(value=bwd_flops(sub) / dt / 1e12, unit=UNIT, cores=1, kind="oracle",
+                sample="first %d tokens of %s (one document), %.2f s" % (n, w.name, dt))
+
+
+def bwd_line(args, world, r):
+    w = r["w"]
+    flops = bwd_flops(w)
+    step_ms = r["total_ms"] / args.steps
+    tf = flops / (step_ms * 1e-3) / 1e12
+    return dict(
+        metric=BWD_METRIC, value=round(tf * world, 4), unit=UNIT, n_gpus=world, steps=args.steps,
+        warmup=args.warmup, ms_per_step=round(step_ms, 5), higher_is_better=True, scaling="weak",
+        vs_baseline=None, dtype="f32",
+        data="synthetic (the forward workload's seeded inputs; N(0,1) BF16 upstream gradient)",
+        config=dict(workload=args.workload, T=w.T, window=w.window, use_rope=bool(w.use_rope),
+                    l2="flushed before every timed step (256 MiB write)", per_rank="independent replica",
+                    seed=w.seed, gpu=r["gpu"]),
+        roofline=dict(bound="alu", achieved=round(tf, 4), peak=round(ALU_FP32_TFLOPS, 2), unit=UNIT,
+                      frac=round(tf / ALU_FP32_TFLOPS, 4), traffic=None,
+                      kernel="flint bwd call (segments, prep, dq, dkv, finish kernels)",
+                      peak_source="derived: FP32 FMA rate of 148 SMs x 128 lanes at 1.965 GHz",
+                      flops_per_launch=flops),
+        e2e=dict(value=round(flops / (r["e2e_ms"] * 1e-3) / 1e12 * world, 4), unit=UNIT,
+                 h2d_bytes_per_step=r["h2d"], d2h_bytes_per_step=r["d2h"], ms_per_step=round(r["e2e_ms"], 4)),
+        gpu_launches=5 * args.steps, clocks=r["clocks"])
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD,
-                    choices=sorted(W.CONFIGS) + sorted(W.DECODE_CONFIGS))
+                    choices=sorted(W.CONFIGS) + sorted(W.DECODE_CONFIGS)
+                    + sorted(BWD_PREFIX + n for n in W.CONFIGS))
     ap.add_argument("--impl", default="flint", choices=["flint", "reference"])
     ap.add_argument("--soak", type=float, default=1.0, help="seconds of untimed load before timing")
     ap.add_argument("--cpu-budget", type=float, default=12.0)
@@ -514,6 +675,24 @@ def main():
                                   e2e=dict(value=value, unit="GB/s", h2d_bytes_per_step=0,
                                            d2h_bytes_per_step=0))))
             return 0
+        if args.workload.startswith(BWD_PREFIX):
+            w = W.make(args.workload[len(BWD_PREFIX):])
+            vals, cb = [], None
+            for i in range(args.warmup + args.steps):
+                cb = bwd_cpu_baseline(w, budget_s=min(args.cpu_budget, 60.0 / max(1, args.steps + args.warmup)))
+                if i >= args.warmup:
+                    vals.append(cb["value"])
+            value = statistics.median(vals)
+            cb["value"] = value
+            print(json.dumps(dict(impl="reference", metric=BWD_METRIC, value=value, unit=UNIT,
+                                  n_gpus=args.gpus, steps=args.steps, warmup=args.warmup, ms_per_step=None,
+                                  higher_is_better=True, scaling="weak", vs_baseline=None, dtype="f64",
+                                  data="synthetic", config=dict(workload=args.workload, T=w.T,
+                                                                window=w.window, use_rope=w.use_rope),
+                                  cpu_baseline=cb,
+                                  e2e=dict(value=value, unit=UNIT, h2d_bytes_per_step=0,
+                                           d2h_bytes_per_step=0))))
+            return 0
         w = W.make(args.workload)
         times, cb = [], None
         for i in range(args.warmup + args.steps):
@@ -545,6 +724,17 @@ def main():
         line = decode_line(args, world, d, total_ms, clocks)
         if rank == 0 and world == 1 and not args.profile:
             line["cpu_baseline"] = decode_cpu_baseline(d, budget_s=args.cpu_budget)
+        if world > 1:
+            dist.barrier()
+            dist.destroy_process_group()
+        if rank == 0:
+            print(json.dumps(line))
+        return 0
+    if args.workload.startswith(BWD_PREFIX):
+        r = run_bwd(args, rank, world, local_rank)
+        line = bwd_line(args, world, r)
+        if rank == 0 and world == 1 and not args.profile:
+            line["cpu_baseline"] = bwd_cpu_baseline(r["w"], budget_s=args.cpu_budget)
         if world > 1:
             dist.barrier()
             dist.destroy_process_group()

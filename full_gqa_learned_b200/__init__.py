@@ -1,4 +1,5 @@
-"""B200 (sm_100a) sink-aware GQA attention forward of the Flint decoder.
+"""B200 (sm_100a) sink-aware GQA attention of the Flint decoder: forward,
+gradient and decode step.
 
 This package is a thin ctypes binding over ``libflint_attn.so``, whose C ABI
 is declared in ``include/flint_attn.h``.  The binding only marshals
@@ -16,8 +17,8 @@ import os
 import threading
 from typing import Optional, Tuple
 
-__all__ = ["attn_fwd", "attn_fwd_static", "attn_decode", "workspace_bytes", "decode_workspace_bytes",
-           "device_status", "load_library",
+__all__ = ["attn_fwd", "attn_fwd_static", "attn_decode", "attn_bwd", "workspace_bytes",
+           "decode_workspace_bytes", "bwd_workspace_bytes", "device_status", "load_library",
            "FlintError", "LIB_PATH", "HQ", "HKV", "HEAD_DIM", "STATUS", "STATIC_SCRATCH_BYTES"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -64,6 +65,11 @@ def load_library() -> ctypes.CDLL:
         lib.flint_attn_decode.restype = ctypes.c_int
         lib.flint_attn_decode.argtypes = [P, P, P, P, P, P, P, P, P, I32, I32, I32, I32, F32, F32,
                                           P, P, P, ctypes.c_size_t, P]
+        lib.flint_attn_bwd_workspace_bytes.restype = ctypes.c_size_t
+        lib.flint_attn_bwd_workspace_bytes.argtypes = [I32]
+        lib.flint_attn_bwd.restype = ctypes.c_int
+        lib.flint_attn_bwd.argtypes = [P, P, P, P, P, P, P, P, I32, P, I32, I32, I32, I32, I32,
+                                       F32, F32, P, P, P, P, P, P, P, P, P, P, ctypes.c_size_t, P]
         lib.flint_attn_device_status.restype = ctypes.c_int
         lib.flint_attn_device_status.argtypes = [P, P]
         lib.flint_attn_last_error.restype = ctypes.c_char_p
@@ -215,6 +221,72 @@ def attn_decode(q, k, v, q_norm_w, k_norm_w, sinks, k_cache, v_cache, cache_len,
         raise FlintError(st, lib.flint_attn_last_error().decode())
     attn_decode.last_workspace = workspace
     return out, lse
+
+
+def bwd_workspace_bytes(T: int) -> int:
+    return int(load_library().flint_attn_bwd_workspace_bytes(int(T)))
+
+
+def attn_bwd(q, k, v, q_norm_w, k_norm_w, sinks, out, lse, dout, *, pos_ids=None,
+             cu_seqlens=None, pad_mask=None, window: int = 513, use_rope: bool = True,
+             rope_theta: float = 10000.0, eps: float = 1e-6, grads=None, workspace=None,
+             stream=None) -> dict:
+    """Gradient of attn_fwd (see include/flint_attn.h, flint_attn_bwd).
+
+    The forward's arguments, its out [T,4096] bf16 and lse [32,T] f32, and
+    dout [T,4096] bf16.  Returns a dict of float32 CUDA tensors: dq
+    [T,32,128], dk and dv [T,4,128], dq_norm_w and dk_norm_w [128], dsinks
+    [32] (``grads``: the same dict to write into).  Asynchronous on ``stream``.
+    """
+    import torch
+    lib = load_library()
+    T = int(q.shape[0]) if q.dim() >= 1 else 0
+    _check(q, "q", torch.bfloat16, (T, HQ, HEAD_DIM))
+    _check(k, "k", torch.bfloat16, (T, HKV, HEAD_DIM))
+    _check(v, "v", torch.bfloat16, (T, HKV, HEAD_DIM))
+    _check(q_norm_w, "q_norm_w", torch.float32, (HEAD_DIM,))
+    _check(k_norm_w, "k_norm_w", torch.float32, (HEAD_DIM,))
+    _check(sinks, "sinks", torch.float32, (HQ,))
+    _check(out, "out", torch.bfloat16, (T, HQ * HEAD_DIM))
+    _check(lse, "lse", torch.float32, (HQ, T))
+    _check(dout, "dout", torch.bfloat16, (T, HQ * HEAD_DIM))
+    num_docs, batch, seqlen = 0, 0, 0
+    if pos_ids is not None:
+        _check(pos_ids, "pos_ids", torch.int32, (T,))
+    if cu_seqlens is not None:
+        _check(cu_seqlens, "cu_seqlens", torch.int32)
+        num_docs = int(cu_seqlens.numel()) - 1
+    if pad_mask is not None:
+        _check(pad_mask, "pad_mask", torch.uint8)
+        if pad_mask.dim() != 2:
+            raise ValueError("pad_mask must be [batch, seqlen]")
+        batch, seqlen = int(pad_mask.shape[0]), int(pad_mask.shape[1])
+    dev = q.device
+    shapes = {"dq": (T, HQ, HEAD_DIM), "dk": (T, HKV, HEAD_DIM), "dv": (T, HKV, HEAD_DIM),
+              "dq_norm_w": (HEAD_DIM,), "dk_norm_w": (HEAD_DIM,), "dsinks": (HQ,)}
+    if grads is None:
+        grads = {n: torch.empty(sh, dtype=torch.float32, device=dev) for n, sh in shapes.items()}
+    for n, sh in shapes.items():
+        _check(grads[n], n, torch.float32, sh)
+    need = bwd_workspace_bytes(T)
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
+    _check(workspace, "workspace", torch.uint8)
+    if stream is None:
+        stream = torch.cuda.current_stream(dev)
+    sptr = stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+    with torch.cuda.device(dev):
+        st = lib.flint_attn_bwd(
+            _ptr(q), _ptr(k), _ptr(v), _ptr(q_norm_w), _ptr(k_norm_w), _ptr(sinks),
+            _ptr(pos_ids), _ptr(cu_seqlens), num_docs, _ptr(pad_mask), batch, seqlen, T,
+            int(window), int(bool(use_rope)), float(rope_theta), float(eps), _ptr(out),
+            _ptr(lse), _ptr(dout), _ptr(grads["dq"]), _ptr(grads["dk"]), _ptr(grads["dv"]),
+            _ptr(grads["dq_norm_w"]), _ptr(grads["dk_norm_w"]), _ptr(grads["dsinks"]),
+            _ptr(workspace), int(workspace.numel()), sptr)
+    if st != 0:
+        raise FlintError(st, lib.flint_attn_last_error().decode())
+    attn_bwd.last_workspace = workspace
+    return grads
 
 
 def device_status(workspace, stream=None) -> int:

@@ -297,6 +297,15 @@ flint_status_t run_decode(const void* q, const void* k, const void* v, const flo
                           int32_t use_rope, float rope_theta, float eps, void* out, float* lse,
                           void* workspace, size_t workspace_bytes, void* stream);
 
+size_t bwd_workspace_bytes(int T);
+flint_status_t run_bwd(const void* q, const void* k, const void* v, const float* q_norm_w,
+                       const float* k_norm_w, const float* sinks, const int32_t* pos_ids,
+                       const int32_t* cu_seqlens, int32_t num_docs, const uint8_t* pad_mask,
+                       int32_t batch, int32_t seqlen, int32_t T, int32_t window, int32_t use_rope,
+                       float rope_theta, float eps, const void* out, const float* lse, const void* dout,
+                       float* dq, float* dk, float* dv, float* dq_norm_w, float* dk_norm_w,
+                       float* dsinks, void* workspace, int sms, void* stream);
+
 }  // namespace flint
 
 extern "C" {
@@ -372,6 +381,67 @@ flint_status_t flint_attn_decode(const void* q, const void* k, const void* v, co
     return flint::run_decode(q, k, v, q_norm_w, k_norm_w, sinks, k_cache, v_cache, cache_len, B, cap,
                              window, use_rope, rope_theta, eps, out, lse, workspace, workspace_bytes,
                              stream);
+}
+
+size_t flint_attn_bwd_workspace_bytes(int32_t T) {
+    if (T < 0 || T > FLINT_MAX_TOKENS) return 0;
+    return flint::bwd_workspace_bytes(T);
+}
+
+flint_status_t flint_attn_bwd(const void* q, const void* k, const void* v, const float* q_norm_w,
+                              const float* k_norm_w, const float* sinks, const int32_t* pos_ids,
+                              const int32_t* cu_seqlens, int32_t num_docs, const uint8_t* pad_mask,
+                              int32_t batch, int32_t seqlen, int32_t T, int32_t window,
+                              int32_t use_rope, float rope_theta, float eps, const void* out,
+                              const float* lse, const void* dout, float* dq, float* dk, float* dv,
+                              float* dq_norm_w, float* dk_norm_w, float* dsinks, void* workspace,
+                              size_t workspace_bytes, void* stream) {
+    NvtxRange r("flint_attn_bwd");
+    g_err[0] = '\0';
+    if (T < 0 || T > FLINT_MAX_TOKENS)
+        return fail(FLINT_ERR_INVALID_ARG, "T=%d outside [0, %d]", T, FLINT_MAX_TOKENS);
+    if (window < 0) return fail(FLINT_ERR_INVALID_ARG, "window=%d < 0", window);
+    if (use_rope != 0 && use_rope != 1) return fail(FLINT_ERR_INVALID_ARG, "use_rope must be 0 or 1");
+    if (!(eps > 0.f) || !std::isfinite(eps)) return fail(FLINT_ERR_INVALID_ARG, "eps must be > 0");
+    if (use_rope && (!(rope_theta > 1.f) || !std::isfinite(rope_theta)))
+        return fail(FLINT_ERR_INVALID_ARG, "rope_theta must be > 1");
+    if (cu_seqlens && pad_mask)
+        return fail(FLINT_ERR_INVALID_ARG, "give at most one of cu_seqlens and pad_mask");
+    if (cu_seqlens && (num_docs < 0 || num_docs > FLINT_MAX_TOKENS))
+        return fail(FLINT_ERR_INVALID_ARG, "num_docs=%d", num_docs);
+    if (pad_mask && (batch < 1 || seqlen < 1 || (long long)batch * seqlen != (long long)T))
+        return fail(FLINT_ERR_INVALID_ARG, "pad_mask needs batch*seqlen == T (%d*%d vs %d)", batch,
+                    seqlen, T);
+    if (!dq_norm_w || !dk_norm_w || !dsinks) return fail(FLINT_ERR_INVALID_ARG, "null gradient pointer");
+    if (!aligned(dq_norm_w, 4) || !aligned(dk_norm_w, 4) || !aligned(dsinks, 4))
+        return fail(FLINT_ERR_INVALID_ARG, "misaligned 32-bit array");
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (T == 0) {
+        cudaError_t e = cudaMemsetAsync(dq_norm_w, 0, sizeof(float) * kHD, s);
+        if (e == cudaSuccess) e = cudaMemsetAsync(dk_norm_w, 0, sizeof(float) * kHD, s);
+        if (e == cudaSuccess) e = cudaMemsetAsync(dsinks, 0, sizeof(float) * kHQ, s);
+        if (e != cudaSuccess) return fail(FLINT_ERR_CUDA, "memset: %s", cudaGetErrorString(e));
+        return FLINT_OK;
+    }
+    if (!q || !k || !v || !q_norm_w || !k_norm_w || !sinks || !out || !lse || !dout || !dq || !dk || !dv)
+        return fail(FLINT_ERR_INVALID_ARG, "null tensor pointer");
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) ||
+        !aligned(dout, 16) || !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16))
+        return fail(FLINT_ERR_INVALID_ARG, "q, k, v, out, dout, dq, dk and dv must be 16-byte aligned");
+    if (!aligned(q_norm_w, 4) || !aligned(k_norm_w, 4) || !aligned(sinks, 4) || !aligned(lse, 4) ||
+        (pos_ids && !aligned(pos_ids, 4)) || (cu_seqlens && !aligned(cu_seqlens, 4)))
+        return fail(FLINT_ERR_INVALID_ARG, "misaligned 32-bit array");
+    const size_t need = flint::bwd_workspace_bytes(T);
+    if (!workspace || !aligned(workspace, 256))
+        return fail(FLINT_ERR_WORKSPACE, "workspace missing or not 256-byte aligned");
+    if (workspace_bytes < need)
+        return fail(FLINT_ERR_WORKSPACE, "workspace too small: %zu < %zu bytes", workspace_bytes, need);
+    int sms = 0;
+    flint_status_t st = device_setup(&sms);
+    if (st != FLINT_OK) return st;
+    return flint::run_bwd(q, k, v, q_norm_w, k_norm_w, sinks, pos_ids, cu_seqlens, num_docs, pad_mask,
+                          batch, seqlen, T, window, use_rope, rope_theta, eps, out, lse, dout, dq, dk, dv,
+                          dq_norm_w, dk_norm_w, dsinks, workspace, sms, stream);
 }
 
 flint_status_t flint_attn_device_status(const void* workspace, void* stream) {

@@ -1,6 +1,6 @@
 /*
- * flint_attn.h - C ABI of the B200 (sm_100a) sink-aware GQA attention forward
- * of the Flint hybrid-attention MoE decoder.
+ * flint_attn.h - C ABI of the B200 (sm_100a) sink-aware GQA attention of the
+ * Flint hybrid-attention MoE decoder: forward, its gradient, and a decode step.
  *
  * The operation is the core of FlintAttention.forward (NeMo AutoModel API
  * page "nemo_automodel.components.models.flint.layers", FlintAttention.forward:
@@ -257,7 +257,7 @@ FLINT_API flint_status_t flint_attn_fwd_static(const void* q, const void* k, con
  *  stream     cudaStream_t as void*.
  *
  * Queries, keys and scores are computed in FP32 on CUDA cores; the key
- * range of every (sequence, KV head) is split in blocks of 128 keys whose
+ * range of every (sequence, KV head) is split in blocks of 256 keys whose
  * partial results a second kernel combines with the sink.
  */
 FLINT_API size_t flint_attn_decode_workspace_bytes(int32_t B, int32_t cap, int32_t window);
@@ -268,6 +268,59 @@ FLINT_API flint_status_t flint_attn_decode(const void* q, const void* k, const v
                               int32_t window, int32_t use_rope, float rope_theta,
                               float eps, void* out, float* lse,
                               void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Gradient of flint_attn_fwd.  The "flint" model page (NeMo AutoModel,
+ * "Parallelism and backends") makes every head's sink a trainable FP32
+ * parameter whose adjoint needs care; the call computes the exact derivative
+ * of the forward defined above for a loss that depends on `out` (lse receives
+ * no gradient):
+ *
+ *   D_i = dO_i . out_i,  P_ij = exp(s_ij - lse_i),  dS_ij = P_ij (dO_i . v_j - D_i)
+ *   dv_j = sum P_ij dO_i,  dq~_i = sum_j dS_ij k~_j / sqrt(128),
+ *   dk~_j = sum dS_ij q~_i / sqrt(128),  dsink_h = -sum_i exp(sink_h - lse_i) D_i
+ *
+ * (sums over the query heads of a KV head where the operand is shared), then
+ * back through RoPE (rotation by -p) and the RMSNorm in weight form, which
+ * also gives the norm weights' gradients.
+ *
+ *  q, k, v, q_norm_w, k_norm_w, sinks, pos_ids, cu_seqlens, num_docs,
+ *  pad_mask, batch, seqlen, T, window, use_rope, rope_theta, eps
+ *             the forward's arguments, unchanged (same rules).
+ *  out        bf16 [T,4096]: the forward's result for these arguments.
+ *  lse        fp32 [32,T]: the forward's log-sum-exp (required here).
+ *  dout       bf16 [T,4096]: gradient of the loss with respect to out.
+ *  dq         fp32 [T,32,128]: gradient with respect to q (pre-norm).
+ *  dk, dv     fp32 [T,4,128]: gradients with respect to k (pre-norm) and v.
+ *  dq_norm_w, dk_norm_w   fp32 [128];  dsinks  fp32 [32].
+ *             Every gradient is overwritten, not accumulated; padded tokens
+ *             get zero rows.  q, k, v, out and dout must be 16-byte aligned,
+ *             dq, dk and dv too; no output may overlap an input, another
+ *             output or the workspace.
+ *  workspace  device buffer of at least flint_attn_bwd_workspace_bytes(T)
+ *             bytes (about 18.6 KiB per token), 256-byte aligned; holds the
+ *             device status (flint_attn_device_status: FLINT_ERR_INVALID_ARG
+ *             for an ill-formed cu_seqlens, FLINT_ERR_UNSUPPORTED for a
+ *             non-trailing mask), per-token document bounds, FP32 q~ and k~
+ *             and per-CTA partial sums.
+ *  stream     cudaStream_t as void*.
+ *
+ * T == 0 sets dq_norm_w, dk_norm_w and dsinks to zero and does nothing else.
+ * Computed in FP32 on CUDA cores; the norm-weight and sink gradients are
+ * summed in a fixed order, so repeated calls give identical bits.
+ */
+FLINT_API size_t flint_attn_bwd_workspace_bytes(int32_t T);
+FLINT_API flint_status_t flint_attn_bwd(const void* q, const void* k, const void* v,
+                           const float* q_norm_w, const float* k_norm_w,
+                           const float* sinks, const int32_t* pos_ids,
+                           const int32_t* cu_seqlens, int32_t num_docs,
+                           const uint8_t* pad_mask, int32_t batch, int32_t seqlen,
+                           int32_t T, int32_t window, int32_t use_rope,
+                           float rope_theta, float eps, const void* out,
+                           const float* lse, const void* dout, float* dq, float* dk,
+                           float* dv, float* dq_norm_w, float* dk_norm_w,
+                           float* dsinks, void* workspace, size_t workspace_bytes,
+                           void* stream);
 
 /* Text of the last error raised on the calling host thread ("" if none). */
 FLINT_API const char* flint_attn_last_error(void);

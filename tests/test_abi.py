@@ -173,3 +173,62 @@ def test_decode_invalid_arguments_rejected_on_host(lib, kw, status):
 def test_decode_empty_batch_is_a_noop(lib):
     assert call_decode(lib, B=0) == 0
     assert call_decode(lib, B=0, q=None, kc=None, out=None, ws=None) == 0
+
+
+# ---------------------------------------------------------------- backward entry
+
+def call_bwd(lib, **kw):
+    args = dict(q=A, k=A, v=A, wq=A, wk=A, sinks=A, pos=None, cu=None, ndocs=0, mask=None,
+                batch=0, seqlen=0, T=64, window=513, use_rope=1, theta=1e4, eps=1e-6,
+                out=A, lse=A, dout=A, dq=A, dk=A, dv=A, dwq=A, dwk=A, dsinks=A,
+                ws=A, ws_bytes=1 << 40, stream=None)
+    args.update(kw)
+    return lib.flint_attn_bwd(args["q"], args["k"], args["v"], args["wq"], args["wk"], args["sinks"],
+                              args["pos"], args["cu"], args["ndocs"], args["mask"], args["batch"],
+                              args["seqlen"], args["T"], args["window"], args["use_rope"],
+                              args["theta"], args["eps"], args["out"], args["lse"], args["dout"],
+                              args["dq"], args["dk"], args["dv"], args["dwq"], args["dwk"],
+                              args["dsinks"], args["ws"], args["ws_bytes"], args["stream"])
+
+
+def test_bwd_workspace_bytes(lib):
+    # FP32 q~ and k~ dominate: 18 KiB per token, plus fixed per-CTA partials
+    a = fa.bwd_workspace_bytes(4096)
+    assert 4096 * (16384 + 2048) <= a < 4096 * (16384 + 2048 + 512) + (4 << 20)
+    assert fa.bwd_workspace_bytes(0) > 0
+    assert fa.bwd_workspace_bytes(-1) == 0
+    assert fa.bwd_workspace_bytes((1 << 24) + 1) == 0
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(T=-1), 1),
+    (dict(T=(1 << 24) + 1), 1),
+    (dict(window=-1), 1),
+    (dict(use_rope=2), 1),
+    (dict(eps=0.0), 1),
+    (dict(theta=0.5), 1),
+    (dict(cu=A, mask=A), 1),
+    (dict(cu=A, ndocs=-2), 1),
+    (dict(mask=A, batch=3, seqlen=5, T=16), 1),
+    (dict(dsinks=None), 1),
+    (dict(dwq=A + 2), 1),
+    (dict(q=None), 1),
+    (dict(lse=None), 1),
+    (dict(dout=None), 1),
+    (dict(dq=None), 1),
+    (dict(dv=None), 1),
+    (dict(dout=A + 8), 1),
+    (dict(dk=A + 4), 1),
+    (dict(lse=A + 2), 1),
+    (dict(ws=None), 5),
+    (dict(ws=A + 64), 5),
+    (dict(ws_bytes=4096), 5),
+])
+def test_bwd_invalid_arguments_rejected_on_host(lib, kw, status):
+    assert call_bwd(lib, **kw) == status
+    assert lib.flint_attn_last_error() != b""
+
+
+def test_bwd_empty_input_checks_the_small_gradients_first(lib):
+    # T == 0 zeroes dq_norm_w, dk_norm_w and dsinks, so those must be given
+    assert call_bwd(lib, T=0, dwk=None) == 1
