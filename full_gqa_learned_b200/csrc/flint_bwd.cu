@@ -21,9 +21,10 @@
 //   bwd_segments_kernel  document bounds of every token (THD boundaries or a
 //                        trailing-padding mask), validated
 //   bwd_prep_kernel      q~, k~ in FP32 and D per (token, head)
-//   bwd_dq_kernel        one warp per (query token, head): loops over its keys
-//   bwd_dkv_kernel       one CTA per (key token, KV head), a warp per query
-//                        head of the group: loops over the key's queries
+//   bwd_dq_kernel        a warp per (query token, 4 query heads of a KV
+//                        head): loops over the token's keys
+//   bwd_dkv_kernel       a warp pair per (key token, KV head), 4 query heads
+//                        per warp: loops over the key's queries
 //   bwd_finish_kernel    sums the per-CTA partials of dq_norm_w, dk_norm_w
 //                        and dsinks in a fixed order (deterministic)
 #include <cuda_bf16.h>
@@ -165,36 +166,6 @@ __device__ __forceinline__ void norm_rope(const float x[4], const float* w, floa
     }
 }
 
-// Adjoint of norm_rope: dy (gradient of the rotated row) -> dx; adds the
-// row's contribution dn * x * r to dw[4].
-__device__ __forceinline__ void norm_rope_bwd(const float x[4], const float* w, float eps, bool rope,
-                                              int pos, const double* inv, int lane, const float dy[4],
-                                              float dx[4], float dw[4]) {
-    float dn[4] = {dy[0], dy[1], dy[2], dy[3]};
-    if (rope) {
-#pragma unroll
-        for (int i = 0; i < 2; ++i) {
-            float c, s;
-            rope_cos_sin(pos, inv[lane + 32 * i], &c, &s);
-            const float a = dy[i], b = dy[i + 2];
-            dn[i] = a * c + b * s;
-            dn[i + 2] = b * c - a * s;
-        }
-    }
-    const float ss = warp_sum(x[0] * x[0] + x[1] * x[1] + x[2] * x[2] + x[3] * x[3]);
-    const float r = rsqrtf(ss * (1.f / kHD) + eps);
-    float t = 0.f;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) t += w[lane + 32 * i] * dn[i] * x[i];
-    t = warp_sum(t);
-    const float c3 = r * r * r * t * (1.f / kHD);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        dx[i] = r * w[lane + 32 * i] * dn[i] - x[i] * c3;
-        dw[i] += dn[i] * x[i] * r;
-    }
-}
-
 __device__ __forceinline__ void load_inv_freq(double* s_inv, float theta) {
     if (threadIdx.x < 64) s_inv[threadIdx.x] = exp2(-(double)threadIdx.x / 64.0 * log2((double)theta));
 }
@@ -241,178 +212,290 @@ __device__ __forceinline__ float sink_share(float sink, float lse) {
     return expf(sink - lse);
 }
 
-// ---- dq: unit u = (query token i, KV head g), longest rows first; warp w takes head 8g+w
+// Row layout of the dq and dk/dv loops: a warp carries 4 rows (4 query heads
+// of one KV head), 8 lanes per row.  Lane l = 8 r + sub holds row r's
+// channels 8 sub .. 8 sub + 7 and 64 + 8 sub .. 64 + 8 sub + 7 (16 values,
+// index e), so each RoPE pair (c, c + 64) sits in one lane (e and e + 8) and
+// a row's dot product needs 3 shuffle levels within its 8 lanes.
+constexpr int kRowLanes = 8;
+
+__device__ __forceinline__ int lane_ch(int sub, int e) { return (e < 8 ? 0 : 56) + 8 * sub + e; }
+
+__device__ __forceinline__ float group_sum(float x) {
+    x += __shfl_xor_sync(0xffffffffu, x, 1);
+    x += __shfl_xor_sync(0xffffffffu, x, 2);
+    x += __shfl_xor_sync(0xffffffffu, x, 4);
+    return x;
+}
+
+// 16 FP32 values of a row (two runs of 8 channels), 16-byte loads
+__device__ __forceinline__ void load16f(const float* row, int sub, float v[16]) {
+    const float4* a = reinterpret_cast<const float4*>(row + 8 * sub);
+    const float4* b = reinterpret_cast<const float4*>(row + 64 + 8 * sub);
+    const float4 x0 = a[0], x1 = a[1], y0 = b[0], y1 = b[1];
+    v[0] = x0.x; v[1] = x0.y; v[2] = x0.z; v[3] = x0.w; v[4] = x1.x; v[5] = x1.y; v[6] = x1.z; v[7] = x1.w;
+    v[8] = y0.x; v[9] = y0.y; v[10] = y0.z; v[11] = y0.w; v[12] = y1.x; v[13] = y1.y; v[14] = y1.z; v[15] = y1.w;
+}
+
+__device__ __forceinline__ void unpack8(uint4 u, float* v) {
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        v[2 * i] = __uint_as_float(w[i] << 16);
+        v[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+    }
+}
+
+// 16 BF16 values of a row, widened to FP32
+__device__ __forceinline__ void load16h(const __nv_bfloat16* row, int sub, float v[16]) {
+    const uint4 a = *reinterpret_cast<const uint4*>(row + 8 * sub);
+    const uint4 b = *reinterpret_cast<const uint4*>(row + 64 + 8 * sub);
+    unpack8(a, v);
+    unpack8(b, v + 8);
+}
+
+__device__ __forceinline__ void store16f(float* row, int sub, const float v[16]) {
+    float4* a = reinterpret_cast<float4*>(row + 8 * sub);
+    float4* b = reinterpret_cast<float4*>(row + 64 + 8 * sub);
+    a[0] = make_float4(v[0], v[1], v[2], v[3]);
+    a[1] = make_float4(v[4], v[5], v[6], v[7]);
+    b[0] = make_float4(v[8], v[9], v[10], v[11]);
+    b[1] = make_float4(v[12], v[13], v[14], v[15]);
+}
+
+// Adjoint of RMSNorm (weight form) then RoPE for one row in the 8-lane
+// layout: dy (gradient of the rotated row) -> dx; adds dn * x * r to dw.
+__device__ __forceinline__ void norm_rope_bwd16(const float x[16], const float* w, float eps, bool rope,
+                                                int pos, const double* inv, int sub, const float dy[16],
+                                                float dx[16], float dw[16]) {
+    float dn[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e) dn[e] = dy[e];
+    if (rope) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            float c, s;
+            rope_cos_sin(pos, inv[8 * sub + e], &c, &s);
+            const float a = dy[e], b = dy[e + 8];
+            dn[e] = a * c + b * s;
+            dn[e + 8] = b * c - a * s;
+        }
+    }
+    float ss = 0.f, t = 0.f;
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+        ss = fmaf(x[e], x[e], ss);
+        t = fmaf(w[lane_ch(sub, e)] * dn[e], x[e], t);
+    }
+    ss = group_sum(ss);
+    t = group_sum(t);
+    const float r = rsqrtf(ss * (1.f / kHD) + eps);
+    const float c3 = r * r * r * t * (1.f / kHD);
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+        dx[e] = r * w[lane_ch(sub, e)] * dn[e] - x[e] * c3;
+        dw[e] = fmaf(dn[e] * x[e], r, dw[e]);
+    }
+}
+
+// ---- dq: work item = (query token i, KV head g, half) -> query heads
+// 8g + 4 half .. + 3, one per 8-lane row; longest rows first
 __global__ void __launch_bounds__(kBwdThreads) bwd_dq_kernel(const BwdParams p) {
     __shared__ double s_inv[64];
     __shared__ float s_w[kHD];
     __shared__ float s_dsink[kHQ];
-    __shared__ float s_dw[kBwdThreads / 32][kHD];
+    __shared__ float s_dw[kBwdThreads / kRowLanes][kHD];
     load_inv_freq(s_inv, p.rope_theta);
     if (threadIdx.x < kHD) s_w[threadIdx.x] = p.q_norm_w[threadIdx.x];
     if (threadIdx.x < kHQ) s_dsink[threadIdx.x] = 0.f;
     __syncthreads();
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int r = lane >> 3, sub = lane & 7;
     const float scale = 0.08838834764831845f;            // 1/sqrt(128)
     const float scale_log2e = scale * 1.4426950408889634f;
-    float dw[4] = {0.f, 0.f, 0.f, 0.f};
-    const int units = p.T * kHKV;
-    for (int u = blockIdx.x; u < units; u += gridDim.x) {
-        const int i = p.T - 1 - u / kHKV, g = u % kHKV, h = g * kGroup + warp;
+    float dw[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e) dw[e] = 0.f;
+    const int items = p.T * kHKV * 2;
+    const int nwarps = gridDim.x * (kBwdThreads / 32);
+    for (int it = blockIdx.x * (kBwdThreads / 32) + warp; it < items; it += nwarps) {
+        const int i = p.T - 1 - it / (kHKV * 2), g = (it >> 1) % kHKV, half = it & 1;
+        const int h = g * kGroup + half * 4 + r;
         const size_t qrow = (size_t)i * kHQ + h;
         float* dq = p.dq + qrow * kHD;
-        const int seg = p.seg_lo[i];
-        if (seg < 0) {
+        const int seg = p.seg_lo[i];                       // same for the whole warp
+        float acc[16];
 #pragma unroll
-            for (int c = 0; c < 4; ++c) dq[lane + 32 * c] = 0.f;
+        for (int e = 0; e < 16; ++e) acc[e] = 0.f;
+        if (seg < 0) {
+            store16f(dq, sub, acc);
             continue;
         }
         const int lo = p.window > 0 ? max(seg, i - p.window + 1) : seg;
-        float qt[4], dO[4], acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-            qt[c] = p.qt[qrow * kHD + lane + 32 * c];
-            dO[c] = bf(p.dout, qrow * kHD + lane + 32 * c);
-        }
+        float qt[16], dO[16];
+        load16f(p.qt + qrow * kHD, sub, qt);
+        load16h(p.dout + qrow * kHD, sub, dO);
         const float D = p.delta[qrow];
-        const float L = p.lse[(size_t)h * p.T + i];
         const float sink = p.sinks[h];
-        if (!(isinf(sink) && sink > 0.f)) {
-            const float Ll2 = L * 1.4426950408889634f;
-            for (int j = lo; j <= i; ++j) {
-                const size_t krow = ((size_t)j * kHKV + g) * kHD;
-                float kv[4], vv[4];
+        // a +inf sink: out = 0 and no gradient; an lse of +inf makes every P 0
+        const float L = (isinf(sink) && sink > 0.f) ? INFINITY : p.lse[(size_t)h * p.T + i];
+        const float Ll2 = L * 1.4426950408889634f;
+#pragma unroll 2
+        for (int j = lo; j <= i; ++j) {
+            const size_t krow = ((size_t)j * kHKV + g) * kHD;
+            float kv[16], vv[16];
+            load16f(p.kt + krow, sub, kv);
+            load16h(p.v + krow, sub, vv);
+            float s = 0.f, dp = 0.f;
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    kv[c] = p.kt[krow + lane + 32 * c];
-                    vv[c] = bf(p.v, krow + lane + 32 * c);
-                }
-                float s = qt[0] * kv[0] + qt[1] * kv[1] + qt[2] * kv[2] + qt[3] * kv[3];
-                float dp = dO[0] * vv[0] + dO[1] * vv[1] + dO[2] * vv[2] + dO[3] * vv[3];
-#pragma unroll
-                for (int o = 16; o > 0; o >>= 1) {
-                    s += __shfl_xor_sync(0xffffffffu, s, o);
-                    dp += __shfl_xor_sync(0xffffffffu, dp, o);
-                }
-                const float pr = exp2f(fmaf(s, scale_log2e, -Ll2));
-                const float ds = pr * (dp - D);
-#pragma unroll
-                for (int c = 0; c < 4; ++c) acc[c] = fmaf(ds, kv[c], acc[c]);
+            for (int e = 0; e < 16; ++e) {
+                s = fmaf(qt[e], kv[e], s);
+                dp = fmaf(dO[e], vv[e], dp);
             }
-            if (lane == 0) atomicAdd(&s_dsink[h], -sink_share(sink, L) * D);
-        }
-        float x[4], dy[4], dx[4];
+            s = group_sum(s);
+            dp = group_sum(dp);
+            const float pr = exp2f(fmaf(s, scale_log2e, -Ll2));
+            const float ds = pr * (dp - D);
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-            x[c] = bf(p.q, qrow * kHD + lane + 32 * c);
-            dy[c] = acc[c] * scale;
+            for (int e = 0; e < 16; ++e) acc[e] = fmaf(ds, kv[e], acc[e]);
         }
-        norm_rope_bwd(x, s_w, p.eps, p.use_rope != 0, token_pos(p, i), s_inv, lane, dy, dx, dw);
+        if (sub == 0) atomicAdd(&s_dsink[h], -sink_share(sink, L) * D);
+        float x[16], dy[16], dx[16];
+        load16h(p.q + qrow * kHD, sub, x);
 #pragma unroll
-        for (int c = 0; c < 4; ++c) dq[lane + 32 * c] = dx[c];
+        for (int e = 0; e < 16; ++e) dy[e] = acc[e] * scale;
+        norm_rope_bwd16(x, s_w, p.eps, p.use_rope != 0, token_pos(p, i), s_inv, sub, dy, dx, dw);
+        store16f(dq, sub, dx);
     }
 #pragma unroll
-    for (int c = 0; c < 4; ++c) s_dw[warp][lane + 32 * c] = dw[c];
+    for (int e = 0; e < 16; ++e) s_dw[warp * 4 + r][lane_ch(sub, e)] = dw[e];
     __syncthreads();
     float* part = p.part_q + (size_t)blockIdx.x * kBwdPartQ;
     if (threadIdx.x < kHD) {
         float s = 0.f;
-        for (int w = 0; w < kBwdThreads / 32; ++w) s += s_dw[w][threadIdx.x];
+        for (int k = 0; k < kBwdThreads / kRowLanes; ++k) s += s_dw[k][threadIdx.x];
         part[threadIdx.x] = s;
     } else if (threadIdx.x < kHD + kHQ) {
         part[threadIdx.x] = s_dsink[threadIdx.x - kHD];
     }
 }
 
-// ---- dk, dv: unit u = (key token j, KV head g); warp w takes query head 8g+w
-__global__ void __launch_bounds__(kBwdThreads) bwd_dkv_kernel(const BwdParams p) {
+__device__ __forceinline__ void pair_barrier(int pair) {
+    asm volatile("bar.sync %0, 64;" ::"r"(1 + pair) : "memory");
+}
+
+// ---- dk, dv: work item = (key token j, KV head g), taken by a pair of warps
+// (half 0: query heads 8g .. 8g+3, half 1: 8g+4 .. 8g+7), 4 pairs per CTA
+__global__ void __launch_bounds__(kBwdThreads, 2) bwd_dkv_kernel(const BwdParams p) {
+    constexpr int kPairs = kBwdThreads / 64;
     __shared__ double s_inv[64];
     __shared__ float s_w[kHD];
-    __shared__ float s_red[kBwdThreads / 32][2 * kHD];
+    __shared__ float s_red[kPairs][2][2 * kHD];            // per warp: dk~ (128), dv (128)
+    __shared__ float s_dw[kPairs][kHD];
     load_inv_freq(s_inv, p.rope_theta);
     if (threadIdx.x < kHD) s_w[threadIdx.x] = p.k_norm_w[threadIdx.x];
+    for (int t = threadIdx.x; t < kPairs * kHD; t += kBwdThreads) (&s_dw[0][0])[t] = 0.f;
+    __syncthreads();
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int r = lane >> 3, sub = lane & 7, pair = warp >> 1, half = warp & 1;
     const float scale = 0.08838834764831845f;
     const float scale_log2e = scale * 1.4426950408889634f;
-    float dw[4] = {0.f, 0.f, 0.f, 0.f};                  // warp 0 only
-    const int units = p.T * kHKV;
-    for (int u = blockIdx.x; u < units; u += gridDim.x) {
-        const int j = u / kHKV, g = u % kHKV, h = g * kGroup + warp;
+    const int items = p.T * kHKV;
+    for (int it = blockIdx.x * kPairs + pair; it < items; it += gridDim.x * kPairs) {
+        const int j = it / kHKV, g = it % kHKV;
+        const int h = g * kGroup + half * 4 + r;
         const size_t krow = (size_t)j * kHKV + g;
-        const int seg = p.seg_lo[j];
-        __syncthreads();                                  // s_red of the previous unit is consumed
+        const int seg = p.seg_lo[j];                        // same for both warps of the pair
         if (seg < 0) {
-            if (warp == 0) {
+            if (half == 0 && r == 0) {
+                float z[16];
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    p.dk[krow * kHD + lane + 32 * c] = 0.f;
-                    p.dv[krow * kHD + lane + 32 * c] = 0.f;
-                }
+                for (int e = 0; e < 16; ++e) z[e] = 0.f;
+                store16f(p.dk + krow * kHD, sub, z);
+                store16f(p.dv + krow * kHD, sub, z);
             }
-            continue;                                     // uniform over the CTA
+            continue;
         }
         const int hi = p.window > 0 ? (int)min((long long)p.seg_hi[j], (long long)j + p.window)
                                     : p.seg_hi[j];
-        float kv[4], vv[4], dk[4] = {0.f, 0.f, 0.f, 0.f}, dv[4] = {0.f, 0.f, 0.f, 0.f};
+        float kv[16], vv[16], dk[16], dv[16];
+        load16f(p.kt + krow * kHD, sub, kv);
+        load16h(p.v + krow * kHD, sub, vv);
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-            kv[c] = p.kt[krow * kHD + lane + 32 * c];
-            vv[c] = bf(p.v, krow * kHD + lane + 32 * c);
-        }
+        for (int e = 0; e < 16; ++e) { dk[e] = 0.f; dv[e] = 0.f; }
         const float sink = p.sinks[h];
-        if (!(isinf(sink) && sink > 0.f)) {
-            for (int i = j; i < hi; ++i) {
-                const size_t qrow = (size_t)i * kHQ + h;
-                float qt[4], dO[4];
+        const bool dead = isinf(sink) && sink > 0.f;        // +inf sink: every P is 0
+        for (int i = j; i < hi; ++i) {
+            const size_t qrow = (size_t)i * kHQ + h;
+            float qt[16], dO[16];
+            load16f(p.qt + qrow * kHD, sub, qt);
+            load16h(p.dout + qrow * kHD, sub, dO);
+            const float L = dead ? INFINITY : p.lse[(size_t)h * p.T + i];
+            const float D = p.delta[qrow];
+            float s = 0.f, dp = 0.f;
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    qt[c] = p.qt[qrow * kHD + lane + 32 * c];
-                    dO[c] = bf(p.dout, qrow * kHD + lane + 32 * c);
-                }
-                float s = qt[0] * kv[0] + qt[1] * kv[1] + qt[2] * kv[2] + qt[3] * kv[3];
-                float dp = dO[0] * vv[0] + dO[1] * vv[1] + dO[2] * vv[2] + dO[3] * vv[3];
+            for (int e = 0; e < 16; ++e) {
+                s = fmaf(qt[e], kv[e], s);
+                dp = fmaf(dO[e], vv[e], dp);
+            }
+            s = group_sum(s);
+            dp = group_sum(dp);
+            const float pr = exp2f(fmaf(s, scale_log2e, -L * 1.4426950408889634f));
+            const float ds = pr * (dp - D);
 #pragma unroll
-                for (int o = 16; o > 0; o >>= 1) {
-                    s += __shfl_xor_sync(0xffffffffu, s, o);
-                    dp += __shfl_xor_sync(0xffffffffu, dp, o);
-                }
-                const float L = p.lse[(size_t)h * p.T + i];
-                const float pr = exp2f(fmaf(s, scale_log2e, -L * 1.4426950408889634f));
-                const float ds = pr * (dp - p.delta[qrow]);
-#pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    dk[c] = fmaf(ds, qt[c], dk[c]);
-                    dv[c] = fmaf(pr, dO[c], dv[c]);
-                }
+            for (int e = 0; e < 16; ++e) {
+                dk[e] = fmaf(ds, qt[e], dk[e]);
+                dv[e] = fmaf(pr, dO[e], dv[e]);
             }
         }
+        // sum the warp's 4 rows (lane bits 3 and 4), then the pair's 2 warps
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-            s_red[warp][lane + 32 * c] = dk[c];
-            s_red[warp][kHD + lane + 32 * c] = dv[c];
+        for (int e = 0; e < 16; ++e) {
+            dk[e] += __shfl_xor_sync(0xffffffffu, dk[e], 8);
+            dk[e] += __shfl_xor_sync(0xffffffffu, dk[e], 16);
+            dv[e] += __shfl_xor_sync(0xffffffffu, dv[e], 8);
+            dv[e] += __shfl_xor_sync(0xffffffffu, dv[e], 16);
         }
-        __syncthreads();
-        if (warp == 0) {
-            float dy[4], x[4], dx[4];
+        if (r == 0) {
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                float sk = 0.f, sv = 0.f;
-                for (int w = 0; w < kBwdThreads / 32; ++w) {
-                    sk += s_red[w][lane + 32 * c];
-                    sv += s_red[w][kHD + lane + 32 * c];
-                }
-                dy[c] = sk * scale;
-                p.dv[krow * kHD + lane + 32 * c] = sv;
-                x[c] = bf(p.k, krow * kHD + lane + 32 * c);
+            for (int e = 0; e < 16; ++e) {
+                s_red[pair][half][lane_ch(sub, e)] = dk[e];
+                s_red[pair][half][kHD + lane_ch(sub, e)] = dv[e];
             }
-            norm_rope_bwd(x, s_w, p.eps, p.use_rope != 0, token_pos(p, j), s_inv, lane, dy, dx, dw);
-#pragma unroll
-            for (int c = 0; c < 4; ++c) p.dk[krow * kHD + lane + 32 * c] = dx[c];
         }
+        pair_barrier(pair);
+        if (half == 0) {
+            // every row group of warp 0 computes the key's adjoint (the
+            // shuffles need the whole warp); row group 0 writes the results
+            // and adds the key's k_norm_w share to the pair's row of s_dw
+            if (r == 0) {
+                float dvs[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e)
+                    dvs[e] = s_red[pair][0][kHD + lane_ch(sub, e)] + s_red[pair][1][kHD + lane_ch(sub, e)];
+                store16f(p.dv + krow * kHD, sub, dvs);
+            }
+            float dy[16], x[16], dx[16], dw[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+                dy[e] = (s_red[pair][0][lane_ch(sub, e)] + s_red[pair][1][lane_ch(sub, e)]) * scale;
+                dw[e] = 0.f;
+            }
+            load16h(p.k + krow * kHD, sub, x);
+            norm_rope_bwd16(x, s_w, p.eps, p.use_rope != 0, token_pos(p, j), s_inv, sub, dy, dx, dw);
+            if (r == 0) {
+                store16f(p.dk + krow * kHD, sub, dx);
+#pragma unroll
+                for (int e = 0; e < 16; ++e) s_dw[pair][lane_ch(sub, e)] += dw[e];
+            }
+        }
+        pair_barrier(pair);                                 // s_red is free for the next item
     }
-    if (warp == 0) {
-        float* part = p.part_k + (size_t)blockIdx.x * kHD;
-#pragma unroll
-        for (int c = 0; c < 4; ++c) part[lane + 32 * c] = dw[c];
+    __syncthreads();
+    if (threadIdx.x < kHD) {
+        float s = 0.f;
+        for (int k = 0; k < kPairs; ++k) s += s_dw[k][threadIdx.x];
+        p.part_k[(size_t)blockIdx.x * kHD + threadIdx.x] = s;
     }
 }
 
@@ -490,11 +573,19 @@ flint_status_t run_bwd(const void* q, const void* k, const void* v, const float*
         nseg = batch;
     }
     bp.nseg = nseg;
-    const int units = T * kHKV;
-    int grid = sms * 8;
-    if (grid > kBwdMaxBlocks) grid = kBwdMaxBlocks;
-    if (grid > units) grid = units;
-    bp.grid = grid;
+    // dq: T x 8 warp items, 8 per CTA; dk/dv: T x 4 pair items, 4 per CTA;
+    // both grids one wave of resident CTAs (capped by the partial arrays)
+    int occ_q = 0, occ_k = 0;
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ_q, bwd_dq_kernel, kBwdThreads, 0);
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ_k, bwd_dkv_kernel, kBwdThreads, 0);
+    auto grid_for = [&](int occ) {
+        long long g = (long long)sms * (occ > 0 ? occ : 1);
+        if (g > kBwdMaxBlocks) g = kBwdMaxBlocks;
+        if (g > T) g = T;
+        return (int)g;
+    };
+    const int grid_q = grid_for(occ_q), grid_k = grid_for(occ_k);
+    bp.grid = grid_q;
 
     cudaError_t e = cudaMemsetAsync(ws, 0, 256, s);
     if (e == cudaSuccess) e = cudaMemsetAsync(bp.seg_lo, 0xff, sizeof(int) * (size_t)T, s);
@@ -510,13 +601,13 @@ flint_status_t run_bwd(const void* q, const void* k, const void* v, const float*
     bwd_prep_kernel<<<(unsigned)prep_grid, kBwdThreads, 0, s>>>(bp);
     e = cudaGetLastError();
     if (e != cudaSuccess) return set_error(FLINT_ERR_CUDA, "backward: prep launch failed");
-    bwd_dq_kernel<<<grid, kBwdThreads, 0, s>>>(bp);
+    bwd_dq_kernel<<<grid_q, kBwdThreads, 0, s>>>(bp);
     e = cudaGetLastError();
     if (e != cudaSuccess) return set_error(FLINT_ERR_CUDA, "backward: dq launch failed");
-    bwd_dkv_kernel<<<grid, kBwdThreads, 0, s>>>(bp);
+    bwd_dkv_kernel<<<grid_k, kBwdThreads, 0, s>>>(bp);
     e = cudaGetLastError();
     if (e != cudaSuccess) return set_error(FLINT_ERR_CUDA, "backward: dk/dv launch failed");
-    bwd_finish_kernel<<<1, kHD + kHQ, 0, s>>>(bp, grid, grid);
+    bwd_finish_kernel<<<1, kHD + kHQ, 0, s>>>(bp, grid_q, grid_k);
     e = cudaGetLastError();
     if (e != cudaSuccess) return set_error(FLINT_ERR_CUDA, "backward: finish launch failed");
     return FLINT_OK;
