@@ -228,6 +228,20 @@ __device__ __forceinline__ float group_sum(float x) {
     return x;
 }
 
+// Dot products of a row pair over a lane's 16 channels, as four independent
+// partial sums each (short dependency chains), then summed over the row's 8 lanes.
+__device__ __forceinline__ void dot2_16(const float a[16], const float b[16], const float c[16],
+                                        const float d[16], float* ab, float* cd) {
+    float x[4] = {0.f, 0.f, 0.f, 0.f}, y[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+        x[e & 3] = fmaf(a[e], b[e], x[e & 3]);
+        y[e & 3] = fmaf(c[e], d[e], y[e & 3]);
+    }
+    *ab = group_sum((x[0] + x[1]) + (x[2] + x[3]));
+    *cd = group_sum((y[0] + y[1]) + (y[2] + y[3]));
+}
+
 // 16 FP32 values of a row (two runs of 8 channels), 16-byte loads
 __device__ __forceinline__ void load16f(const float* row, int sub, float v[16]) {
     const float4* a = reinterpret_cast<const float4*>(row + 8 * sub);
@@ -346,14 +360,8 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_dq_kernel(const BwdParams p) 
             float kv[16], vv[16];
             load16f(p.kt + krow, sub, kv);
             load16h(p.v + krow, sub, vv);
-            float s = 0.f, dp = 0.f;
-#pragma unroll
-            for (int e = 0; e < 16; ++e) {
-                s = fmaf(qt[e], kv[e], s);
-                dp = fmaf(dO[e], vv[e], dp);
-            }
-            s = group_sum(s);
-            dp = group_sum(dp);
+            float s, dp;
+            dot2_16(qt, kv, dO, vv, &s, &dp);
             const float pr = exp2f(fmaf(s, scale_log2e, -Ll2));
             const float ds = pr * (dp - D);
 #pragma unroll
@@ -432,14 +440,8 @@ __global__ void __launch_bounds__(kBwdThreads, 2) bwd_dkv_kernel(const BwdParams
             load16h(p.dout + qrow * kHD, sub, dO);
             const float L = dead ? INFINITY : p.lse[(size_t)h * p.T + i];
             const float D = p.delta[qrow];
-            float s = 0.f, dp = 0.f;
-#pragma unroll
-            for (int e = 0; e < 16; ++e) {
-                s = fmaf(qt[e], kv[e], s);
-                dp = fmaf(dO[e], vv[e], dp);
-            }
-            s = group_sum(s);
-            dp = group_sum(dp);
+            float s, dp;
+            dot2_16(qt, kv, dO, vv, &s, &dp);
             const float pr = exp2f(fmaf(s, scale_log2e, -L * 1.4426950408889634f));
             const float ds = pr * (dp - D);
 #pragma unroll
