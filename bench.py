@@ -584,10 +584,8 @@ def bwd_cpu_baseline(w, budget_s):
     until a run takes about budget_s seconds: algorithmic FLOPs per second."""
     from threadpoolctl import threadpool_limits
     from oracle import backward as OB
-    rng = np.random.default_rng(1)
-    n, dt = 32, 0.0
     with threadpool_limits(limits=1):          # one BLAS thread: `cores` below is exact
-        return _bwd_cpu_sample(w, budget_s, OB, rng)
+        return _bwd_cpu_sample(w, budget_s, OB, np.random.default_rng(1))
 
 
 def _bwd_cpu_sample(w, budget_s, OB, rng):

@@ -85,9 +85,9 @@ struct BwdParams {
     float* delta;                // [T,32]: D
     float* qt;                   // [T,32,128]: q~
     float* kt;                   // [T,4,128]: k~
-    float* part_q;               // [grid,160]
-    float* part_k;               // [grid,128]
-    int T, nseg, batch, seqlen, window, use_rope, mode, grid;
+    float* part_q;               // [dq grid,160]
+    float* part_k;               // [dk/dv grid,128]
+    int T, nseg, batch, seqlen, window, use_rope, mode;
     float rope_theta, eps;
 };
 
@@ -587,7 +587,6 @@ flint_status_t run_bwd(const void* q, const void* k, const void* v, const float*
         return (int)g;
     };
     const int grid_q = grid_for(occ_q), grid_k = grid_for(occ_k);
-    bp.grid = grid_q;
 
     cudaError_t e = cudaMemsetAsync(ws, 0, 256, s);
     if (e == cudaSuccess) e = cudaMemsetAsync(bp.seg_lo, 0xff, sizeof(int) * (size_t)T, s);

@@ -41,3 +41,25 @@ def test_profile_records_traffic_and_hash():
     text = open(os.path.join(root, "profiles", "attn_fwd_kernel_full_s4096_ncu.md")).read()
     assert re.search(r"traffic_bytes_per_launch: \d+", text)
     assert re.search(r"kernel_source_sha256: [0-9a-f]{64}", text)
+
+
+def test_backward_flops_are_five_contractions_per_pair_and_head():
+    import workloads as W
+    w = W.make("sliding_s1024")
+    # forward: 2 contractions (QK^T, PV) x 2 FLOPs x 128 x 32 heads per pair
+    assert w.flops() == 2 * 2 * 128 * 32 * w.valid_pairs()
+    assert bench.bwd_flops(w) == 5 * 2 * 128 * 32 * w.valid_pairs()
+
+
+def test_backward_cpu_baseline_reports_one_thread_and_its_sample():
+    import workloads as W
+    r = bench.bwd_cpu_baseline(W.make("sliding_s1024"), budget_s=0.05)
+    assert r["kind"] == "oracle" and r["cores"] == 1 and r["unit"] == bench.UNIT
+    assert r["value"] > 0 and "first" in r["sample"] and "sliding_s1024" in r["sample"]
+
+
+def test_backward_workloads_are_selectable():
+    import workloads as W
+    for name in W.CONFIGS:
+        assert (bench.BWD_PREFIX + name)[len(bench.BWD_PREFIX):] == name
+    assert abs(bench.ALU_FP32_TFLOPS - 74.45) < 0.01
