@@ -317,11 +317,11 @@ __device__ __forceinline__ void norm_rope_bwd16(const float x[16], const float* 
 __global__ void __launch_bounds__(kBwdThreads) bwd_dq_kernel(const BwdParams p) {
     __shared__ double s_inv[64];
     __shared__ float s_w[kHD];
-    __shared__ float s_dsink[kHQ];
+    __shared__ float s_dsink[kBwdThreads / 32][kHQ];    // per warp: only that warp adds to its row
     __shared__ float s_dw[kBwdThreads / kRowLanes][kHD];
     load_inv_freq(s_inv, p.rope_theta);
     if (threadIdx.x < kHD) s_w[threadIdx.x] = p.q_norm_w[threadIdx.x];
-    if (threadIdx.x < kHQ) s_dsink[threadIdx.x] = 0.f;
+    for (int t = threadIdx.x; t < (kBwdThreads / 32) * kHQ; t += kBwdThreads) (&s_dsink[0][0])[t] = 0.f;
     __syncthreads();
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int r = lane >> 3, sub = lane & 7;
@@ -367,7 +367,8 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_dq_kernel(const BwdParams p) 
 #pragma unroll
             for (int e = 0; e < 16; ++e) acc[e] = fmaf(ds, kv[e], acc[e]);
         }
-        if (sub == 0) atomicAdd(&s_dsink[h], -sink_share(sink, L) * D);
+        // the warp's 4 rows are 4 different heads: plain adds in program order
+        if (sub == 0) s_dsink[warp][h] += -sink_share(sink, L) * D;
         float x[16], dy[16], dx[16];
         load16h(p.q + qrow * kHD, sub, x);
 #pragma unroll
@@ -384,7 +385,9 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_dq_kernel(const BwdParams p) 
         for (int k = 0; k < kBwdThreads / kRowLanes; ++k) s += s_dw[k][threadIdx.x];
         part[threadIdx.x] = s;
     } else if (threadIdx.x < kHD + kHQ) {
-        part[threadIdx.x] = s_dsink[threadIdx.x - kHD];
+        float s = 0.f;
+        for (int w = 0; w < kBwdThreads / 32; ++w) s += s_dsink[w][threadIdx.x - kHD];
+        part[threadIdx.x] = s;
     }
 }
 
