@@ -17,7 +17,7 @@ import os
 import threading
 from typing import Optional, Tuple
 
-__all__ = ["attn_fwd", "attn_fwd_static", "attn_decode", "attn_bwd", "workspace_bytes",
+__all__ = ["attn_fwd", "attn_fwd_static", "attn_decode", "attn_bwd", "flint_attention", "workspace_bytes",
            "decode_workspace_bytes", "bwd_workspace_bytes", "device_status", "load_library",
            "FlintError", "LIB_PATH", "HQ", "HKV", "HEAD_DIM", "STATUS", "STATIC_SCRATCH_BYTES"]
 
@@ -287,6 +287,61 @@ def attn_bwd(q, k, v, q_norm_w, k_norm_w, sinks, out, lse, dout, *, pos_ids=None
         raise FlintError(st, lib.flint_attn_last_error().decode())
     attn_bwd.last_workspace = workspace
     return grads
+
+
+def flint_attention(q, k, v, q_norm_w, k_norm_w, sinks, *, pos_ids=None, cu_seqlens=None,
+                    pad_mask=None, window: int = 513, use_rope: bool = True,
+                    rope_theta: float = 10000.0, eps: float = 1e-6):
+    """Differentiable forward: returns (out [T,4096] bf16, lse [32,T] f32).
+
+    Backpropagating a loss through ``out`` runs flint_attn_bwd and yields the
+    gradients of q, k, v (cast to their dtype), q_norm_w, k_norm_w and sinks.
+    lse is returned for inspection and receives no gradient.  Index and mask
+    arguments are not differentiable.
+    """
+    return _FlintAttnFn.apply(q, k, v, q_norm_w, k_norm_w, sinks, pos_ids, cu_seqlens, pad_mask,
+                              int(window), bool(use_rope), float(rope_theta), float(eps))
+
+
+def _make_autograd_fn():
+    import torch
+
+    class FlintAttnFn(torch.autograd.Function):
+        @staticmethod
+        def forward(ctx, q, k, v, q_norm_w, k_norm_w, sinks, pos_ids, cu_seqlens, pad_mask, window,
+                    use_rope, rope_theta, eps):
+            cfg = dict(pos_ids=pos_ids, cu_seqlens=cu_seqlens, pad_mask=pad_mask, window=window,
+                       use_rope=use_rope, rope_theta=rope_theta, eps=eps)
+            out, lse = attn_fwd(q, k, v, q_norm_w, k_norm_w, sinks, **cfg)
+            ctx.save_for_backward(q, k, v, q_norm_w, k_norm_w, sinks, out, lse)
+            ctx.cfg = cfg
+            ctx.mark_non_differentiable(lse)
+            return out, lse
+
+        @staticmethod
+        def backward(ctx, dout, _dlse):
+            q, k, v, q_norm_w, k_norm_w, sinks, out, lse = ctx.saved_tensors
+            g = attn_bwd(q, k, v, q_norm_w, k_norm_w, sinks, out, lse,
+                         dout.to(torch.bfloat16).contiguous(), **ctx.cfg)
+            return (g["dq"].to(q.dtype), g["dk"].to(k.dtype), g["dv"].to(v.dtype),
+                    g["dq_norm_w"].to(q_norm_w.dtype), g["dk_norm_w"].to(k_norm_w.dtype),
+                    g["dsinks"].to(sinks.dtype), None, None, None, None, None, None, None)
+
+    return FlintAttnFn
+
+
+class _LazyFn:
+    """Builds the autograd Function on first use, so importing the package
+    does not import torch."""
+    _fn = None
+
+    def apply(self, *args):
+        if _LazyFn._fn is None:
+            _LazyFn._fn = _make_autograd_fn()
+        return _LazyFn._fn.apply(*args)
+
+
+_FlintAttnFn = _LazyFn()
 
 
 def device_status(workspace, stream=None) -> int:
