@@ -204,3 +204,32 @@ def test_infinite_sinks():
     g = OB.attn_bwd_workload(w, _dout(6, 108))
     assert np.all(g["dsinks"] == 0.0)
     assert np.all(np.isfinite(g["dq"])) and np.any(g["dq"] != 0.0)
+
+
+def test_gradient_matches_finite_differences_on_random_layouts():
+    """Random lengths, windows, RoPE, document splits and trailing padding:
+    central differences of the C forward oracle at random entries."""
+    from hypothesis import given, settings, strategies as st
+
+    @settings(max_examples=12, deadline=None, derandomize=True)
+    @given(T=st.integers(2, 18), window=st.integers(0, 20), rope=st.booleans(),
+           cuts=st.lists(st.integers(1, 17), max_size=3), pad=st.integers(0, 3),
+           seed=st.integers(0, 10 ** 6))
+    def check(T, window, rope, cuts, pad, seed):
+        valid = max(1, T - pad)
+        cu = [0] + sorted({c for c in cuts if c < valid}) + [valid]
+        w = W.make_small(T, seed=seed, window=window, use_rope=rope, cu_seqlens=cu)
+        dO = _dout(T, seed + 1)
+        g = OB.attn_bwd_workload(w, dO)
+        rng = np.random.default_rng(seed + 2)
+        entries = [("q", "dq", (int(rng.integers(T)), int(rng.integers(32)), int(rng.integers(128)))),
+                   ("k", "dk", (int(rng.integers(T)), int(rng.integers(4)), int(rng.integers(128)))),
+                   ("v", "dv", (int(rng.integers(T)), int(rng.integers(4)), int(rng.integers(128)))),
+                   ("wq", "dq_norm_w", (int(rng.integers(128)),)),
+                   ("sinks", "dsinks", (int(rng.integers(32)),))]
+        for name, key, idx in entries:
+            fd = _fd(w, dO, name, idx)
+            an = g[key][idx]
+            assert abs(fd - an) <= 1e-6 * (1.0 + abs(an)), (T, window, rope, cu, name, idx, fd, an)
+
+    check()
