@@ -232,3 +232,23 @@ def test_bwd_invalid_arguments_rejected_on_host(lib, kw, status):
 def test_bwd_empty_input_checks_the_small_gradients_first(lib):
     # T == 0 zeroes dq_norm_w, dk_norm_w and dsinks, so those must be given
     assert call_bwd(lib, T=0, dwk=None) == 1
+
+
+def test_header_is_plain_c_and_links_against_the_library(lib, tmp_path):
+    """A C11 program that includes the header and references every entry
+    point compiles with -Wall -Werror and links against libflint_attn.so
+    (nothing is run)."""
+    import subprocess
+    names = declared_functions()
+    src = tmp_path / "use_abi.c"
+    body = "\n".join("    p = (void (*)(void))&%s; (void)p;" % n for n in names)
+    src.write_text('#include "flint_attn.h"\n#include <stdio.h>\n'
+                   "int main(void) {\n    void (*p)(void);\n%s\n"
+                   '    printf("%%d\\n", (int)FLINT_OK);\n    return 0;\n}\n' % body)
+    exe = tmp_path / "use_abi"
+    r = subprocess.run(["gcc", "-std=c11", "-Wall", "-Wextra", "-Werror", "-Wno-pedantic",
+                        "-I", os.path.dirname(HEADER), str(src), "-o", str(exe),
+                        "-L", os.path.dirname(fa.LIB_PATH), "-lflint_attn",
+                        "-Wl,-rpath," + os.path.dirname(fa.LIB_PATH)],
+                       capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
