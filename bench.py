@@ -353,6 +353,82 @@ def run_flint(args, rank, world, local_rank):
                 gpu=torch.cuda.get_device_name(dev))
 
 
+def time_config(name, dev, steps=20, warmup=5):
+    """Layer, attention-kernel and preparation-kernel times (ms, CUDA events,
+    L2 flushed before every step) of one named workload: the per-config
+    record of the default run.  Inputs are the workload's seeded tensors,
+    already resident in HBM."""
+    import torch
+    import full_gqa_learned_b200 as fa
+    w = W.make(name)
+
+    def bf(x):
+        return torch.from_numpy(np.ascontiguousarray(x)).view(torch.bfloat16).to(dev)
+    d = dict(q=bf(w.q), k=bf(w.k), v=bf(w.v), q_norm_w=torch.from_numpy(w.q_norm_w).to(dev),
+             k_norm_w=torch.from_numpy(w.k_norm_w).to(dev),
+             sinks=torch.from_numpy(np.ascontiguousarray(w.sinks, np.float32)).to(dev))
+    opt = {n: torch.from_numpy(getattr(w, n)).to(dev) for n in ("pos_ids", "cu_seqlens", "pad_mask")
+           if getattr(w, n) is not None}
+    nseg = (len(w.cu_seqlens) - 1) if w.cu_seqlens is not None else (
+        w.pad_mask.shape[0] if w.pad_mask is not None else 1)
+    out = torch.empty((w.T, 4096), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((32, w.T), dtype=torch.float32, device=dev)
+    ws = torch.empty(fa.workspace_bytes(w.T, nseg), dtype=torch.uint8, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    kw = dict(window=w.window, use_rope=w.use_rope, rope_theta=w.rope_theta, eps=w.eps, out=out,
+              lse=lse, workspace=ws, stream=stream, **opt)
+
+    def call(stage="both"):
+        fa.attn_fwd(d["q"], d["k"], d["v"], d["q_norm_w"], d["k_norm_w"], d["sinks"], stage=stage, **kw)
+    for _ in range(warmup):
+        flush.fill_(1)
+        call()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(steps)]
+    torch.cuda.synchronize(dev)
+    for i in range(steps):
+        flush.fill_(i & 0xFF)
+        ev[i][0].record(stream)
+        call()
+        ev[i][1].record(stream)
+        flush.fill_((i + 7) & 0xFF)
+        ev[i][2].record(stream)
+        call("prepare")
+        ev[i][3].record(stream)
+        call("attend")
+        ev[i][4].record(stream)
+    torch.cuda.synchronize(dev)
+    st = fa.device_status(ws)
+    if st != 0:
+        raise RuntimeError("device status %s on %s" % (fa.STATUS.get(st, st), name))
+    layer = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
+    prep = statistics.mean(e[2].elapsed_time(e[3]) for e in ev)
+    attn = statistics.mean(e[3].elapsed_time(e[4]) for e in ev)
+    del d, opt, out, lse, ws, flush
+    torch.cuda.empty_cache()
+    return w, layer, attn, prep
+
+
+def configs_record(dev, peak, main=None):
+    """Per-config record of every named workload (the driver's default run
+    carries it): layer and kernel times, TFLOP/s and fractions of the peak."""
+    rec = {}
+    for name in W.CONFIGS:
+        if main is not None and name == main["name"]:
+            w_flops, layer, attn, prep = main["flops"], main["layer"], main["attn"], main["prep"]
+        else:
+            w, layer, attn, prep = time_config(name, dev)
+            w_flops = w.flops()
+        rec[name] = dict(layer_ms=round(layer, 5), attn_kernel_ms=round(attn, 5),
+                         prep_kernel_ms=round(prep, 5),
+                         layer_tflops=round(w_flops / (layer * 1e-3) / 1e12, 2),
+                         attn_tflops=round(w_flops / (attn * 1e-3) / 1e12, 2),
+                         layer_frac=round(w_flops / (layer * 1e-3) / 1e12 / peak, 4),
+                         attn_frac=round(w_flops / (attn * 1e-3) / 1e12 / peak, 4),
+                         flops=w_flops)
+    return rec
+
+
 def cpu_baseline(w, budget_s, nthreads=0):
     """The oracle, as it stands, on a bounded sample of query rows."""
     import oracle
@@ -634,11 +710,13 @@ def main():
     ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD,
-                    choices=sorted(W.CONFIGS) + sorted(W.DECODE_CONFIGS)
+                    choices=sorted(W.CONFIGS) + sorted(W.PROFILE_CONFIGS) + sorted(W.DECODE_CONFIGS)
                     + sorted(BWD_PREFIX + n for n in W.CONFIGS))
     ap.add_argument("--impl", default="flint", choices=["flint", "reference"])
     ap.add_argument("--soak", type=float, default=1.0, help="seconds of untimed load before timing")
     ap.add_argument("--cpu-budget", type=float, default=12.0)
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the per-config record of the other named workloads")
     ap.add_argument("--profile", action="store_true",
                     help="warm-up and timed steps only (for ncu captures): no soak, e2e or CPU leg")
     ap.add_argument("--traffic", type=float, default=None,
@@ -756,7 +834,8 @@ def main():
                     pv_operands="bf16", l2="flushed before every timed step (256 MiB write)",
                     per_rank="independent replica", seed=w.seed, gpu=r["gpu"]),
         roofline=dict(bound="tensor", achieved=round(attn_tflops, 3), peak=peak, unit=UNIT,
-                      frac=round(attn_tflops / peak, 4),
+                      frac=round(attn_tflops / peak, 4), kernel_frac=round(attn_tflops / peak, 4),
+                      layer_frac=round(value / world / peak, 4),
                       traffic=args.traffic if args.traffic is not None else recorded_traffic(w.name),
                       kernel="flint::attn_fwd_kernel", peak_source="%s bf16_tflops (burst)" % src,
                       flops_per_launch=flops,
@@ -769,6 +848,10 @@ def main():
     )
     if rank == 0 and world == 1 and not args.profile:
         line["cpu_baseline"] = cpu_baseline(w, budget_s=args.cpu_budget)
+    if world == 1 and not args.profile and not args.no_configs:
+        main = dict(name=w.name, flops=flops, layer=r["total_ms"] / args.steps, attn=r["attn_avg"],
+                    prep=r["prep_avg"])
+        line["configs"] = configs_record(torch.device("cuda", local_rank), peak, main)
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()

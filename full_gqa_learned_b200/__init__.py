@@ -17,7 +17,7 @@ import os
 import threading
 from typing import Optional, Tuple
 
-__all__ = ["attn_fwd", "attn_fwd_static", "attn_decode", "attn_bwd", "flint_attention", "workspace_bytes",
+__all__ = ["attn_fwd", "attn_fwd_static", "static_status", "attn_decode", "attn_bwd", "flint_attention", "workspace_bytes",
            "decode_workspace_bytes", "bwd_workspace_bytes", "device_status", "load_library",
            "FlintError", "LIB_PATH", "HQ", "HKV", "HEAD_DIM", "STATUS", "STATIC_SCRATCH_BYTES"]
 
@@ -60,6 +60,8 @@ def load_library() -> ctypes.CDLL:
             getattr(lib, name).argtypes = fwd_args
         lib.flint_attn_fwd_static.restype = ctypes.c_int
         lib.flint_attn_fwd_static.argtypes = fwd_args[:19] + [P]
+        lib.flint_attn_fwd_static_status.restype = ctypes.c_int
+        lib.flint_attn_fwd_static_status.argtypes = [P]
         lib.flint_attn_decode_workspace_bytes.restype = ctypes.c_size_t
         lib.flint_attn_decode_workspace_bytes.argtypes = [I32, I32, I32]
         lib.flint_attn_decode.restype = ctypes.c_int
@@ -396,3 +398,17 @@ def attn_fwd_static(q, k, v, q_norm_w, k_norm_w, sinks, out, lse, *, pos_ids=Non
             _ptr(lse), sptr)
     if st != 0:
         raise FlintError(st, lib.flint_attn_last_error().decode())
+
+
+def static_status(device=None, stream=None) -> int:
+    """flint_attn_fwd_static_status: synchronise ``stream`` and return the
+    device-side status of the last attn_fwd_static call that launched kernels
+    (0 = FLINT_OK).  Reads one word; allocates nothing."""
+    import torch
+    lib = load_library()
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    if stream is None:
+        stream = torch.cuda.current_stream(dev)
+    sptr = stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+    with torch.cuda.device(dev):
+        return int(lib.flint_attn_fwd_static_status(sptr))

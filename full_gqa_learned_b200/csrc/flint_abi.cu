@@ -12,6 +12,7 @@
 
 #include <nvtx3/nvToolsExt.h>   // header-only NVTX v3: named ranges for profilers
 #include <cstring>
+#include <atomic>
 #include <mutex>
 
 #include "../../include/flint_attn.h"
@@ -107,6 +108,24 @@ flint_status_t make_map(EncodeTiledFn enc, CUtensorMap* m, CUtensorMapDataType d
 }
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// Test hook, not part of the ABI.  FLINT_TEST_WAIT_TIMEOUT_MS=n (1..10000),
+// read once when the process first launches the attention kernel, makes that
+// one launch's MMA warps wait n ms on a barrier nothing arrives on, so the
+// bounded-wait timeout path runs; later launches are unaffected.
+std::once_flag g_stall_once;
+std::atomic<unsigned long long> g_stall_ns{0};
+
+unsigned long long test_stall_once() {
+    std::call_once(g_stall_once, [] {
+        if (const char* tw = std::getenv("FLINT_TEST_WAIT_TIMEOUT_MS")) {
+            const long ms = std::strtol(tw, nullptr, 10);
+            if (ms > 0 && ms <= 10000) g_stall_ns.store((unsigned long long)ms * 1000000ull);
+        }
+    });
+    if (g_stall_ns.load(std::memory_order_relaxed) == 0) return 0;
+    return g_stall_ns.exchange(0);
+}
 
 }  // namespace
 
@@ -257,13 +276,7 @@ flint_status_t run_stages(int stages, const void* q, const void* k, const void* 
     ap.use_rope = use_rope;
     ap.rope_theta = rope_theta;
     ap.eps = eps;
-    // test hook (not part of the ABI): FLINT_TEST_WAIT_TIMEOUT_MS=n makes the
-    // attention kernel's bounded waits run out after n ms
-    ap.test_wait_ns = 0;
-    if (const char* tw = std::getenv("FLINT_TEST_WAIT_TIMEOUT_MS")) {
-        const long ms = std::strtol(tw, nullptr, 10);
-        if (ms > 0 && ms <= 10000) ap.test_wait_ns = (unsigned long long)ms * 1000000ull;
-    }
+    ap.test_wait_ns = test_stall_once();
     const int max_units = L.max_items * kHKV;
     const int grid = max_units < sms ? max_units : sms;
     if (stages & kStagePrepare) {

@@ -6,12 +6,10 @@
 // elsewhere (a fixed memory budget carved out up front, an allocator that must
 // not be re-entered from a callback, a plug-in host that only hands out its
 // own buffers).  This entry point serves them: the scratch the kernels need
-// (the work plan and the normalised FP16 keys) lives in a file-scope device
-// array of fixed size, so the call itself allocates nothing.  Inputs and
-// outputs are still passed by the caller.
+// (the work plan, the status word and the normalised FP16 keys) lives in a
+// file-scope device array of fixed size, so the call itself allocates
+// nothing.  Inputs and outputs are still passed by the caller.
 #include <cuda_runtime.h>
-
-#include <mutex>
 
 #include "../../include/flint_attn.h"
 #include "flint_common.cuh"
@@ -32,27 +30,17 @@ constexpr size_t kStaticScratchBytes = FLINT_STATIC_SCRATCH_BYTES;
 
 // Every GPU that loads the library holds this array until the process exits.
 // In host code its name is only a host-side stand-in: the device address comes
-// from cudaGetSymbolAddress, taken once per device below.
+// from cudaGetSymbolAddress, looked up with the device current on every call
+// (cheap, allocates nothing), so no address outlives a device reset or
+// belongs to another context.
 __device__ __align__(256) char g_scratch[kStaticScratchBytes];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_mu;
-void* g_scratch_addr[kMaxDevices] = {nullptr};
-
 flint_status_t scratch_address(void** addr) {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess)
-        return set_error(FLINT_ERR_CUDA, "cudaGetDevice failed");
-    if (dev < 0 || dev >= kMaxDevices) return set_error(FLINT_ERR_UNSUPPORTED, "device index out of range");
-    std::lock_guard<std::mutex> lk(g_mu);
-    if (!g_scratch_addr[dev]) {
-        void* p = nullptr;
-        const cudaError_t e = cudaGetSymbolAddress(&p, g_scratch);
-        if (e != cudaSuccess || !p)
-            return set_error(FLINT_ERR_CUDA, "cudaGetSymbolAddress of the static scratch failed");
-        g_scratch_addr[dev] = p;
-    }
-    *addr = g_scratch_addr[dev];
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_scratch);
+    if (e != cudaSuccess || !p)
+        return set_error(FLINT_ERR_CUDA, "cudaGetSymbolAddress of the static scratch failed");
+    *addr = p;
     return FLINT_OK;
 }
 
@@ -86,6 +74,19 @@ flint_status_t flint_attn_fwd_static(const void* q, const void* k, const void* v
                              cu_seqlens, num_docs, pad_mask, batch, seqlen, T, window, use_rope,
                              rope_theta, eps, out, lse, scratch, flint::kStaticScratchBytes,
                              stream);
+}
+
+flint_status_t flint_attn_fwd_static_status(void* stream) {
+    cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess)
+        return flint::set_error(FLINT_ERR_CUDA, "stream synchronisation failed");
+    // the status word is the first word of the work-plan header, which sits
+    // at the start of the scratch
+    int st = 0;
+    e = cudaMemcpyFromSymbol(&st, flint::g_scratch, sizeof(int), 0, cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess)
+        return flint::set_error(FLINT_ERR_CUDA, "reading the static scratch's status failed");
+    return static_cast<flint_status_t>(st);
 }
 
 }  // extern "C"

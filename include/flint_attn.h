@@ -196,13 +196,17 @@ FLINT_API flint_status_t flint_attn_device_status(const void* workspace, void* s
  *  - A problem whose scratch would exceed FLINT_STATIC_SCRATCH_BYTES
  *    (flint_attn_workspace_bytes(T, n) larger than it) is rejected with
  *    FLINT_ERR_WORKSPACE before any launch.
- *  - The first call on a device looks up the array's device address
- *    (cudaGetSymbolAddress) with that device current; make that first call
+ *  - Every call looks up the array's device address (cudaGetSymbolAddress)
+ *    with the calling thread's current device, so the address always belongs
+ *    to the current context, also after a device reset.  The first call on a
+ *    device may load the library's device code there; make that first call
  *    before any stream capture.
  *  - Every call shares the one array and it keeps the last call's contents
  *    (the kernels initialise what they read); calls that may overlap on the
  *    GPU race on it, so serialise them (one stream, or events).
- *  - Device-side status is not readable for this entry point.
+ *  - Errors only the device can see (ill-formed cu_seqlens, non-trailing
+ *    mask, a timed-out wait) are recorded in the array's status word; read
+ *    it with flint_attn_fwd_static_status.
  */
 FLINT_API flint_status_t flint_attn_fwd_static(const void* q, const void* k, const void* v,
                               const float* q_norm_w, const float* k_norm_w,
@@ -213,6 +217,18 @@ FLINT_API flint_status_t flint_attn_fwd_static(const void* q, const void* k, con
                               float rope_theta, float eps,
                               void* out, float* lse,
                               void* stream);
+
+/*
+ * Synchronises `stream`, then returns the status recorded by the kernels of
+ * the last flint_attn_fwd_static call that launched any (FLINT_OK,
+ * FLINT_ERR_INVALID_ARG for an ill-formed cu_seqlens, FLINT_ERR_UNSUPPORTED
+ * for a non-trailing mask, FLINT_ERR_TIMEOUT), or FLINT_ERR_CUDA if
+ * synchronising or reading failed.  Calls rejected on the host and T == 0
+ * launch nothing and leave the word as it was.  Copies one word from the
+ * device to the host; allocates nothing.  Like the array itself, it is
+ * shared: read it before the next flint_attn_fwd_static call is enqueued.
+ */
+FLINT_API flint_status_t flint_attn_fwd_static_status(void* stream);
 
 /* Largest batch of one decode step (sequences per call). */
 #define FLINT_MAX_DECODE_BATCH 65535

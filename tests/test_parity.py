@@ -7,15 +7,18 @@ output relative L2 error 5e-3, LSE abs error 1e-3; padded query rows exactly
 
 Those bounds apply to the five named workloads.  Two derived readings:
 
-* Massive-activation workload: |out| reaches ~1.6e3 (value channels ~1e3),
-  where one BF16 ulp of the output alone is 8, so no BF16 output meets an
-  absolute 2e-2.  Its per-element error is measured against the absolute-value
-  sum A_ic = sum_j p_ij |v_jc| / Z_i (the oracle run on |v|): the BF16 rounding
-  of P contributes at most 2^-9 A, a logit error ds at most |ds| A and the
-  output rounding 2^-9 |ref| <= 2^-9 A, so |err| <= 2e-2 * max(1, A) while
-  |ds| <= 1.6e-2.  Its LSE bound is that logit-error bound: the FP16 rounding
-  of both normalised operands gives |ds| <= 2^-10 sum_c |q~_c k~_c| / sqrt(128),
-  about 2e-2 for the outlier rows.
+* Massive-activation workload (HF discussion #26 on RecursiveSI/flint,
+  massive activations): it does NOT meet the stated bounds, and the test
+  prints its raw errors against them.  |out| reaches ~1.6e3 (value channels
+  ~1e3), where one BF16 ulp of the output alone is 8, so no BF16 output meets
+  an absolute 2e-2.  Its per-element error is measured against the
+  absolute-value sum A_ic = sum_j p_ij |v_jc| / Z_i (the oracle run on |v|):
+  the BF16 rounding of P contributes at most 2^-9 A, a logit error ds at most
+  |ds| A and the output rounding 2^-9 |ref| <= 2^-9 A, so |err| <= 2e-2 *
+  max(1, A) while |ds| <= 1.6e-2.  Its LSE error has a floor set by the FP16
+  rounding of the normalised outlier channels: the oracle with Q/K rounded to
+  FP16 is 5.1e-3 from the exact result (BF16: 4.5e-2).  The LSE bound is 1.5x
+  that measured floor, 7.5e-3.
 * Synthetic edge cases (window 1, a single token, extreme sinks...): rows
   that see one key carry the raw rounding error of a single FP16 dot product.
   For unit-RMS normalised rows its standard deviation is
@@ -67,10 +70,10 @@ def run_gpu(w, **over):
     return out, lse.cpu().numpy()
 
 
-def compare(w, out_bits, lse_gpu, rows=None, tol=TOL, abs_sum_scaled=False):
+def compare(w, out_bits, lse_gpu, rows=None, tol=TOL, abs_sum_scaled=False, ref=None):
     if rows is None:
         rows = w.rows if w.rows is not None else np.arange(w.T)
-    ref_o, ref_l = oracle.attn_fwd_workload(w, rows=rows)
+    ref_o, ref_l = oracle.attn_fwd_workload(w, rows=rows) if ref is None else ref
     got = W.bf16_to_f64(out_bits[rows])
     got_l = lse_gpu[:, rows].T.astype(np.float64)
     err = np.abs(got - ref_o)
@@ -113,34 +116,51 @@ def test_sliding_s1024_all_rows():
     compare(w, o, l, rows=np.arange(w.T))
 
 
-def test_full_s4096_sampled():
+def test_full_s4096_all_rows():
     w = W.make("full_s4096")
-    rng = np.random.default_rng(100)
-    rows = np.unique(np.concatenate([np.arange(40), [127, 128, 129, 4095, 4094, 2047, 2048],
-                                     rng.choice(w.T, 900, replace=False)]))
     o, l = run_gpu(w)
-    compare(w, o, l, rows=rows)
+    compare(w, o, l, rows=np.arange(w.T))
 
 
-def test_thd_8docs_32768_sampled():
+def test_thd_8docs_32768_all_rows():
     w = W.make("thd_8docs_32768")
     o, l = run_gpu(w)
-    compare(w, o, l)
+    assert check_padding(w, o, l) == 0
+    compare(w, o, l, rows=np.arange(w.T))
 
 
 def test_sliding_s262144_sampled():
+    """The one named workload checked on sampled rows (4096, seeded, forced
+    to include 0, 1, 511, 512, 513 and T-1): the full oracle would take hours."""
     w = W.make("sliding_s262144")
     o, l = run_gpu(w)
     compare(w, o, l)
 
 
-def test_stress_full_4x8192_pad_sampled():
+TOL_STRESS = dict(max_abs=2e-2, rel_l2=5e-3, lse=7.5e-3)   # derived (module docstring)
+
+
+def test_stress_full_4x8192_pad_all_rows(record_property):
     w = W.make("stress_full_4x8192_pad")
     o, l = run_gpu(w)
     assert check_padding(w, o, l) > 0
-    # error scaled by the absolute-value sum; LSE bound from the FP16-operand
-    # logit error (module docstring)
-    compare(w, o, l, tol=dict(max_abs=2e-2, rel_l2=5e-3, lse=2e-2), abs_sum_scaled=True)
+    rows = np.arange(w.T)
+    # raw errors against the stated bounds, printed and recorded: this
+    # workload misses them (module docstring)
+    ref_o, ref_l = oracle.attn_fwd_workload(w, rows=rows)
+    got = W.bf16_to_f64(o[rows])
+    got_l = l[:, rows].T.astype(np.float64)
+    fin = np.isfinite(ref_l)
+    raw_abs = float(np.abs(got - ref_o).max())
+    raw_lse = float(np.abs(got_l[fin] - ref_l[fin]).max())
+    print("stress_full_4x8192_pad raw: max_abs %.3e (stated 2e-2), lse %.3e (stated 1e-3)"
+          % (raw_abs, raw_lse))
+    record_property("stress_raw_max_abs", raw_abs)
+    record_property("stress_raw_lse", raw_lse)
+    max_abs, rel, lse = compare(w, o, l, rows=rows, tol=TOL_STRESS, abs_sum_scaled=True,
+                                ref=(ref_o, ref_l))
+    record_property("stress_scaled_max_abs", max_abs)
+    record_property("stress_rel_l2", rel)
 
 
 # ------------------------------------------------------------------ small cases, all rows
@@ -289,18 +309,37 @@ def test_later_chunk_raises_the_max(mix):
     compare(w, o, l, rows=rows, tol=TOL_EDGE)
 
 
-def test_bounded_wait_timeout_reports_status(monkeypatch):
-    """Failure detection without a fault: a test hook makes every CTA's MMA
-    warp wait 20 ms on a barrier nothing arrives on.  The bounded wait runs
-    out, the status reads FLINT_ERR_TIMEOUT, every warp unwinds (drains its
-    copies, frees TMEM) and the next call on the same context is correct."""
-    import full_gqa_learned_b200 as fa
-    w = W.make_small(300, seed=19, window=0, use_rope=False)
-    t = to_device(w)
-    monkeypatch.setenv("FLINT_TEST_WAIT_TIMEOUT_MS", "20")
-    fa.attn_fwd(t["q"], t["k"], t["v"], t["q_norm_w"], t["k_norm_w"], t["sinks"], window=0,
-                use_rope=False)
-    assert fa.device_status(fa.attn_fwd.last_workspace) == 4      # FLINT_ERR_TIMEOUT
-    monkeypatch.delenv("FLINT_TEST_WAIT_TIMEOUT_MS")
-    o, l = run_gpu(w)
-    compare(w, o, l, tol=TOL_EDGE)
+_TIMEOUT_CHILD = r"""
+import sys
+sys.path.insert(0, %r)
+import numpy as np
+import full_gqa_learned_b200 as fa
+import workloads as W
+from tests.test_parity import to_device, run_gpu, compare, TOL_EDGE
+w = W.make_small(300, seed=19, window=0, use_rope=False)
+t = to_device(w)
+fa.attn_fwd(t["q"], t["k"], t["v"], t["q_norm_w"], t["k_norm_w"], t["sinks"], window=0,
+            use_rope=False)
+st = fa.device_status(fa.attn_fwd.last_workspace)
+assert st == 4, st                                   # FLINT_ERR_TIMEOUT
+o, l = run_gpu(w)                                    # the hook is one-shot
+compare(w, o, l, tol=TOL_EDGE)
+print("TIMEOUT_CHILD_OK")
+"""
+
+
+def test_bounded_wait_timeout_reports_status():
+    """Failure detection without a fault: a test hook, read once per process
+    from FLINT_TEST_WAIT_TIMEOUT_MS, makes the first launch's MMA warps wait
+    20 ms on a barrier nothing arrives on.  The bounded wait runs out, the
+    status reads FLINT_ERR_TIMEOUT, every warp unwinds (drains its copies,
+    frees TMEM) and the next call on the same context is correct.  Runs in a
+    fresh process so that the hook is read there."""
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = dict(os.environ, FLINT_TEST_WAIT_TIMEOUT_MS="20")
+    r = subprocess.run([sys.executable, "-c", _TIMEOUT_CHILD % root], env=env, cwd=root,
+                       capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0 and "TIMEOUT_CHILD_OK" in r.stdout, r.stdout + r.stderr

@@ -259,7 +259,17 @@ CONFIGS = {
 }
 
 
+# Smaller stand-ins with the structure of a named workload, sized for
+# profiler captures (a few hundred MB on the device): the long-context
+# sliding layer's per-tile chunk structure at 32,768 tokens.
+PROFILE_CONFIGS = {
+    "sliding_s32768": lambda: make_long(T=32768, seed=3, name="sliding_s32768"),
+}
+
+
 def make(name: str, **kw) -> Workload:
+    if name in PROFILE_CONFIGS:
+        return PROFILE_CONFIGS[name](**kw)
     return CONFIGS[name](**kw)
 
 
