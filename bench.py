@@ -53,12 +53,13 @@ KERNEL_SOURCES = [os.path.join(os.path.dirname(os.path.abspath(__file__)), "full
                                "csrc", f) for f in ("flint_attn.cu", "flint_common.cuh", "sm100.cuh")]
 
 
-def recorded_traffic(workload):
+def recorded_traffic(workload, profiles_dir=None):
     """DRAM bytes (read + write) per attention-kernel launch from the committed
     ncu summary of `workload`, or None when there is none or the kernel's
     sources changed since it was taken."""
-    path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "profiles",
-                        "attn_fwd_kernel_%s_ncu.md" % workload)
+    if profiles_dir is None:
+        profiles_dir = os.path.join(os.path.dirname(os.path.abspath(__file__)), "profiles")
+    path = os.path.join(profiles_dir, "attn_fwd_kernel_%s_ncu.md" % workload)
     if not os.path.exists(path):
         return None
     vals = {}
@@ -704,6 +705,163 @@ def bwd_line(args, world, r):
         gpu_launches=5 * args.steps, clocks=r["clocks"])
 
 
+# ---------------------------------------------------------------- whole-layer leg
+
+LAYER_METRIC = ("attention layer TFLOP/s (q/k/v projection GEMM + sink attention + o_proj GEMM, "
+                "BF16, window-aware attention FLOPs)")
+
+
+def run_layer(args, rank, world, local_rank):
+    """One flint_attn_layer_fwd call per timed step (hidden states to the
+    layer's output), L2 flushed before each; then the two projection GEMMs
+    apart for their own roofline."""
+    import torch
+    import full_gqa_learned_b200 as fa
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    lw = W.make_layer_named(args.workload)
+    w = lw.attn
+
+    def bf(x):
+        return torch.from_numpy(np.ascontiguousarray(x)).view(torch.bfloat16)
+    host = dict(x=bf(lw.x), w_qkv=bf(lw.w_qkv), w_o=bf(lw.w_o), q_norm_w=torch.from_numpy(w.q_norm_w),
+                k_norm_w=torch.from_numpy(w.k_norm_w),
+                sinks=torch.from_numpy(np.ascontiguousarray(w.sinks, np.float32)))
+    for n in ("pos_ids", "cu_seqlens", "pad_mask"):
+        if getattr(w, n) is not None:
+            host[n] = torch.from_numpy(getattr(w, n))
+    d = {k: v.to(dev) for k, v in host.items()}
+    kw = dict(pos_ids=d.get("pos_ids"), cu_seqlens=d.get("cu_seqlens"), pad_mask=d.get("pad_mask"),
+              window=w.window, use_rope=w.use_rope, rope_theta=w.rope_theta, eps=w.eps)
+    out = fa.attn_layer_fwd(d["x"], d["w_qkv"], d["w_o"], d["q_norm_w"], d["k_norm_w"], d["sinks"], **kw)
+    ws = fa.attn_layer_fwd.last_workspace
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        fa.attn_layer_fwd(d["x"], d["w_qkv"], d["w_o"], d["q_norm_w"], d["k_norm_w"], d["sinks"],
+                          out=out, workspace=ws, stream=stream, **kw)
+    for _ in range(args.warmup):
+        flush.fill_(1)
+        step()
+    st = fa.device_status(ws)
+    if st != 0:
+        raise RuntimeError("device status %s" % fa.STATUS.get(st, st))
+    sampler = ClockSampler(local_rank if "CUDA_VISIBLE_DEVICES" not in os.environ else
+                           os.environ["CUDA_VISIBLE_DEVICES"].split(",")[local_rank])
+    sampler.start()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    for i in range(args.steps):
+        flush.fill_(i & 0xFF)
+        evs[i][0].record(stream)
+        step()
+        evs[i][1].record(stream)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+    total_ms = sum(e[0].elapsed_time(e[1]) for e in evs)
+    st = fa.device_status(ws)
+    if st != 0:
+        raise RuntimeError("device status %s" % fa.STATUS.get(st, st))
+    # the projection GEMMs apart (same inputs, L2 flushed before each)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    for i in range(args.steps):
+        flush.fill_(i & 0xFF)
+        ev[i][0].record(stream)
+        fa.qkv_proj(d["x"], d["w_qkv"], q=out["q"], k=out["k"], v=out["v"], stream=stream)
+        ev[i][1].record(stream)
+        flush.fill_((i + 3) & 0xFF)
+        ev[i][2].record(stream)
+        fa.o_proj(out["attn_out"], d["w_o"], y=out["y"], stream=stream)
+        ev[i][3].record(stream)
+    torch.cuda.synchronize(dev)
+    qkv_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
+    o_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in ev)
+
+    e2e_ms, h2d, d2h = float("nan"), 0, 0
+    if not args.profile:
+        pinned = {k: v.pin_memory() for k, v in host.items()}
+        y_h = torch.empty(tuple(out["y"].shape), dtype=torch.bfloat16).pin_memory()
+        h2d = sum(v.numel() * v.element_size() for v in pinned.values())
+        d2h = y_h.numel() * 2
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        n_e2e = max(3, min(args.steps, 10))
+        e2e_ms = 0.0
+        for _ in range(n_e2e):
+            flush.fill_(3)
+            e0.record(stream)
+            dd = {k: v.to(dev, non_blocking=True) for k, v in pinned.items()}
+            fa.attn_layer_fwd(dd["x"], dd["w_qkv"], dd["w_o"], dd["q_norm_w"], dd["k_norm_w"], dd["sinks"],
+                              pos_ids=dd.get("pos_ids"), cu_seqlens=dd.get("cu_seqlens"),
+                              pad_mask=dd.get("pad_mask"), window=w.window, use_rope=w.use_rope,
+                              rope_theta=w.rope_theta, eps=w.eps, out=out, workspace=ws, stream=stream)
+            y_h.copy_(out["y"], non_blocking=True)
+            e1.record(stream)
+            torch.cuda.synchronize(dev)
+            e2e_ms += e0.elapsed_time(e1)
+        e2e_ms /= n_e2e
+    total_ms, e2e_ms = max_over_ranks([total_ms, e2e_ms], device=dev)
+    return dict(lw=lw, total_ms=total_ms, qkv_ms=qkv_ms, o_ms=o_ms, e2e_ms=e2e_ms, h2d=h2d, d2h=d2h,
+                clocks=clocks, gpu=torch.cuda.get_device_name(dev))
+
+
+def layer_cpu_baseline(lw, budget_s):
+    """The layer oracle (FP64 projections, attention oracle, o_proj), as it
+    stands, on a prefix of the workload's tokens (a prefix of a causal single
+    sequence is a self-contained problem), grown until a run takes about
+    budget_s seconds: algorithmic FLOPs per second."""
+    from oracle import projection as OP
+    n, dt = 16, 0.0
+    while True:
+        sub = W.make_layer(n, seed=0, hidden=lw.hidden, window=lw.attn.window, use_rope=lw.attn.use_rope)
+        a = lw.attn
+        t0 = time.time()
+        OP.attn_layer(lw.x[:n], lw.w_qkv[:4096], lw.w_qkv[4096:4608], lw.w_qkv[4608:], lw.w_o, a.q_norm_w,
+                      a.k_norm_w, a.sinks, window=a.window, use_rope=a.use_rope, rope_theta=a.rope_theta,
+                      eps=a.eps)
+        dt = time.time() - t0
+        if dt > budget_s / 4 or 2 * n > lw.T:
+            break
+        n *= 2
+    return dict(value=sub.flops() / dt / 1e12, unit=UNIT, cores=os.cpu_count(), kind="oracle",
+                sample="first %d tokens of %s (one sequence), %.2f s" % (n, lw.name, dt))
+
+
+def layer_line(args, world, r):
+    lw = r["lw"]
+    peaks, src = load_peaks()
+    peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    flops = lw.flops()
+    step_ms = r["total_ms"] / args.steps
+    tf = flops / (step_ms * 1e-3) / 1e12
+    qkv_flops = 2.0 * lw.T * lw.hidden * 5120
+    o_flops = 2.0 * lw.T * 4096 * lw.hidden
+    qkv_tf = qkv_flops / (r["qkv_ms"] * 1e-3) / 1e12
+    return dict(
+        metric=LAYER_METRIC, value=round(tf * world, 3), unit=UNIT, n_gpus=world, steps=args.steps,
+        warmup=args.warmup, ms_per_step=round(step_ms, 5), higher_is_better=True, scaling="weak",
+        vs_baseline=None, dtype="bf16",
+        data="synthetic (seeded N(0,1) BF16 hidden states, N(0,1/fan_in) BF16 weights, 1+N(0,0.1) norm "
+             "weights, N(0,1) sinks)",
+        config=dict(workload=lw.name, T=lw.T, hidden=lw.hidden, window=lw.attn.window,
+                    use_rope=bool(lw.attn.use_rope), l2="flushed before every timed step (256 MiB write)",
+                    per_rank="independent replica", gpu=r["gpu"]),
+        roofline=dict(bound="tensor", achieved=round(qkv_tf, 3), peak=peak, unit=UNIT,
+                      frac=round(qkv_tf / peak, 4), traffic=None, kernel="flint::gemm_kernel (q/k/v projection)",
+                      peak_source="%s bf16_tflops (burst)" % src, flops_per_launch=qkv_flops,
+                      kernel_ms=round(r["qkv_ms"], 5), o_proj_ms=round(r["o_ms"], 5),
+                      o_proj_tflops=round(o_flops / (r["o_ms"] * 1e-3) / 1e12, 3),
+                      layer_frac=round(tf / peak, 4)),
+        e2e=dict(value=round(flops / (r["e2e_ms"] * 1e-3) / 1e12 * world, 3), unit=UNIT,
+                 h2d_bytes_per_step=r["h2d"], d2h_bytes_per_step=r["d2h"], ms_per_step=round(r["e2e_ms"], 4)),
+        gpu_launches=4 * args.steps, clocks=r["clocks"])
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -711,6 +869,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD,
                     choices=sorted(W.CONFIGS) + sorted(W.PROFILE_CONFIGS) + sorted(W.DECODE_CONFIGS)
+                    + sorted(W.LAYER_CONFIGS)
                     + sorted(BWD_PREFIX + n for n in W.CONFIGS))
     ap.add_argument("--impl", default="flint", choices=["flint", "reference"])
     ap.add_argument("--soak", type=float, default=1.0, help="seconds of untimed load before timing")
@@ -749,6 +908,25 @@ def main():
                                                                 window=d.window, use_rope=d.use_rope),
                                   cpu_baseline=cb,
                                   e2e=dict(value=value, unit="GB/s", h2d_bytes_per_step=0,
+                                           d2h_bytes_per_step=0))))
+            return 0
+        if args.workload in W.LAYER_CONFIGS:
+            lw = W.make_layer_named(args.workload)
+            vals, cb = [], None
+            for i in range(args.warmup + args.steps):
+                cb = layer_cpu_baseline(lw, budget_s=min(args.cpu_budget, 60.0 / max(1, args.steps + args.warmup)))
+                if i >= args.warmup:
+                    vals.append(cb["value"])
+            value = statistics.median(vals)
+            cb["value"] = value
+            print(json.dumps(dict(impl="reference", metric=LAYER_METRIC, value=value, unit=UNIT,
+                                  n_gpus=args.gpus, steps=args.steps, warmup=args.warmup, ms_per_step=None,
+                                  higher_is_better=True, scaling="weak", vs_baseline=None, dtype="f64",
+                                  data="synthetic", config=dict(workload=lw.name, T=lw.T, hidden=lw.hidden,
+                                                                window=lw.attn.window,
+                                                                use_rope=lw.attn.use_rope),
+                                  cpu_baseline=cb,
+                                  e2e=dict(value=value, unit=UNIT, h2d_bytes_per_step=0,
                                            d2h_bytes_per_step=0))))
             return 0
         if args.workload.startswith(BWD_PREFIX):
@@ -800,6 +978,17 @@ def main():
         line = decode_line(args, world, d, total_ms, clocks)
         if rank == 0 and world == 1 and not args.profile:
             line["cpu_baseline"] = decode_cpu_baseline(d, budget_s=args.cpu_budget)
+        if world > 1:
+            dist.barrier()
+            dist.destroy_process_group()
+        if rank == 0:
+            print(json.dumps(line))
+        return 0
+    if args.workload in W.LAYER_CONFIGS:
+        r = run_layer(args, rank, world, local_rank)
+        line = layer_line(args, world, r)
+        if rank == 0 and world == 1 and not args.profile:
+            line["cpu_baseline"] = layer_cpu_baseline(r["lw"], budget_s=args.cpu_budget)
         if world > 1:
             dist.barrier()
             dist.destroy_process_group()

@@ -17,7 +17,8 @@ import os
 import threading
 from typing import Optional, Tuple
 
-__all__ = ["attn_fwd", "attn_fwd_static", "static_status", "attn_decode", "attn_bwd", "flint_attention", "workspace_bytes",
+__all__ = ["attn_fwd", "attn_fwd_static", "static_status", "qkv_proj", "o_proj", "attn_layer_fwd",
+           "attn_decode", "attn_bwd", "flint_attention", "workspace_bytes",
            "decode_workspace_bytes", "bwd_workspace_bytes", "device_status", "load_library",
            "FlintError", "LIB_PATH", "HQ", "HKV", "HEAD_DIM", "STATUS", "STATIC_SCRATCH_BYTES"]
 
@@ -72,6 +73,13 @@ def load_library() -> ctypes.CDLL:
         lib.flint_attn_bwd.restype = ctypes.c_int
         lib.flint_attn_bwd.argtypes = [P, P, P, P, P, P, P, P, I32, P, I32, I32, I32, I32, I32,
                                        F32, F32, P, P, P, P, P, P, P, P, P, P, ctypes.c_size_t, P]
+        lib.flint_qkv_proj.restype = ctypes.c_int
+        lib.flint_qkv_proj.argtypes = [P, P, I32, I32, P, P, P, P]
+        lib.flint_o_proj.restype = ctypes.c_int
+        lib.flint_o_proj.argtypes = [P, P, I32, I32, P, P]
+        lib.flint_attn_layer_fwd.restype = ctypes.c_int
+        lib.flint_attn_layer_fwd.argtypes = [P, P, P, P, P, P, P, P, I32, P, I32, I32, I32, I32, I32, I32,
+                                             F32, F32, P, P, P, P, P, P, P, ctypes.c_size_t, P]
         lib.flint_attn_device_status.restype = ctypes.c_int
         lib.flint_attn_device_status.argtypes = [P, P]
         lib.flint_attn_last_error.restype = ctypes.c_char_p
@@ -412,3 +420,106 @@ def static_status(device=None, stream=None) -> int:
     sptr = stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
     with torch.cuda.device(dev):
         return int(lib.flint_attn_fwd_static_status(sptr))
+
+
+def _stream_ptr(stream, dev):
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream(dev)
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def qkv_proj(x, w_qkv, *, q=None, k=None, v=None, stream=None):
+    """flint_qkv_proj: x [T, hidden] bf16, w_qkv [5120, hidden] bf16 (W_q, W_k,
+    W_v stacked, Linear layout).  Returns (q [T,32,128], k [T,4,128],
+    v [T,4,128]) bf16."""
+    import torch
+    lib = load_library()
+    T, hidden = int(x.shape[0]), int(x.shape[1])
+    _check(x, "x", torch.bfloat16, (T, hidden))
+    _check(w_qkv, "w_qkv", torch.bfloat16, (HQ * HEAD_DIM + 2 * HKV * HEAD_DIM, hidden))
+    dev = x.device
+    q = torch.empty((T, HQ, HEAD_DIM), dtype=torch.bfloat16, device=dev) if q is None else q
+    k = torch.empty((T, HKV, HEAD_DIM), dtype=torch.bfloat16, device=dev) if k is None else k
+    v = torch.empty((T, HKV, HEAD_DIM), dtype=torch.bfloat16, device=dev) if v is None else v
+    _check(q, "q", torch.bfloat16, (T, HQ, HEAD_DIM))
+    _check(k, "k", torch.bfloat16, (T, HKV, HEAD_DIM))
+    _check(v, "v", torch.bfloat16, (T, HKV, HEAD_DIM))
+    with torch.cuda.device(dev):
+        st = lib.flint_qkv_proj(_ptr(x), _ptr(w_qkv), T, hidden, _ptr(q), _ptr(k), _ptr(v),
+                                _stream_ptr(stream, dev))
+    if st != 0:
+        raise FlintError(st, lib.flint_attn_last_error().decode())
+    return q, k, v
+
+
+def o_proj(attn_out, w_o, *, y=None, stream=None):
+    """flint_o_proj: attn_out [T, 4096] bf16, w_o [hidden, 4096] bf16.
+    Returns y [T, hidden] bf16."""
+    import torch
+    lib = load_library()
+    T, hidden = int(attn_out.shape[0]), int(w_o.shape[0])
+    _check(attn_out, "attn_out", torch.bfloat16, (T, HQ * HEAD_DIM))
+    _check(w_o, "w_o", torch.bfloat16, (hidden, HQ * HEAD_DIM))
+    dev = attn_out.device
+    y = torch.empty((T, hidden), dtype=torch.bfloat16, device=dev) if y is None else y
+    _check(y, "y", torch.bfloat16, (T, hidden))
+    with torch.cuda.device(dev):
+        st = lib.flint_o_proj(_ptr(attn_out), _ptr(w_o), T, hidden, _ptr(y), _stream_ptr(stream, dev))
+    if st != 0:
+        raise FlintError(st, lib.flint_attn_last_error().decode())
+    return y
+
+
+def attn_layer_fwd(x, w_qkv, w_o, q_norm_w, k_norm_w, sinks, *, pos_ids=None, cu_seqlens=None,
+                   pad_mask=None, window: int = 513, use_rope: bool = True, rope_theta: float = 10000.0,
+                   eps: float = 1e-6, out=None, workspace=None, stream=None, want_lse: bool = True) -> dict:
+    """flint_attn_layer_fwd: the whole attention layer, x [T, hidden] -> y
+    [T, hidden] (see include/flint_attn.h).  Returns a dict with y, the
+    projections q, k, v, the attention output attn_out and lse.  ``out``: the
+    same dict to write into."""
+    import torch
+    lib = load_library()
+    T, hidden = int(x.shape[0]), int(x.shape[1])
+    _check(x, "x", torch.bfloat16, (T, hidden))
+    _check(w_qkv, "w_qkv", torch.bfloat16, (HQ * HEAD_DIM + 2 * HKV * HEAD_DIM, hidden))
+    _check(w_o, "w_o", torch.bfloat16, (hidden, HQ * HEAD_DIM))
+    _check(q_norm_w, "q_norm_w", torch.float32, (HEAD_DIM,))
+    _check(k_norm_w, "k_norm_w", torch.float32, (HEAD_DIM,))
+    _check(sinks, "sinks", torch.float32, (HQ,))
+    num_docs, batch, seqlen, nseg = 0, 0, 0, 1
+    if pos_ids is not None:
+        _check(pos_ids, "pos_ids", torch.int32, (T,))
+    if cu_seqlens is not None:
+        _check(cu_seqlens, "cu_seqlens", torch.int32)
+        num_docs = int(cu_seqlens.numel()) - 1
+        nseg = max(num_docs, 1)
+    if pad_mask is not None:
+        _check(pad_mask, "pad_mask", torch.uint8)
+        batch, seqlen = int(pad_mask.shape[0]), int(pad_mask.shape[1])
+        nseg = batch
+    dev = x.device
+    shapes = dict(q=(T, HQ, HEAD_DIM), k=(T, HKV, HEAD_DIM), v=(T, HKV, HEAD_DIM),
+                  attn_out=(T, HQ * HEAD_DIM), y=(T, hidden))
+    if out is None:
+        out = {n: torch.empty(sh, dtype=torch.bfloat16, device=dev) for n, sh in shapes.items()}
+        out["lse"] = torch.empty((HQ, T), dtype=torch.float32, device=dev) if want_lse else None
+    for n, sh in shapes.items():
+        _check(out[n], n, torch.bfloat16, sh)
+    if out.get("lse") is not None:
+        _check(out["lse"], "lse", torch.float32, (HQ, T))
+    need = workspace_bytes(T, nseg)
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
+    _check(workspace, "workspace", torch.uint8)
+    with torch.cuda.device(dev):
+        st = lib.flint_attn_layer_fwd(
+            _ptr(x), _ptr(w_qkv), _ptr(w_o), _ptr(q_norm_w), _ptr(k_norm_w), _ptr(sinks), _ptr(pos_ids),
+            _ptr(cu_seqlens), num_docs, _ptr(pad_mask), batch, seqlen, T, hidden, int(window),
+            int(bool(use_rope)), float(rope_theta), float(eps), _ptr(out["q"]), _ptr(out["k"]),
+            _ptr(out["v"]), _ptr(out["attn_out"]), _ptr(out["y"]), _ptr(out.get("lse")), _ptr(workspace),
+            int(workspace.numel()), _stream_ptr(stream, dev))
+    if st != 0:
+        raise FlintError(st, lib.flint_attn_last_error().decode())
+    attn_layer_fwd.last_workspace = workspace
+    return out

@@ -17,6 +17,7 @@
 
 #include "../../include/flint_attn.h"
 #include "flint_common.cuh"
+#include "flint_host.cuh"
 
 namespace flint {
 __global__ void prep_kernel(PrepParams p);
@@ -32,8 +33,11 @@ extern const unsigned kAttnThreads;
 using namespace flint;
 
 namespace {
-
 thread_local char g_err[512] = "";
+std::mutex g_mu;
+}  // namespace
+
+namespace flint {
 
 flint_status_t fail(flint_status_t s, const char* fmt, ...) {
     va_list ap;
@@ -43,16 +47,12 @@ flint_status_t fail(flint_status_t s, const char* fmt, ...) {
     return s;
 }
 
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-std::mutex g_mu;
+namespace {
 EncodeTiledFn g_encode = nullptr;
 constexpr int kMaxDevices = 64;
 int g_sms[kMaxDevices] = {0};
 bool g_attr_set[kMaxDevices] = {false};
+}  // namespace
 
 flint_status_t get_encoder(EncodeTiledFn* fn) {
     std::lock_guard<std::mutex> lk(g_mu);
@@ -91,6 +91,10 @@ flint_status_t device_setup(int* sms) {
     *sms = g_sms[dev];
     return FLINT_OK;
 }
+
+}  // namespace flint
+
+namespace {
 
 // 3-D map over a [T, heads, 128] tensor of 16-bit elements: dims (128, heads,
 // T), box (64, box_heads, box_tokens), 128-byte swizzle, zero fill outside.
@@ -213,9 +217,9 @@ flint_status_t run_stages(int stages, const void* q, const void* k, const void* 
     if (st != FLINT_OK) return st;
     char* ws = static_cast<char*>(workspace);
     CUtensorMap tm_q, tm_k, tm_v, tm_o, tm_o1;
-    // Q operand: the FP16 normalised queries that the preparation kernel
-    // left in the output rows
-    st = make_map(enc, &tm_q, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, out, kHQ, T, kGroup, kTokPerTile);
+    // Q tiles: the raw BF16 queries, normalised and rotated in shared memory
+    // by the attention kernel
+    st = make_map(enc, &tm_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, q, kHQ, T, kGroup, kTokPerTile);
     if (st != FLINT_OK) return st;
     st = make_map(enc, &tm_k, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, ws + L.kn, kHKV, T, 1, kKeyChunk);
     if (st != FLINT_OK) return st;
@@ -249,6 +253,7 @@ flint_status_t run_stages(int stages, const void* q, const void* k, const void* 
     pp.window = window;
     pp.use_rope = use_rope;
     pp.mode = mode;
+    pp.keys_ready = (stages & kStageKeysReady) ? 1 : 0;
     pp.rope_theta = rope_theta;
     pp.eps = eps;
     // ws_layout is always evaluated with max(nseg, 1) segments
@@ -303,6 +308,14 @@ flint_status_t run_stages(int stages, const void* q, const void* k, const void* 
 
 flint_status_t set_error(flint_status_t s, const char* msg) { return fail(s, "%s", msg); }
 
+struct GemmParams;
+flint_status_t launch_qkv_gemm(const void* x, const void* w_qkv, int T, int hidden, void* q, void* k,
+                               void* v, void* kn, const float* k_norm_w, float eps, int use_rope,
+                               float rope_theta, const int32_t* pos_ids, const int32_t* cu_seqlens,
+                               int nseg, int seqlen, int* status, cudaStream_t s);
+flint_status_t launch_plain_gemm(const void* a, const void* b, int M, int N, int K, void* c, int* status,
+                                 cudaStream_t s);
+
 size_t decode_workspace_bytes(int B, int cap, int window);
 flint_status_t run_decode(const void* q, const void* k, const void* v, const float* q_norm_w,
                           const float* k_norm_w, const float* sinks, void* k_cache, void* v_cache,
@@ -351,6 +364,90 @@ flint_status_t flint_attn_prepare(FLINT_ARGS) {
 flint_status_t flint_attn_attend(FLINT_ARGS) {
     NvtxRange r("flint_attn_attend");
     return run_stages(kStageAttend, FLINT_FWD_ARGS);
+}
+
+namespace {
+
+flint_status_t check_proj(int32_t T, int32_t hidden) {
+    if (T < 0 || T > FLINT_MAX_TOKENS)
+        return fail(FLINT_ERR_INVALID_ARG, "T=%d outside [0, %d]", T, FLINT_MAX_TOKENS);
+    if (hidden < 64 || hidden > FLINT_MAX_HIDDEN || hidden % 64 != 0)
+        return fail(FLINT_ERR_INVALID_ARG, "hidden=%d must be a multiple of 64 in [64, %d]", hidden,
+                    FLINT_MAX_HIDDEN);
+    return FLINT_OK;
+}
+
+}  // namespace
+
+flint_status_t flint_qkv_proj(const void* x, const void* w_qkv, int32_t T, int32_t hidden, void* q,
+                              void* k, void* v, void* stream) {
+    NvtxRange r("flint_qkv_proj");
+    g_err[0] = '\0';
+    flint_status_t st = check_proj(T, hidden);
+    if (st != FLINT_OK) return st;
+    if (T == 0) return FLINT_OK;
+    if (!x || !w_qkv || !q || !k || !v) return fail(FLINT_ERR_INVALID_ARG, "null tensor pointer");
+    if (!aligned(x, 16) || !aligned(w_qkv, 16) || !aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16))
+        return fail(FLINT_ERR_INVALID_ARG, "x, w_qkv, q, k and v must be 16-byte aligned");
+    return flint::launch_qkv_gemm(x, w_qkv, T, hidden, q, k, v, nullptr, nullptr, 1e-6f, 0, 10000.f,
+                                  nullptr, nullptr, 0, 0, nullptr, static_cast<cudaStream_t>(stream));
+}
+
+flint_status_t flint_o_proj(const void* attn_out, const void* w_o, int32_t T, int32_t hidden, void* y,
+                            void* stream) {
+    NvtxRange r("flint_o_proj");
+    g_err[0] = '\0';
+    flint_status_t st = check_proj(T, hidden);
+    if (st != FLINT_OK) return st;
+    if (T == 0) return FLINT_OK;
+    if (!attn_out || !w_o || !y) return fail(FLINT_ERR_INVALID_ARG, "null tensor pointer");
+    if (!aligned(attn_out, 16) || !aligned(w_o, 16) || !aligned(y, 16))
+        return fail(FLINT_ERR_INVALID_ARG, "attn_out, w_o and y must be 16-byte aligned");
+    return flint::launch_plain_gemm(attn_out, w_o, T, hidden, kHQ * kHD, y, nullptr,
+                                    static_cast<cudaStream_t>(stream));
+}
+
+flint_status_t flint_attn_layer_fwd(const void* x, const void* w_qkv, const void* w_o,
+                                    const float* q_norm_w, const float* k_norm_w, const float* sinks,
+                                    const int32_t* pos_ids, const int32_t* cu_seqlens, int32_t num_docs,
+                                    const uint8_t* pad_mask, int32_t batch, int32_t seqlen, int32_t T,
+                                    int32_t hidden, int32_t window, int32_t use_rope, float rope_theta,
+                                    float eps, void* q, void* k, void* v, void* attn_out, void* y,
+                                    float* lse, void* workspace, size_t workspace_bytes, void* stream) {
+    NvtxRange r("flint_attn_layer_fwd");
+    g_err[0] = '\0';
+    flint_status_t st = check_proj(T, hidden);
+    if (st != FLINT_OK) return st;
+    if (T > 0) {
+        if (!x || !w_qkv || !w_o || !y) return fail(FLINT_ERR_INVALID_ARG, "null tensor pointer");
+        if (!aligned(x, 16) || !aligned(w_qkv, 16) || !aligned(w_o, 16) || !aligned(y, 16))
+            return fail(FLINT_ERR_INVALID_ARG, "x, w_qkv, w_o and y must be 16-byte aligned");
+    }
+    // 1. plan and padded rows (every other argument is validated here, before
+    //    any launch); the keys come from the projection's epilogue
+    st = run_stages(kStagePrepare | kStageKeysReady, q, k, v, q_norm_w, k_norm_w, sinks, pos_ids,
+                    cu_seqlens, num_docs, pad_mask, batch, seqlen, T, window, use_rope, rope_theta, eps,
+                    attn_out, lse, workspace, workspace_bytes, stream);
+    if (st != FLINT_OK || T == 0) return st;
+    int nseg = 1;
+    if (cu_seqlens) nseg = num_docs;
+    else if (pad_mask) nseg = batch;
+    const WsLayout L = ws_layout(T, nseg < 1 ? 1 : nseg);
+    char* ws = static_cast<char*>(workspace);
+    int* status = &reinterpret_cast<PlanHeader*>(ws + L.header)->status;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    // 2. q, k, v and the attention kernel's key operand
+    st = flint::launch_qkv_gemm(x, w_qkv, T, hidden, q, k, v, ws + L.kn, k_norm_w, eps, use_rope, rope_theta,
+                                pos_ids, cu_seqlens, cu_seqlens ? num_docs : 0, pad_mask ? seqlen : 0,
+                                status, s);
+    if (st != FLINT_OK) return st;
+    // 3. attention
+    st = run_stages(kStageAttend, q, k, v, q_norm_w, k_norm_w, sinks, pos_ids, cu_seqlens, num_docs,
+                    pad_mask, batch, seqlen, T, window, use_rope, rope_theta, eps, attn_out, lse, workspace,
+                    workspace_bytes, stream);
+    if (st != FLINT_OK) return st;
+    // 4. o_proj
+    return flint::launch_plain_gemm(attn_out, w_o, T, hidden, kHQ * kHD, y, status, s);
 }
 
 size_t flint_attn_decode_workspace_bytes(int32_t B, int32_t cap, int32_t window) {

@@ -55,8 +55,20 @@ constexpr uint32_t kStageBytes = 32 * 128;                   // 32 rows x 64 cha
 constexpr uint32_t kOffBar = kOffStage + 8 * kStageBytes;    // mbarriers
 constexpr uint32_t kNumBars = 32;
 constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
-constexpr uint32_t kSmemUsed = kOffMisc + 64;
+constexpr uint32_t kOffInvFreq = kOffMisc + 64;              // 64 RoPE inverse frequencies (double)
+constexpr uint32_t kOffWq = kOffInvFreq + 64 * 8;            // q_norm weight (128 floats)
+constexpr uint32_t kSmemUsed = kOffWq + kHD * 4;
 constexpr uint32_t kSmemBytes = kSmemUsed + 1024;            // + alignment slack
+static_assert(kSmemBytes <= 232448, "shared memory per block");
+// RoPE table of one softmax warp's 4 tokens in its staging block: per token,
+// 32 frequency pairs (f, f+1) as {cos f, cos f+1, sin f, sin f+1} (16 bytes
+// each), then the 32 pairs {-sin f, -sin f+1} (8 bytes each); rows padded
+// by 16 bytes against bank conflicts (784 = 49 x 16 keeps every row 16-byte
+// aligned)
+constexpr uint32_t kTabCs = 32 * 16;
+constexpr uint32_t kTabStride = kTabCs + 32 * 8 + 16;
+static_assert(kTabStride % 16 == 0, "16-byte aligned table rows");
+static_assert(4 * kTabStride <= kStageBytes, "RoPE table fits the staging block");
 
 // barrier indices
 enum : uint32_t {
@@ -64,7 +76,8 @@ enum : uint32_t {
     B_Q_FULL = 4, B_Q_EMPTY = 8,
     B_K_FULL = 10, B_K_EMPTY = 12, B_V_FULL = 14, B_V_EMPTY = 16,
     B_S_FULL = 18, B_P_FULL = 20, B_O_FULL = 22, B_DRAIN = 24,
-    B_TEST_WAIT = 26     // nothing arrives here: the timeout test hook waits on it
+    B_TEST_WAIT = 26,    // nothing arrives here: the timeout test hook waits on it
+    B_Q_READY = 28       // the tile's queries normalised in place (128 arrivals)
 };
 
 struct Misc {
@@ -72,6 +85,8 @@ struct Misc {
     uint32_t tmem_base;
     int abort_flag;
     float logit_scale;   // log2(e)/sqrt(128) * 2^-(eq+ek)
+    float q_scale;       // 2^eq
+    float logit_bound;   // bound on every scaled logit (log2 units), or +inf
 };
 
 __device__ __forceinline__ float ex2(float x) {
@@ -108,6 +123,11 @@ __device__ __forceinline__ float f2_hi(uint64_t v) {
 __device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
     uint64_t r;
     asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+    return r;
+}
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
     return r;
 }
 __device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
@@ -201,6 +221,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             mbar_init(bar(B_S_FULL + t), 1);
             mbar_init(bar(B_P_FULL + t), 128);      // every softmax thread of tile t
             mbar_init(bar(B_O_FULL + t), 1);
+            mbar_init(bar(B_Q_READY + t), 128);     // every softmax thread of tile t
         }
         mbar_init(bar(B_DRAIN), 1);
         mbar_init(bar(B_TEST_WAIT), 1);
@@ -222,7 +243,29 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         if (lane == 0) {
             const int eq = prescale_exponent(mq), ek = prescale_exponent(mk);
             misc->logit_scale = ldexpf(1.4426950408889634f * 0.08838834764831845f, -(eq + ek));
+            misc->q_scale = ldexpf(1.f, eq);
+            // After the weight-form RMSNorm a head row has |x / rms(x)|_2 <=
+            // sqrt(128), so |q~|_2 <= sqrt(128) max|w_q| and likewise for k~;
+            // RoPE preserves the norm.  Every logit q~.k~ / sqrt(128) is then
+            // within sqrt(128) max|w_q| max|w_k|, i.e. log2(e) sqrt(128) =
+            // 16.3222 times that in log2 units (16.35: margin for the FP16
+            // rounding of both operands).  When that bound is small enough
+            // that 2^(s - bound) stays a normal FP32 for every logit s
+            // (bound <= 48), the online softmax starts its running max at the
+            // bound: no row max and no rescale on any chunk.
+            const float bnd = 16.35f * mq * mk + 1e-3f;
+            misc->logit_bound = (bnd <= 48.f) ? bnd : INFINITY;
         }
+    }
+    if (warp == 3) {
+        // q_norm weight and the RoPE inverse frequencies theta^(-f/64), f < 64
+        float* wq = reinterpret_cast<float*>(smem + kOffWq);
+        double* inv_freq = reinterpret_cast<double*>(smem + kOffInvFreq);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) wq[lane + 32 * i] = p.q_norm_w[lane + 32 * i];
+        const double l2t = log2((double)p.rope_theta);
+        inv_freq[lane] = exp2(-(double)lane / 64.0 * l2t);
+        inv_freq[lane + 32] = exp2(-(double)(lane + 32) / 64.0 * l2t);
     }
     // everything above overlaps the tail of the preparation kernel; the work
     // plan and the prepared keys and queries are read only after it completed
@@ -243,14 +286,32 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         if (lane == 0) {
             uint32_t sslot = 0, sph = 0, qph = 0, kst = 0, kph = 0, vst = 0, vph = 0;
             uint32_t narm_q = 0, narm_k = 0, narm_v = 0;   // loads armed so far
+            // Units are taken one ahead: while unit u streams, the raw query
+            // tiles and the first key/value chunk of the next unit are
+            // prefetched into L2, so its query prologue does not wait on HBM.
+            int u = atomicAdd(&hdr->counter, 1);
+            if (u >= n_units) u = -1;
             for (;;) {
-                int u = atomicAdd(&hdr->counter, 1);
-                if (u >= n_units) u = -1;
                 if (!mbar_wait(bar(B_SCHED_EMPTY + sslot), sph ^ 1, abort_flag, status)) break;
                 misc->sched[sslot] = u;
                 mbar_arrive(bar(B_SCHED_FULL + sslot));
                 sslot ^= 1; if (sslot == 0) sph ^= 1;
                 if (u < 0) break;
+                int un = atomicAdd(&hdr->counter, 1);
+                if (un >= n_units) un = -1;
+                if (un >= 0) {
+                    const int4 nx = items[un >> 2];
+                    const int gn = un & 3;
+                    const int kbn = p.window > 0 ? max(nx.z, nx.x - p.window + 1) : nx.z;
+                    for (int t = 0; t < 2; ++t) {
+                        tma_prefetch_3d(&tm_q, 0, kGroup * gn, nx.x + kTokPerTile * t);
+                        tma_prefetch_3d(&tm_q, 64, kGroup * gn, nx.x + kTokPerTile * t);
+                    }
+                    tma_prefetch_3d(&tm_k, 0, gn, kbn);
+                    tma_prefetch_3d(&tm_k, 64, gn, kbn);
+                    tma_prefetch_3d(&tm_v, 0, gn, kbn);
+                    tma_prefetch_3d(&tm_v, 64, gn, kbn);
+                }
                 const int4 it = items[u >> 2];
                 const int g = u & 3;
                 const int q0 = it.x, nq = it.y, ds = it.z, nch = it.w;
@@ -290,6 +351,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     vst ^= 1; if (vst == 0) vph ^= 1;
                 }
                 if (!ok) break;
+                u = un;
             }
             // drain: every armed load has landed before shared memory is released
             const unsigned long long lim = 100ull * 1000ull * 1000ull;
@@ -354,12 +416,12 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 const int kb = p.window > 0 ? max(ds, q0 - p.window + 1) : ds;
                 // S for chunk 0, each tile as soon as its Q tile has landed
                 if (!mbar_wait(bar(B_K_FULL + kst), kph, abort_flag, status)) break;
-                if (!mbar_wait(bar(B_Q_FULL + 0), qrph, abort_flag, status)) break;
+                if (!mbar_wait(bar(B_Q_READY + 0), qrph, abort_flag, status)) break;
                 tc_fence_after();
                 int ncol = chunk_cols(kb, ke);
                 issue_s(0, kst, ncol);
                 mma_commit(bar(B_S_FULL + 0));
-                if (!mbar_wait(bar(B_Q_FULL + 1), qrph, abort_flag, status)) break;
+                if (!mbar_wait(bar(B_Q_READY + 1), qrph, abort_flag, status)) break;
                 tc_fence_after();
                 qrph ^= 1;
                 issue_s(1, kst, ncol);
@@ -427,22 +489,133 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         const uint32_t t_s = tmem + (lane_base << 16) + 128u * t;
         const uint32_t t_o = tmem + (lane_base << 16) + 256u + 128u * t;
         const float C = misc->logit_scale;
-        uint32_t sslot = 0, sph = 0, s_ph = 0, oph = 0;
+        const float LB = misc->logit_bound;
+        uint32_t sslot = 0, sph = 0, s_ph = 0, oph = 0, qph = 0;
         // this warp's output staging: its 32 rows = tokens 4*(warp&3) .. +3
-        // of the tile, 64 channels at a time
+        // of the tile, 64 channels at a time; it also holds the RoPE table of
+        // those 4 tokens while a new query tile is prepared
         uint8_t* stg = smem + kOffStage + (warp - 4) * kStageBytes;
         const uint32_t stg_s = sbase + kOffStage + (warp - 4) * kStageBytes;
-        for (;;) {
-            // Warps of the warpgroup run without block-level barriers; every
-            // wait's outcome is made warp-uniform (tcgen05.ld/st are
-            // .sync.aligned) and a warp that gives up simply leaves the loop.
-            bool ok = __all_sync(0xffffffffu, mbar_wait(bar(B_SCHED_FULL + sslot), sph, abort_flag, status));
-            if (!ok) break;
-            const int u = misc->sched[sslot];
+        // Warps of the warpgroup run without block-level barriers; every
+        // wait's outcome is made warp-uniform (tcgen05.ld/st are
+        // .sync.aligned) and a warp that gives up simply leaves the loop.
+        auto fetch_unit = [&](int* u_out) -> bool {
+            if (!__all_sync(0xffffffffu, mbar_wait(bar(B_SCHED_FULL + sslot), sph, abort_flag, status)))
+                return false;
+            *u_out = misc->sched[sslot];
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(B_SCHED_EMPTY + sslot));
             sslot ^= 1; if (sslot == 0) sph ^= 1;
-            if (u < 0) break;
+            return true;
+        };
+        // Query prologue of unit `un` on this tile (FlintAttention.forward on
+        // the "flint.layers" API page: q_norm, then _apply_rope on sliding
+        // layers; model page "Model Architecture": normalisation precedes
+        // RoPE).  The producer loaded the raw BF16 rows by TMA into this
+        // tile's Q slot (128-byte swizzle, row r = token r/8, head r%8);
+        // thread r normalises row r (weight-form RMSNorm with eps), rotates
+        // channel pairs (f, f+64) by pos * theta^(-f/64) when RoPE is on,
+        // scales by 2^eq and writes it back in place as FP16, the QK^T
+        // operand.  This runs between the unit's last softmax chunk and its
+        // epilogue, while the tensor pipe works on the last PV MMAs.
+        auto prepare_q = [&](const int un) -> bool {
+            if (!__all_sync(0xffffffffu, mbar_wait(bar(B_Q_FULL + t), qph, abort_flag, status)))
+                return false;
+            qph ^= 1;
+            const int4 itn = items[un >> 2];
+            const int tok = itn.x + kTokPerTile * t + tl;
+            const uint8_t* tab = stg + (lane >> 3) * kTabStride;
+            if (p.use_rope) {
+                // this warp's 4 tokens x 32 frequency pairs, lane (token, head
+                // hl) computing pairs 4 hl .. 4 hl + 3; the block is free once
+                // lane 0's earlier output stores have read it
+                if (lane == 0) bulk_wait_group_read0();
+                __syncwarp();
+                int pos = 0;
+                if (tok < p.T) pos = p.pos_ids ? p.pos_ids[tok] : tok - itn.z;
+                const double* inv_freq = reinterpret_cast<const double*>(smem + kOffInvFreq);
+                uint8_t* tw = stg + (lane >> 3) * kTabStride;
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int pp = 4 * hl + e;                       // pair (2 pp, 2 pp + 1)
+                    float c0, s0, c1, s1;
+                    rope_cos_sin(pos, inv_freq[2 * pp], &c0, &s0);
+                    rope_cos_sin(pos, inv_freq[2 * pp + 1], &c1, &s1);
+                    *reinterpret_cast<float4*>(tw + 16 * pp) = make_float4(c0, c1, s0, s1);
+                    *reinterpret_cast<float2*>(tw + kTabCs + 8 * pp) = make_float2(-s0, -s1);
+                }
+                __syncwarp();
+            }
+            uint8_t* qrow = smem + kOffQ + t * kTileBytes + r * 128;
+            const int swz = r & 7;
+            // pass 1: sum of squares of the row (16 x 16 bytes)
+            uint64_t ss2[4] = {0ull, 0ull, 0ull, 0ull};
+#pragma unroll
+            for (int c = 0; c < 16; ++c) {
+                const uint4 a = *reinterpret_cast<const uint4*>(qrow + (c >> 3) * kHalfTile + (((c & 7) ^ swz) << 4));
+                const uint32_t av[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const uint64_t v2 = f2(__uint_as_float(av[j] << 16), __uint_as_float(av[j] & 0xFFFF0000u));
+                    ss2[j] = f2_fma(v2, v2, ss2[j]);
+                }
+            }
+            const uint64_t sst = f2_add(f2_add(ss2[0], ss2[1]), f2_add(ss2[2], ss2[3]));
+            const float rn = rsqrtf((f2_lo(sst) + f2_hi(sst)) * (1.f / kHD) + p.eps) * misc->q_scale;
+            const uint64_t rn2 = f2(rn, rn);
+            const float* wq = reinterpret_cast<const float*>(smem + kOffWq);
+            // pass 2: channels 8c .. 8c+7 of each half per step, as pairs
+            // (f, f+1) in packed FP32; y = Rot(x w) rn, written back in place
+            // as FP16
+#pragma unroll 2
+            for (int c = 0; c < 8; ++c) {
+                uint8_t* pa = qrow + ((c ^ swz) << 4);
+                uint8_t* pb = pa + kHalfTile;
+                const uint4 a = *reinterpret_cast<const uint4*>(pa);
+                const uint4 b = *reinterpret_cast<const uint4*>(pb);
+                const uint32_t av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
+                const float4 w0a = *reinterpret_cast<const float4*>(wq + 8 * c);
+                const float4 w0b = *reinterpret_cast<const float4*>(wq + 8 * c + 4);
+                const float4 w1a = *reinterpret_cast<const float4*>(wq + 64 + 8 * c);
+                const float4 w1b = *reinterpret_cast<const float4*>(wq + 64 + 8 * c + 4);
+                const uint64_t w0[4] = {f2(w0a.x, w0a.y), f2(w0a.z, w0a.w), f2(w0b.x, w0b.y), f2(w0b.z, w0b.w)};
+                const uint64_t w1[4] = {f2(w1a.x, w1a.y), f2(w1a.z, w1a.w), f2(w1b.x, w1b.y), f2(w1b.z, w1b.w)};
+                uint32_t h0[4], h1[4];
+#pragma unroll
+                for (int e2 = 0; e2 < 4; ++e2) {
+                    const uint64_t x0 = f2(__uint_as_float(av[e2] << 16), __uint_as_float(av[e2] & 0xFFFF0000u));
+                    const uint64_t x1 = f2(__uint_as_float(bv[e2] << 16), __uint_as_float(bv[e2] & 0xFFFF0000u));
+                    uint64_t n0 = f2_mul(x0, w0[e2]);
+                    uint64_t n1 = f2_mul(x1, w1[e2]);
+                    if (p.use_rope) {
+                        const int pp = 4 * c + e2;
+                        const float4 cs = *reinterpret_cast<const float4*>(tab + 16 * pp);
+                        const float2 ns = *reinterpret_cast<const float2*>(tab + kTabCs + 8 * pp);
+                        const uint64_t cc = f2(cs.x, cs.y), sn = f2(cs.z, cs.w), nsn = f2(ns.x, ns.y);
+                        const uint64_t y0 = f2_fma(n1, nsn, f2_mul(n0, cc));   // n0 cos - n1 sin
+                        const uint64_t y1 = f2_fma(n0, sn, f2_mul(n1, cc));    // n1 cos + n0 sin
+                        n0 = y0;
+                        n1 = y1;
+                    }
+                    n0 = f2_mul(n0, rn2);
+                    n1 = f2_mul(n1, rn2);
+                    const __half2 lo = __floats2half2_rn(f2_lo(n0), f2_hi(n0));
+                    const __half2 hi = __floats2half2_rn(f2_lo(n1), f2_hi(n1));
+                    h0[e2] = *reinterpret_cast<const uint32_t*>(&lo);
+                    h1[e2] = *reinterpret_cast<const uint32_t*>(&hi);
+                }
+                *reinterpret_cast<uint4*>(pa) = make_uint4(h0[0], h0[1], h0[2], h0[3]);
+                *reinterpret_cast<uint4*>(pb) = make_uint4(h1[0], h1[1], h1[2], h1[3]);
+            }
+            // generic-proxy writes -> the tensor core's (async proxy) reads
+            fence_proxy_async_smem();
+            mbar_arrive(bar(B_Q_READY + t));
+            return true;
+        };
+        int u = -1;
+        bool ok = fetch_unit(&u);
+        if (ok && u >= 0) ok = prepare_q(u);
+        while (ok && u >= 0) {
             const int4 it = items[u >> 2];
             const int g = u & 3;
             const int q0 = it.x, nq = it.y, ds = it.z, nch = it.w;
@@ -453,10 +626,21 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             const int ke = q0 + nq;
             const int kb = p.window > 0 ? max(ds, q0 - p.window + 1) : ds;
 
-            // ---- online softmax over the key chunks
+            // ---- online softmax over the key chunks.  The sink is the
+            // extra zero-value column: m starts at sink * log2(e) with l = 1,
+            // or, with a logit bound, at max(sink, bound) with l the sink's
+            // term 2^(sink - m)
             const float sink = p.sinks[h];
-            float m = sink * 1.4426950408889634f;      // log2 domain
-            float l = (sink == -INFINITY) ? 0.f : 1.f;
+            const float sink_l2 = sink * 1.4426950408889634f;   // log2 domain
+            const bool bnd = __all_sync(0xffffffffu, LB < INFINITY && sink_l2 < INFINITY);
+            float m, l;
+            if (bnd) {
+                m = fmaxf(sink_l2, LB);
+                l = ex2(sink_l2 - m);
+            } else {
+                m = sink_l2;
+                l = (sink == -INFINITY) ? 0.f : 1.f;
+            }
             const int lo = p.window > 0 ? i - p.window + 1 : -(1 << 30);
             bool alive = true;
             for (int c = 0; c < nch; ++c) {
@@ -469,10 +653,11 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 tc_fence_after();
                 const bool boundary = (c == nch - 1) || (ks + nc - 1 > tok0) ||
                                       (p.window > 0 && ks < tok0 + kTokPerTile - p.window);
-                // Interior chunks after the first with a finite running max
-                // take the fast path below (no row max).
+                // Interior chunks after the first with a finite running max,
+                // and every interior chunk under a logit bound, take the fast
+                // path below (no row max).
                 const bool fastp =
-                    !boundary && c > 0 && __all_sync(0xffffffffu, m > -INFINITY && m < INFINITY);
+                    !boundary && (bnd || (c > 0 && __all_sync(0xffffffffu, m > -INFINITY && m < INFINITY)));
                 // S columns of this chunk, one TMEM load per 32 columns.  On
                 // the fast path the exponentials of columns 0..63 overlap the
                 // load of columns 64..127.
@@ -534,6 +719,17 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                         }
                     }
                     return max3(max3(mxp[0], mxp[1], mxp[2]), max3(mxp[3], mxp[4], mxp[5]), fmaxf(mxp[6], mxp[7]));
+                };
+                // masked columns become -inf in sv (no row max)
+                auto apply_mask = [&]() {
+#pragma unroll
+                    for (int b = 0; b < 4; ++b) {
+                        if (!(fullm & (1u << b)) && !(emptym & (1u << b))) {
+#pragma unroll
+                            for (int j = 32 * b; j < 32 * b + 32; ++j)
+                                if (j < jlo || j > jhi) sv[j] = __float_as_uint(-INFINITY);
+                        }
+                    }
                 };
                 // Raise the running max to cover mx (always on the first
                 // chunk, where m still holds the sink; later only when it grew
@@ -661,7 +857,15 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     return f2_lo(ls) + f2_hi(ls);
                 };
                 float lsum = 0.f;
-                if (fastp) {
+                if (fastp && bnd) {
+                    // m is at least the logit bound: every term is at most 1
+                    lsum = exp_part(0, 2);
+                    tmem_wait_ld();                        // columns 64..127
+                    lsum += exp_part(2, 4);
+                } else if (bnd) {
+                    apply_mask();
+                    lsum = exp_blocks();
+                } else if (fastp) {
                     // Exponentials against the current m without a row max.
                     // Every term is at most the row sum, so a sum within 2^8
                     // keeps each term inside the lazy-rescale bound.  A larger
@@ -690,6 +894,12 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 mbar_arrive(bar(B_P_FULL + t));
             }
             if (!alive) break;
+
+            // ---- the next unit: its query tile is prepared now, while the
+            // tensor pipe runs this unit's last PV MMAs
+            int un = -1;
+            if (!fetch_unit(&un)) break;
+            if (un >= 0 && !prepare_q(un)) break;
 
             // ---- epilogue: O / l -> BF16, LSE
             ok = __all_sync(0xffffffffu, mbar_wait(bar(B_O_FULL + t), oph, abort_flag, status));
@@ -750,6 +960,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             }
             if (row_valid && p.lse) p.lse[(size_t)h * p.T + i] = m * 0.6931471805599453f + logf(l);
             tc_fence_before();
+            u = un;
         }
     }
 

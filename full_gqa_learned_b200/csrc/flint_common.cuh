@@ -105,7 +105,10 @@ __device__ __forceinline__ void rope_cos_sin(int pos, double inv_freq, float* c,
 }
 
 // Stages of one forward call (host side).
-enum Stage : int { kStagePrepare = 1, kStageAttend = 2, kStageBoth = 3 };
+enum Stage : int {
+    kStagePrepare = 1, kStageAttend = 2, kStageBoth = 3,
+    kStageKeysReady = 4   // with kStagePrepare: the keys were prepared by the projection GEMM
+};
 
 // Kernel parameter blocks (passed by value).
 struct PrepParams {
@@ -121,6 +124,7 @@ struct PrepParams {
     float* lse;
     char* ws;
     int T, nseg, batch, seqlen, window, use_rope, mode;
+    int keys_ready;      // 1: the key operand is already in the workspace
     float rope_theta, eps;
 };
 

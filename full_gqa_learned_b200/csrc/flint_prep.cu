@@ -6,15 +6,15 @@
 // their number of 128-key chunks, longest first, so the attention kernel's
 // dynamic scheduler hands out the largest items first.
 //
-// The other blocks prepare the keys and queries once per token instead of
-// once per use: per-head RMSNorm with k_norm_w / q_norm_w (weight form; HF
-// discussion #26 on RecursiveSI/flint), then on sliding layers NeoX RoPE at
-// the document-local position (FlintAttention._apply_rope), scaled by a power
-// of two and rounded to FP16.  Keys go to the workspace; queries go to the
-// output rows of their own token, which the attention kernel reads back as
-// its Q operand before it writes the result over them.  Padded query tokens
-// get their final outputs here: zeros and lse = sink (FlintAttention.forward,
-// attention_mask: the sink remains valid for padded queries).
+// The other blocks prepare the keys once per token instead of once per use
+// (each key is read by up to 33 query tiles on a sliding layer): per-head
+// RMSNorm with k_norm_w (weight form; HF discussion #26 on RecursiveSI/flint),
+// then on sliding layers NeoX RoPE at the document-local position
+// (FlintAttention._apply_rope), scaled by a power of two and rounded to FP16
+// into the workspace.  Queries are used by one tile only; the attention kernel
+// normalises and rotates them itself.  Padded query tokens get their final
+// outputs here: zeros and lse = sink (FlintAttention.forward, attention_mask:
+// the sink remains valid for padded queries).
 #include "flint_common.cuh"
 #include "sm100.cuh"
 
@@ -248,8 +248,8 @@ __device__ __forceinline__ void norm_rope_row(const __nv_bfloat16* src, __half* 
 
 __device__ void prepare_tokens(const PrepParams& p) {
     __shared__ double s_inv_freq[64];
-    __shared__ float s_wk[kHD], s_wq[kHD];
-    __shared__ float s_kscale, s_qscale;
+    __shared__ float s_wk[kHD];
+    __shared__ float s_kscale;
     __shared__ int s_thd_end;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const WsLayout L = ws_layout(p.T, p.nseg);
@@ -257,27 +257,22 @@ __device__ void prepare_tokens(const PrepParams& p) {
 
     if (tid < 64) s_inv_freq[tid] = exp2(-(double)tid / 64.0 * log2((double)p.rope_theta));
     if (tid < kHD) s_wk[tid] = p.k_norm_w[tid];
-    if (tid >= kHD && tid < 2 * kHD) s_wq[tid - kHD] = p.q_norm_w[tid - kHD];
     if (warp == 0) {
         const float m = warp_max_abs128(p.k_norm_w);
         if (lane == 0) s_kscale = ldexpf(1.f, prescale_exponent(m));
-    }
-    if (warp == 1) {
-        const float m = warp_max_abs128(p.q_norm_w);
-        if (lane == 0) s_qscale = ldexpf(1.f, prescale_exponent(m));
     }
     if (tid == 0) s_thd_end = (p.mode == kMaskThd) ? p.cu_seqlens[p.nseg] : p.T;
     __syncthreads();
 
     const int head = lane >> 3, sub = lane & 7;
     const int nwarps_total = (gridDim.x - 1) * (blockDim.x >> 5);
-    const float kscale = s_kscale, qscale = s_qscale;
+    const float kscale = s_kscale;
     const bool rope = p.use_rope != 0;
     for (int t = (blockIdx.x - 1) * (blockDim.x >> 5) + warp; t < p.T; t += nwarps_total) {
         // ---- the lane's 8 (cos, sin) pairs f = 8*sub + e at the token's
-        // document-local position, shared by its 4 key and 32 query heads
+        // document-local position, shared by its 4 key heads
         float cc[8], sn[8];
-        if (rope) {
+        if (rope && !p.keys_ready) {
             int pos;
             if (p.pos_ids) pos = p.pos_ids[t];
             else if (p.mode == kMaskThd) pos = t - (t < s_thd_end ? thd_segment_start(p.cu_seqlens, p.nseg, t) : s_thd_end);
@@ -297,8 +292,9 @@ __device__ void prepare_tokens(const PrepParams& p) {
             }
         }
         // ---- the 4 key heads (head = lane / 8)
-        norm_rope_row(p.k + ((size_t)t * kHKV + head) * kHD, kn + ((size_t)t * kHKV + head) * kHD,
-                      s_wk, p.eps, kscale, sub, rope, cc, sn);
+        if (!p.keys_ready)
+            norm_rope_row(p.k + ((size_t)t * kHKV + head) * kHD, kn + ((size_t)t * kHKV + head) * kHD,
+                          s_wk, p.eps, kscale, sub, rope, cc, sn);
 
         bool padded;
         if (p.mode == kMaskThd) padded = t >= s_thd_end;
@@ -311,17 +307,6 @@ __device__ void prepare_tokens(const PrepParams& p) {
 #pragma unroll 4
             for (int i = lane; i < kHQ * kHD / 8; i += 32) o[i] = z;
             if (p.lse) p.lse[(size_t)lane * p.T + t] = p.sinks[lane];
-        } else {
-            // ---- the 32 query heads, 4 per pass, into the output rows of
-            // the token: the attention kernel reads them back as its FP16
-            // Q operand and overwrites them with the result
-            const __nv_bfloat16* qrow = p.q + (size_t)t * kHQ * kHD;
-            __half* qdst = reinterpret_cast<__half*>(p.out + (size_t)t * kHQ * kHD);
-#pragma unroll 2
-            for (int hq = 0; hq < kHQ / kHKV; ++hq) {
-                const int hh = kHKV * hq + head;
-                norm_rope_row(qrow + hh * kHD, qdst + hh * kHD, s_wq, p.eps, qscale, sub, rope, cc, sn);
-            }
         }
     }
 }

@@ -107,11 +107,9 @@ FLINT_API size_t flint_attn_workspace_bytes(int32_t T, int32_t num_segments);
  *  rope_theta RoPE base (> 1), e.g. 10000.
  *  eps        RMSNorm epsilon (> 0), 1e-6 for Flint.
  *  out        bf16 [T,4096]: out[t, h*128 + c], the o_proj input.  Rows of
- *             padded tokens are written as +0.0.  The call also uses out as
- *             scratch: the preparation kernel leaves each valid token's
- *             normalised FP16 queries in its rows and the attention kernel
- *             overwrites them with the result.  out may be q itself; it must
- *             not overlap k, v, lse or the workspace.
+ *             padded tokens are written as +0.0.  out may be q itself (each
+ *             query row is read before the result is written over it); it
+ *             must not overlap k, v, lse or the workspace.
  *  lse        fp32 [32,T] natural-log sum of exponentials including the sink
  *             (lse[h*T + t]); padded tokens get sinks[h].  May be NULL.
  *  workspace  device buffer of at least flint_attn_workspace_bytes(T, n)
@@ -135,13 +133,12 @@ FLINT_API flint_status_t flint_attn_fwd(const void* q, const void* k, const void
 /*
  * The two stages flint_attn_fwd enqueues, exposed so a caller (or a profiler)
  * can time them apart.  flint_attn_prepare runs the preparation kernel: the
- * work plan, the normalised/rotated FP16 keys in the workspace, the
- * normalised/rotated FP16 queries in the rows of out (intermediate values,
- * not a result) and the outputs of padded query tokens.  flint_attn_attend
- * runs the attention kernel on a workspace and an out that flint_attn_prepare
- * filled with the same arguments; calling it with other arguments, or after
- * out was modified in between, is undefined.  Both take the
- * arguments of flint_attn_fwd and validate them the same way.
+ * work plan, the normalised/rotated FP16 keys in the workspace and the
+ * outputs of padded query tokens.  flint_attn_attend runs the attention
+ * kernel (which normalises and rotates the queries itself) on a workspace
+ * that flint_attn_prepare filled with the same arguments; calling it with
+ * other arguments is undefined.  Both take the arguments of flint_attn_fwd
+ * and validate them the same way.
  */
 FLINT_API flint_status_t flint_attn_prepare(const void* q, const void* k, const void* v,
                               const float* q_norm_w, const float* k_norm_w,
@@ -314,16 +311,18 @@ FLINT_API flint_status_t flint_attn_decode(const void* q, const void* k, const v
  *             dq, dk and dv too; no output may overlap an input, another
  *             output or the workspace.
  *  workspace  device buffer of at least flint_attn_bwd_workspace_bytes(T)
- *             bytes (about 18.6 KiB per token), 256-byte aligned; holds the
+ *             bytes (about 9.3 KiB per token), 256-byte aligned; holds the
  *             device status (flint_attn_device_status: FLINT_ERR_INVALID_ARG
  *             for an ill-formed cu_seqlens, FLINT_ERR_UNSUPPORTED for a
- *             non-trailing mask), per-token document bounds, FP32 q~ and k~
- *             and per-CTA partial sums.
+ *             non-trailing mask, FLINT_ERR_TIMEOUT), per-token document
+ *             bounds, D, the FP16 operands q~ and k~ and per-CTA partial sums.
  *  stream     cudaStream_t as void*.
  *
  * T == 0 sets dq_norm_w, dk_norm_w and dsinks to zero and does nothing else.
- * Computed in FP32 on CUDA cores; the norm-weight and sink gradients are
- * summed in a fixed order, so repeated calls give identical bits.
+ * The products run on the tensor cores (tcgen05; q~, k~ and dS in FP16, v,
+ * dout and P in BF16, FP32 accumulation), the RoPE and RMSNorm adjoints on
+ * CUDA cores in FP32; every sum has a fixed order, so repeated calls give
+ * identical bits.
  */
 FLINT_API size_t flint_attn_bwd_workspace_bytes(int32_t T);
 FLINT_API flint_status_t flint_attn_bwd(const void* q, const void* k, const void* v,
@@ -337,6 +336,67 @@ FLINT_API flint_status_t flint_attn_bwd(const void* q, const void* k, const void
                            float* dv, float* dq_norm_w, float* dk_norm_w,
                            float* dsinks, void* workspace, size_t workspace_bytes,
                            void* stream);
+
+/* Largest hidden size of the projection entry points. */
+#define FLINT_MAX_HIDDEN 65536
+
+/*
+ * The projections around the attention core: FlintAttention.forward (NeMo
+ * AutoModel "flint.layers" API page) maps hidden states x [T, hidden] to
+ * q = x W_q^T, k = x W_k^T, v = x W_v^T (bias-free: FlintConfig
+ * attention_bias = False), runs the attention above on them and returns
+ * y = a W_o^T.  Weights use the PyTorch Linear layout [out, in], BF16; q, k
+ * and v are head-major (column h*128 + c).  Products accumulate in FP32 on
+ * the tensor cores (tcgen05) and are rounded to BF16 once.
+ *
+ * flint_qkv_proj: the fused projection.
+ *  x          bf16 [T, hidden], hidden a multiple of 64 in [64, FLINT_MAX_HIDDEN].
+ *  w_qkv      bf16 [5120, hidden]: W_q (rows 0..4095), W_k (4096..4607) and
+ *             W_v (4608..5119) stacked.
+ *  q          bf16 [T, 32, 128]; k, v bf16 [T, 4, 128]: the projections,
+ *             as flint_attn_fwd takes them.
+ *  All pointers are device pointers, 16-byte aligned; no output may overlap
+ *  an input.  T == 0 is a no-op.  Asynchronous on `stream`.
+ *
+ * flint_o_proj: y = attn_out W_o^T.
+ *  attn_out   bf16 [T, 4096] (flint_attn_fwd's out);  w_o bf16 [hidden, 4096];
+ *  y          bf16 [T, hidden].
+ *
+ * Bounded waits inside these two kernels cannot report a timeout (there is
+ * no workspace); flint_attn_layer_fwd records one in its workspace status.
+ */
+FLINT_API flint_status_t flint_qkv_proj(const void* x, const void* w_qkv, int32_t T, int32_t hidden,
+                              void* q, void* k, void* v, void* stream);
+FLINT_API flint_status_t flint_o_proj(const void* attn_out, const void* w_o, int32_t T,
+                              int32_t hidden, void* y, void* stream);
+
+/*
+ * The whole attention layer: flint_qkv_proj, the attention forward, then
+ * flint_o_proj, with the key prologue fused into the projection: its
+ * epilogue writes the normalised, rotated FP16 keys the attention kernel
+ * reads straight into the workspace (FlintAttention.forward; model page
+ * "Model Architecture": query/key normalisation precedes RoPE), so the
+ * preparation kernel only plans the work and writes padded rows, and the
+ * attention kernel normalises and rotates the queries on tile load.
+ *
+ *  x, w_qkv, w_o, hidden      as for flint_qkv_proj / flint_o_proj.
+ *  q_norm_w ... eps           as for flint_attn_fwd.
+ *  q, k, v    bf16 outputs: the raw projections (kept for the backward).
+ *  attn_out   bf16 [T, 4096]: the attention output (o_proj's input).
+ *  y          bf16 [T, hidden]: the layer's output.
+ *  lse        fp32 [32, T] or NULL.
+ *  workspace  at least flint_attn_workspace_bytes(T, n) bytes, as for
+ *             flint_attn_fwd; read its status with flint_attn_device_status.
+ */
+FLINT_API flint_status_t flint_attn_layer_fwd(const void* x, const void* w_qkv, const void* w_o,
+                              const float* q_norm_w, const float* k_norm_w,
+                              const float* sinks, const int32_t* pos_ids,
+                              const int32_t* cu_seqlens, int32_t num_docs,
+                              const uint8_t* pad_mask, int32_t batch, int32_t seqlen,
+                              int32_t T, int32_t hidden, int32_t window, int32_t use_rope,
+                              float rope_theta, float eps, void* q, void* k, void* v,
+                              void* attn_out, void* y, float* lse,
+                              void* workspace, size_t workspace_bytes, void* stream);
 
 /* Text of the last error raised on the calling host thread ("" if none). */
 FLINT_API const char* flint_attn_last_error(void);

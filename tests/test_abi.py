@@ -23,7 +23,7 @@ def lib():
 def declared_functions():
     text = open(HEADER).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(flint_attn_\w+)\s*\(", text)))
+    return sorted(set(re.findall(r"\b(flint_\w+)\s*\(", text)))
 
 
 def test_header_declares_the_boundary():
@@ -192,9 +192,10 @@ def call_bwd(lib, **kw):
 
 
 def test_bwd_workspace_bytes(lib):
-    # FP32 q~ and k~ dominate: 18 KiB per token, plus fixed per-CTA partials
+    # the FP16 tensor-core operands q~, k~ dominate: 9 KiB per token, plus
+    # bounds and D (136 bytes per token) and fixed per-CTA partials
     a = fa.bwd_workspace_bytes(4096)
-    assert 4096 * (16384 + 2048) <= a < 4096 * (16384 + 2048 + 512) + (4 << 20)
+    assert 4096 * (8192 + 1024) <= a < 4096 * (8192 + 1024 + 256) + (4 << 20)
     assert fa.bwd_workspace_bytes(0) > 0
     assert fa.bwd_workspace_bytes(-1) == 0
     assert fa.bwd_workspace_bytes((1 << 24) + 1) == 0
@@ -252,3 +253,50 @@ def test_header_is_plain_c_and_links_against_the_library(lib, tmp_path):
                         "-Wl,-rpath," + os.path.dirname(fa.LIB_PATH)],
                        capture_output=True, text=True)
     assert r.returncode == 0, r.stderr
+
+
+# ---------------------------------------------------------------- projections and layer
+
+def call_proj(lib, which, **kw):
+    a = dict(x=A, w=A, T=64, hidden=2048, o0=A, o1=A, o2=A, stream=None)
+    a.update(kw)
+    if which == "qkv":
+        return lib.flint_qkv_proj(a["x"], a["w"], a["T"], a["hidden"], a["o0"], a["o1"], a["o2"],
+                                  a["stream"])
+    return lib.flint_o_proj(a["x"], a["w"], a["T"], a["hidden"], a["o0"], a["stream"])
+
+
+@pytest.mark.parametrize("which", ["qkv", "o"])
+@pytest.mark.parametrize("kw", [dict(T=-1), dict(T=(1 << 24) + 1), dict(hidden=0), dict(hidden=100),
+                                dict(hidden=1 << 20), dict(x=None), dict(w=None), dict(o0=None),
+                                dict(x=A + 8), dict(w=A + 2), dict(o0=A + 4)])
+def test_projection_arguments_rejected_on_host(lib, which, kw):
+    assert call_proj(lib, which, **kw) == 1
+    assert lib.flint_attn_last_error() != b""
+
+
+@pytest.mark.parametrize("which", ["qkv", "o"])
+def test_projection_empty_input_is_a_noop(lib, which):
+    assert call_proj(lib, which, T=0, x=None, w=None, o0=None, o1=None, o2=None) == 0
+
+
+def call_layer(lib, **kw):
+    a = dict(x=A, wqkv=A, wo=A, wq=A, wk=A, sinks=A, pos=None, cu=None, ndocs=0, mask=None, batch=0,
+             seqlen=0, T=64, hidden=2048, window=513, use_rope=1, theta=1e4, eps=1e-6, q=A, k=A, v=A,
+             a=A, y=A, lse=A, ws=A, ws_bytes=1 << 40, stream=None)
+    a.update(kw)
+    return lib.flint_attn_layer_fwd(a["x"], a["wqkv"], a["wo"], a["wq"], a["wk"], a["sinks"], a["pos"],
+                                    a["cu"], a["ndocs"], a["mask"], a["batch"], a["seqlen"], a["T"],
+                                    a["hidden"], a["window"], a["use_rope"], a["theta"], a["eps"],
+                                    a["q"], a["k"], a["v"], a["a"], a["y"], a["lse"], a["ws"],
+                                    a["ws_bytes"], a["stream"])
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(hidden=96), 1), (dict(x=None), 1), (dict(wo=None), 1), (dict(y=A + 2), 1),
+    (dict(window=-1), 1), (dict(q=None), 1), (dict(a=None), 1), (dict(ws=None), 5),
+    (dict(ws_bytes=1024), 5), (dict(cu=A, mask=A), 1),
+])
+def test_layer_arguments_rejected_on_host(lib, kw, status):
+    assert call_layer(lib, **kw) == status
+    assert lib.flint_attn_last_error() != b""

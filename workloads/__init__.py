@@ -377,3 +377,66 @@ DECODE_CONFIGS = {
 
 def make_decode_named(name: str) -> DecodeWorkload:
     return make_decode(name=name, **DECODE_CONFIGS[name])
+
+
+# ---------------------------------------------------------------- whole layer
+
+HIDDEN = 2048    # FlintConfig hidden size ("flint" model page, "Model Architecture")
+
+
+@dataclasses.dataclass
+class LayerWorkload:
+    """Inputs of the whole attention layer: hidden states and the projection
+    weights in the PyTorch Linear layout, plus the attention's own inputs.
+
+    x: uint16 [T, hidden] BF16 bits, N(0,1).
+    w_qkv: uint16 [5120, hidden]: W_q, W_k, W_v stacked, N(0, 1/hidden), so
+      the projections are ~N(0,1) like the attention workloads' q, k, v.
+    w_o: uint16 [hidden, 4096], N(0, 1/4096).
+    attn: the attention part (norm weights, sinks, positions, masks, window;
+      its q, k, v are unused)."""
+    name: str
+    x: np.ndarray
+    w_qkv: np.ndarray
+    w_o: np.ndarray
+    attn: Workload
+
+    @property
+    def T(self) -> int:
+        return int(self.x.shape[0])
+
+    @property
+    def hidden(self) -> int:
+        return int(self.x.shape[1])
+
+    def proj_flops(self) -> float:
+        """QKV projection plus o_proj: 2 FLOPs per multiply-add."""
+        return 2.0 * self.T * self.hidden * (HQ * D + 2 * HKV * D) + 2.0 * self.T * (HQ * D) * self.hidden
+
+    def flops(self) -> float:
+        return self.proj_flops() + self.attn.flops()
+
+
+def make_layer(T, seed, *, hidden=HIDDEN, window=0, use_rope=False, cu_seqlens=None, pad_mask=None,
+               name="layer") -> LayerWorkload:
+    """Seeded whole-layer inputs; draw order x, w_qkv, w_o, then the attention
+    part (make_small with seed + 1)."""
+    rng = np.random.default_rng(seed)
+    x = bf16_bits(_normal(rng, (T, hidden)))
+    w_qkv = bf16_bits(_normal(rng, (HQ * D + 2 * HKV * D, hidden), 1.0 / np.sqrt(hidden)))
+    w_o = bf16_bits(_normal(rng, (hidden, HQ * D), 1.0 / np.sqrt(HQ * D)))
+    attn = make_small(T, seed + 1, window=window, use_rope=use_rope, cu_seqlens=cu_seqlens,
+                      pad_mask=pad_mask, name=name)
+    return LayerWorkload(name, x, w_qkv, w_o, attn)
+
+
+# whole-layer workloads: the full layer at S=4096 and the sliding layer at
+# S=1024, with the checkpoint's hidden size
+LAYER_CONFIGS = {
+    "layer_full_s4096": dict(T=4096, seed=41, window=0, use_rope=False),
+    "layer_sliding_s1024": dict(T=1024, seed=42, window=WINDOW, use_rope=True),
+}
+
+
+def make_layer_named(name: str) -> LayerWorkload:
+    return make_layer(name=name, **LAYER_CONFIGS[name])
