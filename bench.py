@@ -555,8 +555,6 @@ def decode_line(args, world, d, total_ms, clocks):
 BWD_PREFIX = "bwd_"
 BWD_METRIC = ("sink-attn backward TFLOP/s (window-aware algorithmic FLOPs: 2.5x the forward's, "
               "five contractions per pair and head)")
-# FP32 FMA rate of the CUDA cores: 148 SMs x 128 lanes x 2 FLOPs x 1.965 GHz
-ALU_FP32_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 
 
 def bwd_flops(w):
@@ -684,25 +682,27 @@ def _bwd_cpu_sample(w, budget_s, OB, rng):
 
 def bwd_line(args, world, r):
     w = r["w"]
+    peaks, src = load_peaks()
+    peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     flops = bwd_flops(w)
     step_ms = r["total_ms"] / args.steps
     tf = flops / (step_ms * 1e-3) / 1e12
     return dict(
         metric=BWD_METRIC, value=round(tf * world, 4), unit=UNIT, n_gpus=world, steps=args.steps,
         warmup=args.warmup, ms_per_step=round(step_ms, 5), higher_is_better=True, scaling="weak",
-        vs_baseline=None, dtype="f32",
+        vs_baseline=None, dtype="bf16",
         data="synthetic (the forward workload's seeded inputs; N(0,1) BF16 upstream gradient)",
         config=dict(workload=args.workload, T=w.T, window=w.window, use_rope=bool(w.use_rope),
                     l2="flushed before every timed step (256 MiB write)", per_rank="independent replica",
                     seed=w.seed, gpu=r["gpu"]),
-        roofline=dict(bound="alu", achieved=round(tf, 4), peak=round(ALU_FP32_TFLOPS, 2), unit=UNIT,
-                      frac=round(tf / ALU_FP32_TFLOPS, 4), traffic=None,
-                      kernel="flint bwd call (segments, prep, dq, dkv, finish kernels)",
-                      peak_source="derived: FP32 FMA rate of 148 SMs x 128 lanes at 1.965 GHz",
-                      flops_per_launch=flops),
+        roofline=dict(bound="tensor", achieved=round(tf, 4), peak=peak, unit=UNIT,
+                      frac=round(tf / peak, 4), traffic=None,
+                      kernel="flint bwd call (segments, prep, tcgen05 dq and dk/dv, adjoint, finish kernels)",
+                      peak_source="%s bf16_tflops (burst)" % src, flops_per_launch=flops,
+                      note="algorithmic FLOPs (5 products per pair); the tensor cores run 7"),
         e2e=dict(value=round(flops / (r["e2e_ms"] * 1e-3) / 1e12 * world, 4), unit=UNIT,
                  h2d_bytes_per_step=r["h2d"], d2h_bytes_per_step=r["d2h"], ms_per_step=round(r["e2e_ms"], 4)),
-        gpu_launches=5 * args.steps, clocks=r["clocks"])
+        gpu_launches=6 * args.steps, clocks=r["clocks"])
 
 
 # ---------------------------------------------------------------- whole-layer leg

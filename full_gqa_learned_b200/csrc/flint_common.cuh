@@ -34,6 +34,9 @@ enum MaskMode : int { kMaskSingle = 0, kMaskThd = 1, kMaskPad = 2 };
 // Workspace layout; all regions 256-byte aligned, the key buffer 1024-byte.
 struct WsLayout {
     size_t header, seg, prefix, hist, items, kn, total;
+    // FP16 attention-compute policy only (after `total`): the normalised,
+    // rotated FP16 queries and the FP16 values
+    size_t qn, vh, total_f16;
     int max_items, hist_len;
 };
 
@@ -50,8 +53,11 @@ __host__ __device__ inline WsLayout ws_layout(int T, int nseg) {
     L.prefix = o; o = ws_align(o + sizeof(int) * (size_t)(nseg + 2), 256);
     L.hist = o;   o = ws_align(o + sizeof(int) * (size_t)L.hist_len, 256);
     L.items = o;  o = ws_align(o + sizeof(int) * 4 * (size_t)L.max_items, 1024);
-    L.kn = o;     o = ws_align(o + (size_t)T * kHKV * kHD * 2, 256);
+    L.kn = o;     o = ws_align(o + (size_t)T * kHKV * kHD * 2, 1024);
     L.total = o;
+    L.qn = o;     o = ws_align(o + (size_t)T * kHQ * kHD * 2, 1024);
+    L.vh = o;     o = ws_align(o + (size_t)T * kHKV * kHD * 2, 256);
+    L.total_f16 = o;
     return L;
 }
 
@@ -107,7 +113,8 @@ __device__ __forceinline__ void rope_cos_sin(int pos, double inv_freq, float* c,
 // Stages of one forward call (host side).
 enum Stage : int {
     kStagePrepare = 1, kStageAttend = 2, kStageBoth = 3,
-    kStageKeysReady = 4   // with kStagePrepare: the keys were prepared by the projection GEMM
+    kStageKeysReady = 4,  // with kStagePrepare: the keys were prepared by the projection GEMM
+    kStageF16 = 8         // FP16 attention-compute policy: FP32 q/k/v in, FP16 out
 };
 
 // Kernel parameter blocks (passed by value).
@@ -125,6 +132,11 @@ struct PrepParams {
     char* ws;
     int T, nseg, batch, seqlen, window, use_rope, mode;
     int keys_ready;      // 1: the key operand is already in the workspace
+    int f16;             // FP16 policy: q, k, v are FP32 (qf, kf, vf); queries
+                         // and values are prepared into the workspace in FP16
+    const float* qf;
+    const float* kf;
+    const float* vf;
     float rope_theta, eps;
 };
 

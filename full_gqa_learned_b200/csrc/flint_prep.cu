@@ -194,23 +194,36 @@ __device__ __forceinline__ int thd_segment_start(const int* cu, int ndocs, int t
 // Normalise one 128-channel head row held by 8 lanes (lane sub owns channels
 // 8*sub .. 8*sub+7 of each 64-channel half): RMSNorm in weight form, optional
 // NeoX rotation with the lane's 8 (cos, sin) pairs, x scale, FP16.
-__device__ __forceinline__ void norm_rope_row(const __nv_bfloat16* src, __half* dst, const float* w,
-                                              float eps, float scale, int sub, bool rope,
-                                              const float* cc, const float* sn) {
+// The lane's 16 input values: channels 8 sub .. 8 sub + 7 and 64 + 8 sub ..
+__device__ __forceinline__ void load_row16(const __nv_bfloat16* src, int sub, float* x0, float* x1) {
     const uint4 a = *reinterpret_cast<const uint4*>(src + 8 * sub);
     const uint4 b = *reinterpret_cast<const uint4*>(src + 64 + 8 * sub);
-    float x0[8], x1[8];
-    {
-        const __nv_bfloat162* pa = reinterpret_cast<const __nv_bfloat162*>(&a);
-        const __nv_bfloat162* pb = reinterpret_cast<const __nv_bfloat162*>(&b);
+    const __nv_bfloat162* pa = reinterpret_cast<const __nv_bfloat162*>(&a);
+    const __nv_bfloat162* pb = reinterpret_cast<const __nv_bfloat162*>(&b);
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const float2 fa = __bfloat1622float2(pa[e]);
-            const float2 fb = __bfloat1622float2(pb[e]);
-            x0[2 * e] = fa.x; x0[2 * e + 1] = fa.y;
-            x1[2 * e] = fb.x; x1[2 * e + 1] = fb.y;
-        }
+    for (int e = 0; e < 4; ++e) {
+        const float2 fa = __bfloat1622float2(pa[e]);
+        const float2 fb = __bfloat1622float2(pb[e]);
+        x0[2 * e] = fa.x; x0[2 * e + 1] = fa.y;
+        x1[2 * e] = fb.x; x1[2 * e + 1] = fb.y;
     }
+}
+__device__ __forceinline__ void load_row16(const float* src, int sub, float* x0, float* x1) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const float4 a = *reinterpret_cast<const float4*>(src + 8 * sub + 4 * h);
+        const float4 b = *reinterpret_cast<const float4*>(src + 64 + 8 * sub + 4 * h);
+        x0[4 * h] = a.x; x0[4 * h + 1] = a.y; x0[4 * h + 2] = a.z; x0[4 * h + 3] = a.w;
+        x1[4 * h] = b.x; x1[4 * h + 1] = b.y; x1[4 * h + 2] = b.z; x1[4 * h + 3] = b.w;
+    }
+}
+
+template <typename In>
+__device__ __forceinline__ void norm_rope_row(const In* src, __half* dst, const float* w,
+                                              float eps, float scale, int sub, bool rope,
+                                              const float* cc, const float* sn) {
+    float x0[8], x1[8];
+    load_row16(src, sub, x0, x1);
     float ss = 0.f;
 #pragma unroll
     for (int e = 0; e < 8; ++e) ss = fmaf(x0[e], x0[e], fmaf(x1[e], x1[e], ss));
@@ -248,8 +261,8 @@ __device__ __forceinline__ void norm_rope_row(const __nv_bfloat16* src, __half* 
 
 __device__ void prepare_tokens(const PrepParams& p) {
     __shared__ double s_inv_freq[64];
-    __shared__ float s_wk[kHD];
-    __shared__ float s_kscale;
+    __shared__ float s_wk[kHD], s_wq[kHD];
+    __shared__ float s_kscale, s_qscale;
     __shared__ int s_thd_end;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const WsLayout L = ws_layout(p.T, p.nseg);
@@ -257,9 +270,14 @@ __device__ void prepare_tokens(const PrepParams& p) {
 
     if (tid < 64) s_inv_freq[tid] = exp2(-(double)tid / 64.0 * log2((double)p.rope_theta));
     if (tid < kHD) s_wk[tid] = p.k_norm_w[tid];
+    if (tid >= kHD && tid < 2 * kHD) s_wq[tid - kHD] = p.q_norm_w[tid - kHD];
     if (warp == 0) {
         const float m = warp_max_abs128(p.k_norm_w);
         if (lane == 0) s_kscale = ldexpf(1.f, prescale_exponent(m));
+    }
+    if (warp == 1) {
+        const float m = warp_max_abs128(p.q_norm_w);
+        if (lane == 0) s_qscale = ldexpf(1.f, prescale_exponent(m));
     }
     if (tid == 0) s_thd_end = (p.mode == kMaskThd) ? p.cu_seqlens[p.nseg] : p.T;
     __syncthreads();
@@ -272,7 +290,7 @@ __device__ void prepare_tokens(const PrepParams& p) {
         // ---- the lane's 8 (cos, sin) pairs f = 8*sub + e at the token's
         // document-local position, shared by its 4 key heads
         float cc[8], sn[8];
-        if (rope && !p.keys_ready) {
+        if (rope && (p.f16 || !p.keys_ready)) {
             int pos;
             if (p.pos_ids) pos = p.pos_ids[t];
             else if (p.mode == kMaskThd) pos = t - (t < s_thd_end ? thd_segment_start(p.cu_seqlens, p.nseg, t) : s_thd_end);
@@ -292,9 +310,25 @@ __device__ void prepare_tokens(const PrepParams& p) {
             }
         }
         // ---- the 4 key heads (head = lane / 8)
-        if (!p.keys_ready)
+        if (p.f16)
+            norm_rope_row(p.kf + ((size_t)t * kHKV + head) * kHD, kn + ((size_t)t * kHKV + head) * kHD,
+                          s_wk, p.eps, kscale, sub, rope, cc, sn);
+        else if (!p.keys_ready)
             norm_rope_row(p.k + ((size_t)t * kHKV + head) * kHD, kn + ((size_t)t * kHKV + head) * kHD,
                           s_wk, p.eps, kscale, sub, rope, cc, sn);
+        if (p.f16) {
+            // FP16 policy: the values cast to FP16 (4 heads x 128 per token,
+            // 16 per lane)
+            __half* vh = reinterpret_cast<__half*>(p.ws + L.vh) + (size_t)t * kHKV * kHD;
+            const float* vs = p.vf + (size_t)t * kHKV * kHD;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const float4 a = *reinterpret_cast<const float4*>(vs + 4 * lane + 128 * i);
+                const __half2 lo = __floats2half2_rn(a.x, a.y), hi = __floats2half2_rn(a.z, a.w);
+                *reinterpret_cast<uint2*>(vh + 4 * lane + 128 * i) =
+                    make_uint2(*reinterpret_cast<const uint32_t*>(&lo), *reinterpret_cast<const uint32_t*>(&hi));
+            }
+        }
 
         bool padded;
         if (p.mode == kMaskThd) padded = t >= s_thd_end;
@@ -307,6 +341,16 @@ __device__ void prepare_tokens(const PrepParams& p) {
 #pragma unroll 4
             for (int i = lane; i < kHQ * kHD / 8; i += 32) o[i] = z;
             if (p.lse) p.lse[(size_t)lane * p.T + t] = p.sinks[lane];
+        } else if (p.f16) {
+            // ---- FP16 policy: the 32 query heads normalised and rotated in
+            // FP32 and cast to FP16 (x 2^eq) into the workspace, 4 per pass
+            const float* qrow = p.qf + (size_t)t * kHQ * kHD;
+            __half* qdst = reinterpret_cast<__half*>(p.ws + L.qn) + (size_t)t * kHQ * kHD;
+#pragma unroll 2
+            for (int hq = 0; hq < kHQ / kHKV; ++hq) {
+                const int hh = kHKV * hq + head;
+                norm_rope_row(qrow + hh * kHD, qdst + hh * kHD, s_wq, p.eps, s_qscale, sub, rope, cc, sn);
+            }
         }
     }
 }

@@ -80,7 +80,7 @@ def _segments(doc):
 
 
 def attn_bwd(q, k, v, q_norm_w, k_norm_w, sinks, dout, *, pos_ids=None, cu_seqlens=None,
-             pad_mask=None, window=0, use_rope=False, rope_theta=10000.0, eps=1e-6):
+             pad_mask=None, window=0, use_rope=False, rope_theta=10000.0, eps=1e-6, out_given=None):
     """Gradients of sum(dout * out) for the forward with these arguments.
 
     q [T,32,128], k and v [T,4,128] (BF16 bit patterns or floats), weights
@@ -88,6 +88,10 @@ def attn_bwd(q, k, v, q_norm_w, k_norm_w, sinks, dout, *, pos_ids=None, cu_seqle
     index of each token within its document.  Returns a dict of
     float64 arrays: dq [T,32,128], dk, dv [T,4,128], dq_norm_w, dk_norm_w
     [128], dsinks [32], and the forward's out [T,32,128] and lse [T,32].
+
+    out_given: a forward output [T,32,128] to take D_i = dO_i . out_i from
+    instead of the exact one (the same formula evaluated at a stored forward
+    output, as a backward that receives `out` does); None: the exact output.
     """
     qx, kx, vx = _f64(q), _f64(k), _f64(v)
     T = qx.shape[0]
@@ -95,6 +99,7 @@ def attn_bwd(q, k, v, q_norm_w, k_norm_w, sinks, dout, *, pos_ids=None, cu_seqle
     kx = kx.reshape(T, HKV, D)
     vx = vx.reshape(T, HKV, D)
     do = _f64(dout).reshape(T, HQ, D)
+    og = None if out_given is None else _f64(out_given).reshape(T, HQ, D)
     wq = _f64(q_norm_w).reshape(D)
     wk = _f64(k_norm_w).reshape(D)
     sk = np.asarray(sinks, np.float64).reshape(HQ)
@@ -145,7 +150,7 @@ def attn_bwd(q, k, v, q_norm_w, k_norm_w, sinks, dout, *, pos_ids=None, cu_seqle
                 out[a:b, h] = O
                 lse[a:b, h] = ls
                 dO = do[a:b, h]
-                Dr = np.sum(dO * O, axis=1)
+                Dr = np.sum(dO * (O if og is None else og[a:b, h]), axis=1)
                 dv[a:b, g] += P.T @ dO
                 dS = P * (dO @ V.T - Dr[:, None])
                 dsinks[h] += -np.sum(Psink * Dr)
@@ -169,8 +174,8 @@ def attn_bwd(q, k, v, q_norm_w, k_norm_w, sinks, dout, *, pos_ids=None, cu_seqle
                 out=out, lse=lse)
 
 
-def attn_bwd_workload(w, dout):
+def attn_bwd_workload(w, dout, out_given=None):
     """The oracle on a ``workloads.Workload`` with upstream gradient dout."""
     return attn_bwd(w.q, w.k, w.v, w.q_norm_w, w.k_norm_w, w.sinks, dout, pos_ids=w.pos_ids,
                     cu_seqlens=w.cu_seqlens, pad_mask=w.pad_mask, window=w.window,
-                    use_rope=w.use_rope, rope_theta=w.rope_theta, eps=w.eps)
+                    use_rope=w.use_rope, rope_theta=w.rope_theta, eps=w.eps, out_given=out_given)

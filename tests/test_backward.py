@@ -4,19 +4,26 @@ The GPU path is the one a training step runs: the library's forward produces
 out and lse, and the backward takes them with a BF16 upstream gradient.  The
 oracle computes the exact gradient from the same inputs (its own forward).
 
-Tolerances, from the arithmetic:
+The backward takes the forward's out and computes D_i = dO_i . out_i from it
+(include/flint_attn.h, flint_attn_bwd), so the reference is the gradient
+formula evaluated at the same stored output (the oracle's out_given); the
+forward's own error is covered by the forward's parity tests.  Against that
+reference, from the arithmetic:
 * each probability is exp(s - lse) with the forward's FP32 lse, whose error
   is at most the forward's LSE bound (1e-3) and in practice the FP16-operand
   floor (~5e-4); that scales a row's probabilities by at most 1e-3;
-* D = dO . out uses the forward's BF16 out (2^-9 relative rounding per
-  element, plus the forward's own error);
-* everything else runs in FP32 (~1e-6 relative over a few thousand terms).
-So dq, dk, dv: relative L2 <= 5e-3 and max |err| <= 1e-2 max |ref| (a CPU
-emulation of these error sources, with lse perturbed by +-5e-4, gives 3e-4).
+* the products run on the tensor cores with q~, k~ and dS in FP16 and P in
+  BF16 (an FP64 emulation of those roundings: dv 1.7e-3, dq and dk 7e-4
+  relative L2), accumulating in FP32.
+So dq, dk, dv: relative L2 <= 5e-3 and max |err| <= 1e-2 max |ref|.
 dsinks_h = -sum_i exp(sink_h - lse_i) D_i sums signed terms, so its bound is
 relative to the sum of absolute terms A_h = sum_i exp(sink_h - lse_i)
 sum_c |dO_ic out_ic|: |err| <= 1e-2 A_h.  The norm weights' gradients sum
 T x heads signed row terms: relative L2 <= 1e-2.
+
+End to end, against the exact gradient (exact out in D), the forward's BF16
+output adds its rounding to D; where a row's D nearly cancels dO . v (a row
+dominated by one key) that error is amplified, so the bound there is 1e-2.
 """
 import numpy as np
 import pytest
@@ -50,7 +57,9 @@ def _run(w, dO_bits):
     g = fa.attn_bwd(q, k, v, wq, wk, sk, out, lse, dO, **kw)
     assert fa.device_status(fa.attn_bwd.last_workspace) == 0
     torch.cuda.synchronize()
-    return {n: x.cpu().numpy().astype(np.float64) for n, x in g.items()}, (q, k, v, wq, wk, sk, out, lse, dO, kw)
+    got = {n: x.cpu().numpy().astype(np.float64) for n, x in g.items()}
+    got["fwd_out"] = out.float().cpu().numpy().astype(np.float64).reshape(w.T, 32, 128)
+    return got, (q, k, v, wq, wk, sk, out, lse, dO, kw)
 
 
 def _dout_bits(T, seed):
@@ -58,7 +67,12 @@ def _dout_bits(T, seed):
 
 
 def _compare(w, dO_bits, got):
-    ref = OB.attn_bwd_workload(w, oracle._f64(dO_bits))
+    exact = OB.attn_bwd_workload(w, oracle._f64(dO_bits))
+    for key in ("dq", "dk", "dv"):
+        e = got[key] - exact[key]
+        assert np.linalg.norm(e) <= 1e-2 * np.linalg.norm(exact[key]) + 1e-30, \
+            ("end to end", key, np.linalg.norm(e) / np.linalg.norm(exact[key]))
+    ref = OB.attn_bwd_workload(w, oracle._f64(dO_bits), out_given=got["fwd_out"])
     for key in ("dq", "dk", "dv"):
         e = got[key] - ref[key]
         scale = np.abs(ref[key]).max()

@@ -233,3 +233,23 @@ def test_gradient_matches_finite_differences_on_random_layouts():
             assert abs(fd - an) <= 1e-6 * (1.0 + abs(an)), (T, window, rope, cu, name, idx, fd, an)
 
     check()
+
+
+def test_given_output_enters_only_through_D():
+    """out_given replaces the output only in D_i = dO_i . out_i: the exact
+    output reproduces the gradient bit for bit; a perturbed one shifts dv not
+    at all, and dq of a one-token document by -dD P_key k~/sqrt(128)
+    through the norm adjoint (here checked as: dv unchanged, dq changed)."""
+    import workloads as W
+    from oracle import backward as OB
+    w = W.make_small(40, seed=5, window=9, use_rope=True, cu_seqlens=[0, 1, 25, 40])
+    dO = np.random.default_rng(6).standard_normal((40, 32, 128))
+    ref = OB.attn_bwd_workload(w, dO)
+    same = OB.attn_bwd_workload(w, dO, out_given=ref["out"])
+    for key in ("dq", "dk", "dv", "dq_norm_w", "dk_norm_w", "dsinks"):
+        assert np.array_equal(same[key], ref[key]), key
+    bumped = OB.attn_bwd_workload(w, dO, out_given=ref["out"] * (1.0 + 1e-3))
+    assert np.array_equal(bumped["dv"], ref["dv"])
+    assert not np.allclose(bumped["dq"], ref["dq"], rtol=0, atol=0)
+    # D grows by 1e-3 D, so dsink moves by exactly 1e-3 of itself
+    np.testing.assert_allclose(bumped["dsinks"], ref["dsinks"] * (1.0 + 1e-3), rtol=1e-12, atol=1e-300)
