@@ -254,6 +254,10 @@ flint_status_t run_stages(int stages, const void* q, const void* k, const void* 
     pp.use_rope = use_rope;
     pp.mode = mode;
     pp.keys_ready = (stages & kStageKeysReady) ? 1 : 0;
+    pp.f16 = 0;
+    pp.qf = nullptr;
+    pp.kf = nullptr;
+    pp.vf = nullptr;
     pp.rope_theta = rope_theta;
     pp.eps = eps;
     // ws_layout is always evaluated with max(nseg, 1) segments
