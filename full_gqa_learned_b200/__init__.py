@@ -17,7 +17,7 @@ import os
 import threading
 from typing import Optional, Tuple
 
-__all__ = ["attn_fwd", "attn_fwd_static", "static_status", "qkv_proj", "o_proj", "attn_layer_fwd",
+__all__ = ["attn_fwd", "attn_fwd_heads", "attn_fwd_fp16", "fp16_workspace_bytes", "attn_fwd_static", "static_status", "qkv_proj", "o_proj", "attn_layer_fwd",
            "attn_decode", "attn_bwd", "flint_attention", "workspace_bytes",
            "decode_workspace_bytes", "bwd_workspace_bytes", "device_status", "load_library",
            "FlintError", "LIB_PATH", "HQ", "HKV", "HEAD_DIM", "STATUS", "STATIC_SCRATCH_BYTES"]
@@ -59,6 +59,12 @@ def load_library() -> ctypes.CDLL:
         for name in ("flint_attn_fwd", "flint_attn_prepare", "flint_attn_attend"):
             getattr(lib, name).restype = ctypes.c_int
             getattr(lib, name).argtypes = fwd_args
+        lib.flint_attn_fwd_heads.restype = ctypes.c_int
+        lib.flint_attn_fwd_heads.argtypes = fwd_args[:13] + [I32] + fwd_args[13:]
+        lib.flint_attn_fwd_fp16.restype = ctypes.c_int
+        lib.flint_attn_fwd_fp16.argtypes = fwd_args
+        lib.flint_attn_fp16_workspace_bytes.restype = ctypes.c_size_t
+        lib.flint_attn_fp16_workspace_bytes.argtypes = [I32, I32]
         lib.flint_attn_fwd_static.restype = ctypes.c_int
         lib.flint_attn_fwd_static.argtypes = fwd_args[:19] + [P]
         lib.flint_attn_fwd_static_status.restype = ctypes.c_int
@@ -523,3 +529,109 @@ def attn_layer_fwd(x, w_qkv, w_o, q_norm_w, k_norm_w, sinks, *, pos_ids=None, cu
         raise FlintError(st, lib.flint_attn_last_error().decode())
     attn_layer_fwd.last_workspace = workspace
     return out
+
+
+def fp16_workspace_bytes(T: int, num_segments: int = 1) -> int:
+    return int(load_library().flint_attn_fp16_workspace_bytes(int(T), int(num_segments)))
+
+
+def attn_fwd_fp16(q, k, v, q_norm_w, k_norm_w, sinks, *, pos_ids=None, cu_seqlens=None,
+                  pad_mask=None, window: int = 513, use_rope: bool = True,
+                  rope_theta: float = 10000.0, eps: float = 1e-6, out=None, lse=None,
+                  workspace=None, stream=None, want_lse: bool = True) -> Tuple[object, object]:
+    """flint_attn_fwd_fp16, the FP16 attention-compute policy: q [T,32,128],
+    k/v [T,4,128] float32 CUDA tensors; returns (out [T,4096] float16, lse
+    [32,T] float32 or None).  Other arguments as for attn_fwd."""
+    import torch
+    lib = load_library()
+    T = int(q.shape[0]) if q.dim() >= 1 else 0
+    _check(q, "q", torch.float32, (T, HQ, HEAD_DIM))
+    _check(k, "k", torch.float32, (T, HKV, HEAD_DIM))
+    _check(v, "v", torch.float32, (T, HKV, HEAD_DIM))
+    _check(q_norm_w, "q_norm_w", torch.float32, (HEAD_DIM,))
+    _check(k_norm_w, "k_norm_w", torch.float32, (HEAD_DIM,))
+    _check(sinks, "sinks", torch.float32, (HQ,))
+    num_docs, batch, seqlen, nseg = 0, 0, 0, 1
+    if pos_ids is not None:
+        _check(pos_ids, "pos_ids", torch.int32, (T,))
+    if cu_seqlens is not None:
+        _check(cu_seqlens, "cu_seqlens", torch.int32)
+        num_docs = int(cu_seqlens.numel()) - 1
+        nseg = max(num_docs, 1)
+    if pad_mask is not None:
+        _check(pad_mask, "pad_mask", torch.uint8)
+        batch, seqlen = int(pad_mask.shape[0]), int(pad_mask.shape[1])
+        nseg = batch
+    dev = q.device
+    if out is None:
+        out = torch.empty((T, HQ * HEAD_DIM), dtype=torch.float16, device=dev)
+    _check(out, "out", torch.float16, (T, HQ * HEAD_DIM))
+    if lse is None and want_lse:
+        lse = torch.empty((HQ, T), dtype=torch.float32, device=dev)
+    if lse is not None:
+        _check(lse, "lse", torch.float32, (HQ, T))
+    if workspace is None:
+        workspace = torch.empty(max(fp16_workspace_bytes(T, nseg), 256), dtype=torch.uint8, device=dev)
+    _check(workspace, "workspace", torch.uint8)
+    with torch.cuda.device(dev):
+        st = lib.flint_attn_fwd_fp16(
+            _ptr(q), _ptr(k), _ptr(v), _ptr(q_norm_w), _ptr(k_norm_w), _ptr(sinks), _ptr(pos_ids),
+            _ptr(cu_seqlens), num_docs, _ptr(pad_mask), batch, seqlen, T, int(window),
+            int(bool(use_rope)), float(rope_theta), float(eps), _ptr(out), _ptr(lse), _ptr(workspace),
+            int(workspace.numel()), _stream_ptr(stream, dev))
+    if st != 0:
+        raise FlintError(st, lib.flint_attn_last_error().decode())
+    attn_fwd_fp16.last_workspace = workspace
+    return out, lse
+
+
+def attn_fwd_heads(q, k, v, q_norm_w, k_norm_w, sinks, *, pos_ids=None, cu_seqlens=None,
+                   pad_mask=None, window: int = 513, use_rope: bool = True, rope_theta: float = 10000.0,
+                   eps: float = 1e-6, out=None, lse=None, workspace=None, stream=None,
+                   want_lse: bool = True) -> Tuple[object, object]:
+    """flint_attn_fwd_heads: the forward on a slice of kv_heads KV heads
+    (q [T, 8 kv_heads, 128], k/v [T, kv_heads, 128], sinks [8 kv_heads]);
+    returns (out [T, 8 kv_heads x 128] bf16, lse [8 kv_heads, T])."""
+    import torch
+    lib = load_library()
+    T = int(q.shape[0]) if q.dim() >= 1 else 0
+    ng = int(k.shape[1]) if k.dim() == 3 else 0
+    nh = 8 * ng
+    _check(q, "q", torch.bfloat16, (T, nh, HEAD_DIM))
+    _check(k, "k", torch.bfloat16, (T, ng, HEAD_DIM))
+    _check(v, "v", torch.bfloat16, (T, ng, HEAD_DIM))
+    _check(q_norm_w, "q_norm_w", torch.float32, (HEAD_DIM,))
+    _check(k_norm_w, "k_norm_w", torch.float32, (HEAD_DIM,))
+    _check(sinks, "sinks", torch.float32, (nh,))
+    num_docs, batch, seqlen, nseg = 0, 0, 0, 1
+    if pos_ids is not None:
+        _check(pos_ids, "pos_ids", torch.int32, (T,))
+    if cu_seqlens is not None:
+        _check(cu_seqlens, "cu_seqlens", torch.int32)
+        num_docs = int(cu_seqlens.numel()) - 1
+        nseg = max(num_docs, 1)
+    if pad_mask is not None:
+        _check(pad_mask, "pad_mask", torch.uint8)
+        batch, seqlen = int(pad_mask.shape[0]), int(pad_mask.shape[1])
+        nseg = batch
+    dev = q.device
+    if out is None:
+        out = torch.empty((T, nh * HEAD_DIM), dtype=torch.bfloat16, device=dev)
+    _check(out, "out", torch.bfloat16, (T, nh * HEAD_DIM))
+    if lse is None and want_lse:
+        lse = torch.empty((nh, T), dtype=torch.float32, device=dev)
+    if lse is not None:
+        _check(lse, "lse", torch.float32, (nh, T))
+    if workspace is None:
+        workspace = torch.empty(max(workspace_bytes(T, nseg), 256), dtype=torch.uint8, device=dev)
+    _check(workspace, "workspace", torch.uint8)
+    with torch.cuda.device(dev):
+        st = lib.flint_attn_fwd_heads(
+            _ptr(q), _ptr(k), _ptr(v), _ptr(q_norm_w), _ptr(k_norm_w), _ptr(sinks), _ptr(pos_ids),
+            _ptr(cu_seqlens), num_docs, _ptr(pad_mask), batch, seqlen, T, ng, int(window),
+            int(bool(use_rope)), float(rope_theta), float(eps), _ptr(out), _ptr(lse), _ptr(workspace),
+            int(workspace.numel()), _stream_ptr(stream, dev))
+    if st != 0:
+        raise FlintError(st, lib.flint_attn_last_error().decode())
+    attn_fwd_heads.last_workspace = workspace
+    return out, lse

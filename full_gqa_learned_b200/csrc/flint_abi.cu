@@ -26,6 +26,11 @@ __global__ void attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q,
                                 const __grid_constant__ CUtensorMap tm_v,
                                 const __grid_constant__ CUtensorMap tm_o,
                                 const __grid_constant__ CUtensorMap tm_o1, const AttnParams p);
+__global__ void attn_fwd_f16_kernel(const __grid_constant__ CUtensorMap tm_q,
+                                    const __grid_constant__ CUtensorMap tm_k,
+                                    const __grid_constant__ CUtensorMap tm_v,
+                                    const __grid_constant__ CUtensorMap tm_o,
+                                    const __grid_constant__ CUtensorMap tm_o1, const AttnParams p);
 extern const unsigned kAttnSmemBytes;
 extern const unsigned kAttnThreads;
 }  // namespace flint
@@ -83,6 +88,9 @@ flint_status_t device_setup(int* sms) {
             return fail(FLINT_ERR_UNSUPPORTED, "needs an sm_100 GPU, found sm_%d%d", major, minor);
         e = cudaFuncSetAttribute(attn_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)kAttnSmemBytes);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(attn_fwd_f16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)kAttnSmemBytes);
         if (e != cudaSuccess)
             return fail(FLINT_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
         cudaDeviceGetAttribute(&g_sms[dev], cudaDevAttrMultiProcessorCount, dev);
@@ -167,8 +175,12 @@ flint_status_t run_stages(int stages, const void* q, const void* k, const void* 
                    const int32_t* cu_seqlens, int32_t num_docs, const uint8_t* pad_mask,
                    int32_t batch, int32_t seqlen, int32_t T, int32_t window, int32_t use_rope,
                    float rope_theta, float eps, void* out, float* lse, void* workspace,
-                   size_t workspace_bytes, void* stream) {
+                   size_t workspace_bytes, void* stream, int ng = kHKV) {
     g_err[0] = '\0';
+    if (ng != 1 && ng != 2 && ng != 4)
+        return fail(FLINT_ERR_INVALID_ARG, "kv_heads=%d: a head slice has 1, 2 or 4 KV heads", ng);
+    if (ng != kHKV && (stages & (kStageF16 | kStageKeysReady)))
+        return fail(FLINT_ERR_UNSUPPORTED, "head slices use the BF16 forward only");
     // ---- host-side validation: nothing below touches the GPU until it passes
     if (T < 0 || T > FLINT_MAX_TOKENS)
         return fail(FLINT_ERR_INVALID_ARG, "T=%d outside [0, %d]", T, FLINT_MAX_TOKENS);
@@ -201,12 +213,13 @@ flint_status_t run_stages(int stages, const void* q, const void* k, const void* 
         (lse && !aligned(lse, 4)) || (pos_ids && !aligned(pos_ids, 4)) ||
         (cu_seqlens && !aligned(cu_seqlens, 4)))
         return fail(FLINT_ERR_INVALID_ARG, "misaligned 32-bit array");
+    const bool f16 = (stages & kStageF16) != 0;
     const WsLayout L = ws_layout(T, nseg < 1 ? 1 : nseg);
+    const size_t need = f16 ? L.total_f16 : L.total;
     if (!workspace || !aligned(workspace, 256))
         return fail(FLINT_ERR_WORKSPACE, "workspace missing or not 256-byte aligned");
-    if (workspace_bytes < L.total)
-        return fail(FLINT_ERR_WORKSPACE, "workspace too small: %zu < %zu bytes", workspace_bytes,
-                    L.total);
+    if (workspace_bytes < need)
+        return fail(FLINT_ERR_WORKSPACE, "workspace too small: %zu < %zu bytes", workspace_bytes, need);
 
     // ---- launch
     int sms = 0;
@@ -218,18 +231,21 @@ flint_status_t run_stages(int stages, const void* q, const void* k, const void* 
     char* ws = static_cast<char*>(workspace);
     CUtensorMap tm_q, tm_k, tm_v, tm_o, tm_o1;
     // Q tiles: the raw BF16 queries, normalised and rotated in shared memory
-    // by the attention kernel
-    st = make_map(enc, &tm_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, q, kHQ, T, kGroup, kTokPerTile);
+    // by the attention kernel (FP16 policy: the FP16 queries the preparation
+    // kernel normalised and rotated into the workspace)
+    const CUtensorMapDataType t16 = f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    const int nh = kGroup * ng;      // query heads in the tensors
+    st = make_map(enc, &tm_q, t16, f16 ? static_cast<const void*>(ws + L.qn) : q, nh, T, kGroup, kTokPerTile);
     if (st != FLINT_OK) return st;
-    st = make_map(enc, &tm_k, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, ws + L.kn, kHKV, T, 1, kKeyChunk);
+    st = make_map(enc, &tm_k, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, ws + L.kn, ng, T, 1, kKeyChunk);
     if (st != FLINT_OK) return st;
     // result: 4 tokens (the rows of one softmax warp), and single tokens
     // where a document ends inside a warp's 4
-    st = make_map(enc, &tm_o, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, out, kHQ, T, kGroup, 4);
+    st = make_map(enc, &tm_o, t16, out, nh, T, kGroup, 4);
     if (st != FLINT_OK) return st;
-    st = make_map(enc, &tm_o1, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, out, kHQ, T, kGroup, 1);
+    st = make_map(enc, &tm_o1, t16, out, nh, T, kGroup, 1);
     if (st != FLINT_OK) return st;
-    st = make_map(enc, &tm_v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, v, kHKV, T, 1, kKeyChunk);
+    st = make_map(enc, &tm_v, t16, f16 ? static_cast<const void*>(ws + L.vh) : v, ng, T, 1, kKeyChunk);
     if (st != FLINT_OK) return st;
 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -254,10 +270,15 @@ flint_status_t run_stages(int stages, const void* q, const void* k, const void* 
     pp.use_rope = use_rope;
     pp.mode = mode;
     pp.keys_ready = (stages & kStageKeysReady) ? 1 : 0;
-    pp.f16 = 0;
-    pp.qf = nullptr;
-    pp.kf = nullptr;
-    pp.vf = nullptr;
+    pp.ng = ng;
+    pp.f16 = f16 ? 1 : 0;
+    pp.qf = f16 ? static_cast<const float*>(q) : nullptr;
+    pp.kf = f16 ? static_cast<const float*>(k) : nullptr;
+    pp.vf = f16 ? static_cast<const float*>(v) : nullptr;
+    if (f16) {
+        pp.q = nullptr;
+        pp.k = nullptr;
+    }
     pp.rope_theta = rope_theta;
     pp.eps = eps;
     // ws_layout is always evaluated with max(nseg, 1) segments
@@ -283,10 +304,11 @@ flint_status_t run_stages(int stages, const void* q, const void* k, const void* 
     ap.nseg = pp.nseg;
     ap.window = window;
     ap.use_rope = use_rope;
+    ap.ng = ng;
     ap.rope_theta = rope_theta;
     ap.eps = eps;
     ap.test_wait_ns = test_stall_once();
-    const int max_units = L.max_items * kHKV;
+    const int max_units = L.max_items * ng;
     const int grid = max_units < sms ? max_units : sms;
     if (stages & kStagePrepare) {
         // launched right behind the preparation kernel: a programmatic
@@ -301,9 +323,13 @@ flint_status_t run_stages(int stages, const void* q, const void* k, const void* 
         attr[0].val.programmaticStreamSerializationAllowed = 1;
         cfg.attrs = attr;
         cfg.numAttrs = 1;
-        e = cudaLaunchKernelEx(&cfg, attn_fwd_kernel, tm_q, tm_k, tm_v, tm_o, tm_o1, ap);
+        e = f16 ? cudaLaunchKernelEx(&cfg, attn_fwd_f16_kernel, tm_q, tm_k, tm_v, tm_o, tm_o1, ap)
+                : cudaLaunchKernelEx(&cfg, attn_fwd_kernel, tm_q, tm_k, tm_v, tm_o, tm_o1, ap);
     } else {
-        attn_fwd_kernel<<<grid, kAttnThreads, kAttnSmemBytes, s>>>(tm_q, tm_k, tm_v, tm_o, tm_o1, ap);
+        if (f16)
+            attn_fwd_f16_kernel<<<grid, kAttnThreads, kAttnSmemBytes, s>>>(tm_q, tm_k, tm_v, tm_o, tm_o1, ap);
+        else
+            attn_fwd_kernel<<<grid, kAttnThreads, kAttnSmemBytes, s>>>(tm_q, tm_k, tm_v, tm_o, tm_o1, ap);
         e = cudaGetLastError();
     }
     if (e != cudaSuccess) return fail(FLINT_ERR_CUDA, "attention launch: %s", cudaGetErrorString(e));
@@ -360,6 +386,29 @@ struct NvtxRange {
 flint_status_t flint_attn_fwd(FLINT_ARGS) {
     NvtxRange r("flint_attn_fwd");
     return run_stages(kStageBoth, FLINT_FWD_ARGS);
+}
+flint_status_t flint_attn_fwd_heads(const void* q, const void* k, const void* v, const float* q_norm_w,
+                                    const float* k_norm_w, const float* sinks, const int32_t* pos_ids,
+                                    const int32_t* cu_seqlens, int32_t num_docs, const uint8_t* pad_mask,
+                                    int32_t batch, int32_t seqlen, int32_t T, int32_t kv_heads,
+                                    int32_t window, int32_t use_rope, float rope_theta, float eps, void* out,
+                                    float* lse, void* workspace, size_t workspace_bytes, void* stream) {
+    NvtxRange r("flint_attn_fwd_heads");
+    return run_stages(kStageBoth, FLINT_FWD_ARGS, kv_heads);
+}
+size_t flint_attn_fp16_workspace_bytes(int32_t T, int32_t num_segments) {
+    if (T < 0 || T > FLINT_MAX_TOKENS || num_segments < 0 || num_segments > FLINT_MAX_TOKENS)
+        return 0;
+    return ws_layout(T, num_segments < 1 ? 1 : num_segments).total_f16;
+}
+flint_status_t flint_attn_fwd_fp16(const float* q, const float* k, const float* v, const float* q_norm_w,
+                                   const float* k_norm_w, const float* sinks, const int32_t* pos_ids,
+                                   const int32_t* cu_seqlens, int32_t num_docs, const uint8_t* pad_mask,
+                                   int32_t batch, int32_t seqlen, int32_t T, int32_t window,
+                                   int32_t use_rope, float rope_theta, float eps, void* out, float* lse,
+                                   void* workspace, size_t workspace_bytes, void* stream) {
+    NvtxRange r("flint_attn_fwd_fp16");
+    return run_stages(kStageBoth | kStageF16, FLINT_FWD_ARGS);
 }
 flint_status_t flint_attn_prepare(FLINT_ARGS) {
     NvtxRange r("flint_attn_prepare");

@@ -184,10 +184,27 @@ __device__ __forceinline__ int chunk_cols(int ks, int ke) {
     return (n + 15) & ~15;
 }
 
-__global__ void __launch_bounds__(kThreads, 1)
-attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
-                const __grid_constant__ CUtensorMap tm_o1, const AttnParams p) {
+// Two FP32 values -> packed 16-bit pair for the PV operand and the output:
+// BF16, or FP16 under the FP16 attention-compute policy.
+template <bool F16>
+__device__ __forceinline__ uint32_t pack_pv(float lo, float hi) {
+    if constexpr (F16) {
+        const __half2 h = __floats2half2_rn(lo, hi);
+        return *reinterpret_cast<const uint32_t*>(&h);
+    } else {
+        return pack_bf16(lo, hi);
+    }
+}
+
+// The kernel body.  F16: the FP16 attention-compute policy ("flint" model
+// page, "Numerical comparison": normalised, rotated Q/K/V cast to FP16 for
+// the attention): the queries arrive normalised and rotated in FP16 from the
+// preparation kernel, values are FP16, P and the output are FP16, and the
+// softmax keeps its exact running max (P stays within FP16's normal range).
+template <bool F16>
+__device__ __forceinline__ void attn_fwd_body(const CUtensorMap& tm_q, const CUtensorMap& tm_k,
+                                              const CUtensorMap& tm_v, const CUtensorMap& tm_o,
+                                              const CUtensorMap& tm_o1, const AttnParams& p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~uintptr_t(1023));
@@ -254,7 +271,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             // (bound <= 48), the online softmax starts its running max at the
             // bound: no row max and no rescale on any chunk.
             const float bnd = 16.35f * mq * mk + 1e-3f;
-            misc->logit_bound = (bnd <= 48.f) ? bnd : INFINITY;
+            misc->logit_bound = (!F16 && bnd <= 48.f) ? bnd : INFINITY;
         }
     }
     if (warp == 3) {
@@ -274,7 +291,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = misc->tmem_base;
-    const int n_units = hdr->n_items * kHKV;
+    const int n_units = hdr->n_items * p.ng;
 
     // Registers: launched with 384 x 168 = 64512.  Warps 0-3 (producer, MMA,
     // two idle) drop to kRegsControl, the two softmax warpgroups rise to
@@ -300,8 +317,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 int un = atomicAdd(&hdr->counter, 1);
                 if (un >= n_units) un = -1;
                 if (un >= 0) {
-                    const int4 nx = items[un >> 2];
-                    const int gn = un & 3;
+                    const int4 nx = items[un / p.ng];
+                    const int gn = un % p.ng;
                     const int kbn = p.window > 0 ? max(nx.z, nx.x - p.window + 1) : nx.z;
                     for (int t = 0; t < 2; ++t) {
                         tma_prefetch_3d(&tm_q, 0, kGroup * gn, nx.x + kTokPerTile * t);
@@ -312,8 +329,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     tma_prefetch_3d(&tm_v, 0, gn, kbn);
                     tma_prefetch_3d(&tm_v, 64, gn, kbn);
                 }
-                const int4 it = items[u >> 2];
-                const int g = u & 3;
+                const int4 it = items[u / p.ng];
+                const int g = u % p.ng;
                 const int q0 = it.x, nq = it.y, ds = it.z, nch = it.w;
                 bool ok = true;
                 for (int t = 0; t < 2 && ok; ++t) {
@@ -368,7 +385,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       } else if (warp == 1) {
         // ============================================================ MMA issuer
         if (lane == 0) {
-            const uint32_t idesc_pv = idesc_f16(1, 1, 1, 128);
+            const uint32_t idesc_pv = idesc_f16(F16 ? 0u : 1u, F16 ? 0u : 1u, 1, 128);
             // Descriptor words.  Only the low word (start address) changes
             // between MMAs; the issuing thread shares its scheduler with two
             // busy softmax warps, so each MMA is kept to a 32-bit add and the
@@ -410,7 +427,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 mbar_arrive(bar(B_SCHED_EMPTY + sslot));
                 sslot ^= 1; if (sslot == 0) sph ^= 1;
                 if (u < 0) break;
-                const int4 it = items[u >> 2];
+                const int4 it = items[u / p.ng];
                 const int q0 = it.x, nq = it.y, ds = it.z, nch = it.w;
                 const int ke = q0 + nq;
                 const int kb = p.window > 0 ? max(ds, q0 - p.window + 1) : ds;
@@ -522,7 +539,12 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             if (!__all_sync(0xffffffffu, mbar_wait(bar(B_Q_FULL + t), qph, abort_flag, status)))
                 return false;
             qph ^= 1;
-            const int4 itn = items[un >> 2];
+            if constexpr (F16) {
+                // the preparation kernel already normalised and rotated them
+                mbar_arrive(bar(B_Q_READY + t));
+                return true;
+            }
+            const int4 itn = items[un / p.ng];
             const int tok = itn.x + kTokPerTile * t + tl;
             const uint8_t* tab = stg + (lane >> 3) * kTabStride;
             if (p.use_rope) {
@@ -616,8 +638,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         bool ok = fetch_unit(&u);
         if (ok && u >= 0) ok = prepare_q(u);
         while (ok && u >= 0) {
-            const int4 it = items[u >> 2];
-            const int g = u & 3;
+            const int4 it = items[u / p.ng];
+            const int g = u % p.ng;
             const int q0 = it.x, nq = it.y, ds = it.z, nch = it.w;
             const int h = kGroup * g + hl;
             const int tok0 = q0 + kTokPerTile * t;
@@ -781,7 +803,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                                 if ((j & 7) < kPolyPairs) pp = exp2_poly2(x);
                                 else pp = f2(ex2(f2_lo(x)), ex2(f2_hi(x)));
                                 lp[j & 3] = f2_add(lp[j & 3], pp);
-                                pk[j] = pack_bf16(f2_lo(pp), f2_hi(pp));
+                                pk[j] = pack_pv<F16>(f2_lo(pp), f2_hi(pp));
                             }
                             tmem_st16(t_s + 16u * b, pk);
                         }
@@ -795,7 +817,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                                                              __uint_as_float(sv[32 * b + 2 * j + 1])), C2, negm2);
                                 const uint64_t pp = f2(ex2(f2_lo(x)), ex2(f2_hi(x)));
                                 lp[j & 3] = f2_add(lp[j & 3], pp);
-                                pk[j] = pack_bf16(f2_lo(pp), f2_hi(pp));
+                                pk[j] = pack_pv<F16>(f2_lo(pp), f2_hi(pp));
                             }
                             tmem_st16(t_s + 16u * b, pk);
                         }
@@ -820,7 +842,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                             if ((j & 7) < kPolyPairs) pp = exp2_poly2(x);
                             else pp = f2(ex2(f2_lo(x)), ex2(f2_hi(x)));
                             lp[j & 3] = f2_add(lp[j & 3], pp);
-                            pk[j] = pack_bf16(f2_lo(pp), f2_hi(pp));
+                            pk[j] = pack_pv<F16>(f2_lo(pp), f2_hi(pp));
                         }
                         tmem_st16(t_s + 16u * b, pk);
                     }
@@ -848,7 +870,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                                                              __uint_as_float(sv[32 * b + 2 * j + 1])), C2, negm2);
                                 const uint64_t pp = f2(ex2(f2_lo(x)), ex2(f2_hi(x)));
                                 lp[j & 3] = f2_add(lp[j & 3], pp);
-                                pk[j] = pack_bf16(f2_lo(pp), f2_hi(pp));
+                                pk[j] = pack_pv<F16>(f2_lo(pp), f2_hi(pp));
                             }
                         }
                         if (b < nblk) tmem_st16(t_s + 16u * b, pk);
@@ -925,7 +947,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 tmem_wait_ld();
 #pragma unroll
                 for (int j = 0; j < 32; ++j)
-                    pk[j] = pack_bf16(__uint_as_float(v[2 * j]) * inv_l, __uint_as_float(v[2 * j + 1]) * inv_l);
+                    pk[j] = pack_pv<F16>(__uint_as_float(v[2 * j]) * inv_l, __uint_as_float(v[2 * j + 1]) * inv_l);
             }
 #pragma unroll 1
             for (int hb = 0; hb < 2; ++hb) {
@@ -954,7 +976,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     tmem_wait_ld();
 #pragma unroll
                     for (int j = 0; j < 32; ++j)
-                        pk[j] = pack_bf16(__uint_as_float(v[2 * j]) * inv_l,
+                        pk[j] = pack_pv<F16>(__uint_as_float(v[2 * j]) * inv_l,
                                           __uint_as_float(v[2 * j + 1]) * inv_l);
                 }
             }
@@ -973,6 +995,20 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         tc_fence_after();
         tmem_dealloc(tmem, 512);
     }
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+                const __grid_constant__ CUtensorMap tm_o1, const AttnParams p) {
+    attn_fwd_body<false>(tm_q, tm_k, tm_v, tm_o, tm_o1, p);
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+attn_fwd_f16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+                    const __grid_constant__ CUtensorMap tm_o1, const AttnParams p) {
+    attn_fwd_body<true>(tm_q, tm_k, tm_v, tm_o, tm_o1, p);
 }
 
 extern const unsigned kAttnSmemBytes = kSmemBytes;

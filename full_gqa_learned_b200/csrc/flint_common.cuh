@@ -132,6 +132,7 @@ struct PrepParams {
     char* ws;
     int T, nseg, batch, seqlen, window, use_rope, mode;
     int keys_ready;      // 1: the key operand is already in the workspace
+    int ng;              // KV heads in the tensors (4, or a head slice of 1 or 2)
     int f16;             // FP16 policy: q, k, v are FP32 (qf, kf, vf); queries
                          // and values are prepared into the workspace in FP16
     const float* qf;
@@ -149,6 +150,7 @@ struct AttnParams {
     float* lse;
     char* ws;
     int T, nseg, window, use_rope;
+    int ng;              // KV heads in the tensors (4, or a head slice of 1 or 2)
     float rope_theta, eps;
     // > 0: test hook.  The MMA warp of every CTA first waits this many
     // nanoseconds on a barrier nothing arrives on, so the bounded-wait

@@ -221,7 +221,7 @@ __device__ __forceinline__ void load_row16(const float* src, int sub, float* x0,
 template <typename In>
 __device__ __forceinline__ void norm_rope_row(const In* src, __half* dst, const float* w,
                                               float eps, float scale, int sub, bool rope,
-                                              const float* cc, const float* sn) {
+                                              const float* cc, const float* sn, bool store = true) {
     float x0[8], x1[8];
     load_row16(src, sub, x0, x1);
     float ss = 0.f;
@@ -255,8 +255,10 @@ __device__ __forceinline__ void norm_rope_row(const In* src, __half* dst, const 
             hb[e] = __floats2half2_rn(n1[2 * e], n1[2 * e + 1]);
         }
     }
-    *reinterpret_cast<uint4*>(dst + 8 * sub) = oa;
-    *reinterpret_cast<uint4*>(dst + 64 + 8 * sub) = ob;
+    if (store) {
+        *reinterpret_cast<uint4*>(dst + 8 * sub) = oa;
+        *reinterpret_cast<uint4*>(dst + 64 + 8 * sub) = ob;
+    }
 }
 
 __device__ void prepare_tokens(const PrepParams& p) {
@@ -309,13 +311,15 @@ __device__ void prepare_tokens(const PrepParams& p) {
                 sn[e] = __shfl_sync(0xffffffffu, (e & 1) ? s1 : s0, f >> 1);
             }
         }
-        // ---- the 4 key heads (head = lane / 8)
+        // ---- the key heads (head = lane / 8; ng of them, 4 unless the call
+        // covers a head slice).  Every lane takes part in the row's shuffles;
+        // lanes past the slice normalise a valid row and store nothing.
+        const bool kstore = head < p.ng;
+        const size_t krow = ((size_t)t * p.ng + (kstore ? head : 0)) * kHD;
         if (p.f16)
-            norm_rope_row(p.kf + ((size_t)t * kHKV + head) * kHD, kn + ((size_t)t * kHKV + head) * kHD,
-                          s_wk, p.eps, kscale, sub, rope, cc, sn);
+            norm_rope_row(p.kf + krow, kn + krow, s_wk, p.eps, kscale, sub, rope, cc, sn, kstore);
         else if (!p.keys_ready)
-            norm_rope_row(p.k + ((size_t)t * kHKV + head) * kHD, kn + ((size_t)t * kHKV + head) * kHD,
-                          s_wk, p.eps, kscale, sub, rope, cc, sn);
+            norm_rope_row(p.k + krow, kn + krow, s_wk, p.eps, kscale, sub, rope, cc, sn, kstore);
         if (p.f16) {
             // FP16 policy: the values cast to FP16 (4 heads x 128 per token,
             // 16 per lane)
@@ -337,10 +341,11 @@ __device__ void prepare_tokens(const PrepParams& p) {
         if (padded) {
             // ---- padded query token: zero output row, lse = sink
             uint4 z = make_uint4(0, 0, 0, 0);
-            uint4* o = reinterpret_cast<uint4*>(p.out + (size_t)t * kHQ * kHD);
+            const int nh = kGroup * p.ng;                  // query heads in the tensors
+            uint4* o = reinterpret_cast<uint4*>(p.out + (size_t)t * nh * kHD);
 #pragma unroll 4
-            for (int i = lane; i < kHQ * kHD / 8; i += 32) o[i] = z;
-            if (p.lse) p.lse[(size_t)lane * p.T + t] = p.sinks[lane];
+            for (int i = lane; i < nh * kHD / 8; i += 32) o[i] = z;
+            if (p.lse && lane < nh) p.lse[(size_t)lane * p.T + t] = p.sinks[lane];
         } else if (p.f16) {
             // ---- FP16 policy: the 32 query heads normalised and rotated in
             // FP32 and cast to FP16 (x 2^eq) into the workspace, 4 per pass

@@ -21,7 +21,8 @@ flint_status_t run_stages(int stages, const void* q, const void* k, const void* 
                           const int32_t* pos_ids, const int32_t* cu_seqlens, int32_t num_docs,
                           const uint8_t* pad_mask, int32_t batch, int32_t seqlen, int32_t T,
                           int32_t window, int32_t use_rope, float rope_theta, float eps, void* out,
-                          float* lse, void* workspace, size_t workspace_bytes, void* stream);
+                          float* lse, void* workspace, size_t workspace_bytes, void* stream,
+                          int ng = kHKV);
 flint_status_t set_error(flint_status_t s, const char* msg);
 
 namespace {

@@ -162,6 +162,61 @@ FLINT_API flint_status_t flint_attn_attend(const void* q, const void* k, const v
                               void* stream);
 
 /*
+ * The forward on a slice of the KV heads: the unit of work of head-split
+ * context parallelism ("flint" model page, "Parallelism and backends": TE
+ * context parallelism splits the attention heads over the CP group, which
+ * both head counts must divide, so the 4 KV heads permit CP2 or CP4).  Each
+ * rank holds the whole sequence for kv_heads KV heads and their 8 * kv_heads
+ * query heads (after an all-to-all from sequence shards) and runs this call.
+ *
+ *  kv_heads   1, 2 or 4 (4: the same as flint_attn_fwd).
+ *  q          bf16 [T, 8 kv_heads, 128];  k, v  bf16 [T, kv_heads, 128].
+ *  sinks      fp32 [8 kv_heads]: the slice's sinks.
+ *  out        bf16 [T, 8 kv_heads x 128];  lse  fp32 [8 kv_heads, T] or NULL.
+ *  workspace  flint_attn_workspace_bytes(T, n) bytes, as for flint_attn_fwd.
+ *  Every other argument, and the error behaviour, as for flint_attn_fwd.
+ */
+FLINT_API flint_status_t flint_attn_fwd_heads(const void* q, const void* k, const void* v,
+                              const float* q_norm_w, const float* k_norm_w,
+                              const float* sinks, const int32_t* pos_ids,
+                              const int32_t* cu_seqlens, int32_t num_docs,
+                              const uint8_t* pad_mask, int32_t batch, int32_t seqlen,
+                              int32_t T, int32_t kv_heads, int32_t window, int32_t use_rope,
+                              float rope_theta, float eps,
+                              void* out, float* lse,
+                              void* workspace, size_t workspace_bytes,
+                              void* stream);
+
+/*
+ * The FP16 attention-compute policy ("flint" model page, "Numerical
+ * comparison": attention_compute_dtype fp16 casts the normalised, rotated
+ * Q/K/V to FP16 at the attention boundary of an FP32 model and restores FP32
+ * before the output projection; the pages measure it closest to the FP32
+ * reference).  The same operation as flint_attn_fwd on FP32 projections:
+ * q~, k~ are normalised and rotated in FP32 and cast to FP16, v is cast to
+ * FP16, the probabilities multiply v in FP16 with FP32 accumulation, and the
+ * result is written in FP16 (exact in FP32, restoring it is a widening).
+ *
+ *  q          fp32 [T,32,128]; k, v fp32 [T,4,128] (16-byte aligned).
+ *  out        fp16 [T,4096].
+ *  workspace  at least flint_attn_fp16_workspace_bytes(T, n) bytes: the
+ *             forward's workspace plus the FP16 queries (8 KiB per token)
+ *             and values (1 KiB per token).
+ *  Every other argument, and the error behaviour, as for flint_attn_fwd.
+ */
+FLINT_API size_t flint_attn_fp16_workspace_bytes(int32_t T, int32_t num_segments);
+FLINT_API flint_status_t flint_attn_fwd_fp16(const float* q, const float* k, const float* v,
+                              const float* q_norm_w, const float* k_norm_w,
+                              const float* sinks, const int32_t* pos_ids,
+                              const int32_t* cu_seqlens, int32_t num_docs,
+                              const uint8_t* pad_mask, int32_t batch, int32_t seqlen,
+                              int32_t T, int32_t window, int32_t use_rope,
+                              float rope_theta, float eps,
+                              void* out, float* lse,
+                              void* workspace, size_t workspace_bytes,
+                              void* stream);
+
+/*
  * Synchronises `stream`, then returns the status the kernels of the last
  * flint_attn_fwd or flint_attn_decode on `workspace` recorded (FLINT_OK,
  * FLINT_ERR_INVALID_ARG for an ill-formed cu_seqlens or a decode window that

@@ -300,3 +300,20 @@ def call_layer(lib, **kw):
 def test_layer_arguments_rejected_on_host(lib, kw, status):
     assert call_layer(lib, **kw) == status
     assert lib.flint_attn_last_error() != b""
+
+
+def test_fp16_policy_workspace_and_rejection(lib):
+    a = fa.workspace_bytes(4096, 1)
+    b = fa.fp16_workspace_bytes(4096, 1)
+    # plus the FP16 queries and values: 9 KiB per token
+    assert a + 4096 * 9216 <= b < a + 4096 * 9216 + 4096
+    assert fa.fp16_workspace_bytes(-1, 1) == 0
+    args = [A, A, A, A, A, A, None, None, 0, None, 0, 0, 64, 513, 1, 1e4, 1e-6, A, A, A, 0, None]
+    args[20] = fa.workspace_bytes(64, 1)            # enough for the BF16 path, not for this one
+    assert lib.flint_attn_fwd_fp16(*args) == 5
+    args[20] = 1 << 40
+    args[0] = A + 8                                 # misaligned q
+    assert lib.flint_attn_fwd_fp16(*args) == 1
+    args[0] = A
+    args[12] = 0                                    # T = 0: no-op
+    assert lib.flint_attn_fwd_fp16(*args) == 0

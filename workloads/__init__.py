@@ -300,6 +300,20 @@ def make_small(T, seed, *, window=0, use_rope=False, cu_seqlens=None,
                     pad_mask=pad_mask, window=window, use_rope=use_rope, seed=seed)
 
 
+def make_small_f32(T, seed, *, window=0, use_rope=False, cu_seqlens=None, pad_mask=None,
+                   name="small_f32") -> Workload:
+    """Seeded case with FP32 projections (an FP32 model body, as the FP16
+    attention-compute policy takes them): q, k, v float32 N(0,1), not
+    rounded; the rest as make_small."""
+    w = make_small(T, seed, window=window, use_rope=use_rope, cu_seqlens=cu_seqlens,
+                   pad_mask=pad_mask, name=name)
+    rng = np.random.default_rng(seed + 500)
+    w.q = _normal(rng, (T, HQ, D))
+    w.k = _normal(rng, (T, HKV, D))
+    w.v = _normal(rng, (T, HKV, D))
+    return w
+
+
 @dataclasses.dataclass
 class DecodeWorkload:
     """One decode step for B sequences: the new token's projections and a
