@@ -26,6 +26,11 @@ __global__ void attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q,
                                 const __grid_constant__ CUtensorMap tm_v,
                                 const __grid_constant__ CUtensorMap tm_o,
                                 const __grid_constant__ CUtensorMap tm_o1, const AttnParams p);
+__global__ void attn_fwd_qprep_kernel(const __grid_constant__ CUtensorMap tm_q,
+                                      const __grid_constant__ CUtensorMap tm_k,
+                                      const __grid_constant__ CUtensorMap tm_v,
+                                      const __grid_constant__ CUtensorMap tm_o,
+                                      const __grid_constant__ CUtensorMap tm_o1, const AttnParams p);
 __global__ void attn_fwd_f16_kernel(const __grid_constant__ CUtensorMap tm_q,
                                     const __grid_constant__ CUtensorMap tm_k,
                                     const __grid_constant__ CUtensorMap tm_v,
@@ -90,6 +95,9 @@ flint_status_t device_setup(int* sms) {
                                  (int)kAttnSmemBytes);
         if (e == cudaSuccess)
             e = cudaFuncSetAttribute(attn_fwd_f16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)kAttnSmemBytes);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(attn_fwd_qprep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      (int)kAttnSmemBytes);
         if (e != cudaSuccess)
             return fail(FLINT_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
@@ -214,6 +222,10 @@ flint_status_t run_stages(int stages, const void* q, const void* k, const void* 
         (cu_seqlens && !aligned(cu_seqlens, 4)))
         return fail(FLINT_ERR_INVALID_ARG, "misaligned 32-bit array");
     const bool f16 = (stages & kStageF16) != 0;
+    // Queries: prepared on tile load by the attention kernel on full layers;
+    // on sliding layers (short units, measured faster) by the preparation
+    // kernel into the output rows, unless the caller asks for tile load
+    const bool qprep = !f16 && window > 0 && !(stages & kStageTileQ);
     const WsLayout L = ws_layout(T, nseg < 1 ? 1 : nseg);
     const size_t need = f16 ? L.total_f16 : L.total;
     if (!workspace || !aligned(workspace, 256))
@@ -235,7 +247,12 @@ flint_status_t run_stages(int stages, const void* q, const void* k, const void* 
     // kernel normalised and rotated into the workspace)
     const CUtensorMapDataType t16 = f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
     const int nh = kGroup * ng;      // query heads in the tensors
-    st = make_map(enc, &tm_q, t16, f16 ? static_cast<const void*>(ws + L.qn) : q, nh, T, kGroup, kTokPerTile);
+    if (f16)
+        st = make_map(enc, &tm_q, t16, ws + L.qn, nh, T, kGroup, kTokPerTile);
+    else if (qprep)
+        st = make_map(enc, &tm_q, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, out, nh, T, kGroup, kTokPerTile);
+    else
+        st = make_map(enc, &tm_q, t16, q, nh, T, kGroup, kTokPerTile);
     if (st != FLINT_OK) return st;
     st = make_map(enc, &tm_k, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, ws + L.kn, ng, T, 1, kKeyChunk);
     if (st != FLINT_OK) return st;
@@ -271,6 +288,7 @@ flint_status_t run_stages(int stages, const void* q, const void* k, const void* 
     pp.mode = mode;
     pp.keys_ready = (stages & kStageKeysReady) ? 1 : 0;
     pp.ng = ng;
+    pp.qprep = qprep ? 1 : 0;
     pp.f16 = f16 ? 1 : 0;
     pp.qf = f16 ? static_cast<const float*>(q) : nullptr;
     pp.kf = f16 ? static_cast<const float*>(k) : nullptr;
@@ -323,11 +341,14 @@ flint_status_t run_stages(int stages, const void* q, const void* k, const void* 
         attr[0].val.programmaticStreamSerializationAllowed = 1;
         cfg.attrs = attr;
         cfg.numAttrs = 1;
-        e = f16 ? cudaLaunchKernelEx(&cfg, attn_fwd_f16_kernel, tm_q, tm_k, tm_v, tm_o, tm_o1, ap)
-                : cudaLaunchKernelEx(&cfg, attn_fwd_kernel, tm_q, tm_k, tm_v, tm_o, tm_o1, ap);
+        e = f16     ? cudaLaunchKernelEx(&cfg, attn_fwd_f16_kernel, tm_q, tm_k, tm_v, tm_o, tm_o1, ap)
+            : qprep ? cudaLaunchKernelEx(&cfg, attn_fwd_qprep_kernel, tm_q, tm_k, tm_v, tm_o, tm_o1, ap)
+                    : cudaLaunchKernelEx(&cfg, attn_fwd_kernel, tm_q, tm_k, tm_v, tm_o, tm_o1, ap);
     } else {
         if (f16)
             attn_fwd_f16_kernel<<<grid, kAttnThreads, kAttnSmemBytes, s>>>(tm_q, tm_k, tm_v, tm_o, tm_o1, ap);
+        else if (qprep)
+            attn_fwd_qprep_kernel<<<grid, kAttnThreads, kAttnSmemBytes, s>>>(tm_q, tm_k, tm_v, tm_o, tm_o1, ap);
         else
             attn_fwd_kernel<<<grid, kAttnThreads, kAttnSmemBytes, s>>>(tm_q, tm_k, tm_v, tm_o, tm_o1, ap);
         e = cudaGetLastError();
@@ -478,7 +499,7 @@ flint_status_t flint_attn_layer_fwd(const void* x, const void* w_qkv, const void
     }
     // 1. plan and padded rows (every other argument is validated here, before
     //    any launch); the keys come from the projection's epilogue
-    st = run_stages(kStagePrepare | kStageKeysReady, q, k, v, q_norm_w, k_norm_w, sinks, pos_ids,
+    st = run_stages(kStagePrepare | kStageKeysReady | kStageTileQ, q, k, v, q_norm_w, k_norm_w, sinks, pos_ids,
                     cu_seqlens, num_docs, pad_mask, batch, seqlen, T, window, use_rope, rope_theta, eps,
                     attn_out, lse, workspace, workspace_bytes, stream);
     if (st != FLINT_OK || T == 0) return st;
@@ -495,7 +516,7 @@ flint_status_t flint_attn_layer_fwd(const void* x, const void* w_qkv, const void
                                 status, s);
     if (st != FLINT_OK) return st;
     // 3. attention
-    st = run_stages(kStageAttend, q, k, v, q_norm_w, k_norm_w, sinks, pos_ids, cu_seqlens, num_docs,
+    st = run_stages(kStageAttend | kStageTileQ, q, k, v, q_norm_w, k_norm_w, sinks, pos_ids, cu_seqlens, num_docs,
                     pad_mask, batch, seqlen, T, window, use_rope, rope_theta, eps, attn_out, lse, workspace,
                     workspace_bytes, stream);
     if (st != FLINT_OK) return st;

@@ -196,12 +196,16 @@ __device__ __forceinline__ uint32_t pack_pv(float lo, float hi) {
     }
 }
 
-// The kernel body.  F16: the FP16 attention-compute policy ("flint" model
-// page, "Numerical comparison": normalised, rotated Q/K/V cast to FP16 for
-// the attention): the queries arrive normalised and rotated in FP16 from the
-// preparation kernel, values are FP16, P and the output are FP16, and the
-// softmax keeps its exact running max (P stays within FP16's normal range).
-template <bool F16>
+// The kernel body.
+// QPREP: the queries arrive normalised and rotated in FP16 from the
+//   preparation kernel instead of being prepared on tile load.  Sliding
+//   layers use it: their units are 5 chunks long, too short to hide the
+//   prologue between a unit's last chunk and its epilogue.
+// F16 (implies QPREP): the FP16 attention-compute policy ("flint" model page,
+//   "Numerical comparison": normalised, rotated Q/K/V cast to FP16 for the
+//   attention): values are FP16, P and the output are FP16, and the softmax
+//   keeps its exact running max (P stays within FP16's normal range).
+template <bool QPREP, bool F16>
 __device__ __forceinline__ void attn_fwd_body(const CUtensorMap& tm_q, const CUtensorMap& tm_k,
                                               const CUtensorMap& tm_v, const CUtensorMap& tm_o,
                                               const CUtensorMap& tm_o1, const AttnParams& p) {
@@ -303,9 +307,8 @@ __device__ __forceinline__ void attn_fwd_body(const CUtensorMap& tm_q, const CUt
         if (lane == 0) {
             uint32_t sslot = 0, sph = 0, qph = 0, kst = 0, kph = 0, vst = 0, vph = 0;
             uint32_t narm_q = 0, narm_k = 0, narm_v = 0;   // loads armed so far
-            // Units are taken one ahead: while unit u streams, the raw query
-            // tiles and the first key/value chunk of the next unit are
-            // prefetched into L2, so its query prologue does not wait on HBM.
+            // Units are taken one ahead of the loads (the next unit is known
+            // while the current one streams).
             int u = atomicAdd(&hdr->counter, 1);
             if (u >= n_units) u = -1;
             for (;;) {
@@ -316,19 +319,6 @@ __device__ __forceinline__ void attn_fwd_body(const CUtensorMap& tm_q, const CUt
                 if (u < 0) break;
                 int un = atomicAdd(&hdr->counter, 1);
                 if (un >= n_units) un = -1;
-                if (un >= 0) {
-                    const int4 nx = items[un / p.ng];
-                    const int gn = un % p.ng;
-                    const int kbn = p.window > 0 ? max(nx.z, nx.x - p.window + 1) : nx.z;
-                    for (int t = 0; t < 2; ++t) {
-                        tma_prefetch_3d(&tm_q, 0, kGroup * gn, nx.x + kTokPerTile * t);
-                        tma_prefetch_3d(&tm_q, 64, kGroup * gn, nx.x + kTokPerTile * t);
-                    }
-                    tma_prefetch_3d(&tm_k, 0, gn, kbn);
-                    tma_prefetch_3d(&tm_k, 64, gn, kbn);
-                    tma_prefetch_3d(&tm_v, 0, gn, kbn);
-                    tma_prefetch_3d(&tm_v, 64, gn, kbn);
-                }
                 const int4 it = items[u / p.ng];
                 const int g = u % p.ng;
                 const int q0 = it.x, nq = it.y, ds = it.z, nch = it.w;
@@ -539,7 +529,7 @@ __device__ __forceinline__ void attn_fwd_body(const CUtensorMap& tm_q, const CUt
             if (!__all_sync(0xffffffffu, mbar_wait(bar(B_Q_FULL + t), qph, abort_flag, status)))
                 return false;
             qph ^= 1;
-            if constexpr (F16) {
+            if constexpr (QPREP) {
                 // the preparation kernel already normalised and rotated them
                 mbar_arrive(bar(B_Q_READY + t));
                 return true;
@@ -1001,14 +991,21 @@ __global__ void __launch_bounds__(kThreads, 1)
 attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
                 const __grid_constant__ CUtensorMap tm_o1, const AttnParams p) {
-    attn_fwd_body<false>(tm_q, tm_k, tm_v, tm_o, tm_o1, p);
+    attn_fwd_body<false, false>(tm_q, tm_k, tm_v, tm_o, tm_o1, p);
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+attn_fwd_qprep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                      const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+                      const __grid_constant__ CUtensorMap tm_o1, const AttnParams p) {
+    attn_fwd_body<true, false>(tm_q, tm_k, tm_v, tm_o, tm_o1, p);
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
 attn_fwd_f16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
                     const __grid_constant__ CUtensorMap tm_o1, const AttnParams p) {
-    attn_fwd_body<true>(tm_q, tm_k, tm_v, tm_o, tm_o1, p);
+    attn_fwd_body<true, true>(tm_q, tm_k, tm_v, tm_o, tm_o1, p);
 }
 
 extern const unsigned kAttnSmemBytes = kSmemBytes;

@@ -114,7 +114,8 @@ __device__ __forceinline__ void rope_cos_sin(int pos, double inv_freq, float* c,
 enum Stage : int {
     kStagePrepare = 1, kStageAttend = 2, kStageBoth = 3,
     kStageKeysReady = 4,  // with kStagePrepare: the keys were prepared by the projection GEMM
-    kStageF16 = 8         // FP16 attention-compute policy: FP32 q/k/v in, FP16 out
+    kStageF16 = 8,        // FP16 attention-compute policy: FP32 q/k/v in, FP16 out
+    kStageTileQ = 16      // prepare the queries on tile load even on sliding layers
 };
 
 // Kernel parameter blocks (passed by value).
@@ -133,6 +134,9 @@ struct PrepParams {
     int T, nseg, batch, seqlen, window, use_rope, mode;
     int keys_ready;      // 1: the key operand is already in the workspace
     int ng;              // KV heads in the tensors (4, or a head slice of 1 or 2)
+    int qprep;           // 1: normalise and rotate the queries here, FP16 into
+                         // the output rows of their token (the attention kernel
+                         // reads them back before writing the result there)
     int f16;             // FP16 policy: q, k, v are FP32 (qf, kf, vf); queries
                          // and values are prepared into the workspace in FP16
     const float* qf;

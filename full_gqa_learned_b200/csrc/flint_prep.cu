@@ -292,7 +292,7 @@ __device__ void prepare_tokens(const PrepParams& p) {
         // ---- the lane's 8 (cos, sin) pairs f = 8*sub + e at the token's
         // document-local position, shared by its 4 key heads
         float cc[8], sn[8];
-        if (rope && (p.f16 || !p.keys_ready)) {
+        if (rope && (p.f16 || p.qprep || !p.keys_ready)) {
             int pos;
             if (p.pos_ids) pos = p.pos_ids[t];
             else if (p.mode == kMaskThd) pos = t - (t < s_thd_end ? thd_segment_start(p.cu_seqlens, p.nseg, t) : s_thd_end);
@@ -355,6 +355,22 @@ __device__ void prepare_tokens(const PrepParams& p) {
             for (int hq = 0; hq < kHQ / kHKV; ++hq) {
                 const int hh = kHKV * hq + head;
                 norm_rope_row(qrow + hh * kHD, qdst + hh * kHD, s_wq, p.eps, s_qscale, sub, rope, cc, sn);
+            }
+        } else if (p.qprep) {
+            // ---- the query heads (8 ng of them) normalised and rotated into
+            // the output rows of the token as FP16 (x 2^eq), 4 per pass: the
+            // attention tile that owns the rows reads them back as its Q
+            // operand and writes its result over them.  Each head row is read
+            // before it is written, so out may be q itself.
+            const int nh = kGroup * p.ng;
+            const __nv_bfloat16* qrow = p.q + (size_t)t * nh * kHD;
+            __half* qdst = reinterpret_cast<__half*>(p.out + (size_t)t * nh * kHD);
+#pragma unroll 2
+            for (int hq = 0; hq < kGroup; ++hq) {
+                const int hh = kHKV * hq + head;
+                const bool qstore = hh < nh;
+                const int hs = qstore ? hh : 0;
+                norm_rope_row(qrow + hs * kHD, qdst + hs * kHD, s_wq, p.eps, s_qscale, sub, rope, cc, sn, qstore);
             }
         }
     }

@@ -115,13 +115,6 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const void* desc, uint
         : "memory");
 }
 
-// Prefetch of a 3-D tile into L2 (no shared memory, no completion).
-__device__ __forceinline__ void tma_prefetch_3d(const void* desc, int c0, int c1, int c2) {
-    asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(desc), "r"(c0),
-                 "r"(c1), "r"(c2)
-                 : "memory");
-}
-
 // 2-D tiled load into shared memory, completion counted on `bar`.
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const void* desc, uint32_t bar, int c0, int c1) {
     asm volatile(

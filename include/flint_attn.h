@@ -107,9 +107,14 @@ FLINT_API size_t flint_attn_workspace_bytes(int32_t T, int32_t num_segments);
  *  rope_theta RoPE base (> 1), e.g. 10000.
  *  eps        RMSNorm epsilon (> 0), 1e-6 for Flint.
  *  out        bf16 [T,4096]: out[t, h*128 + c], the o_proj input.  Rows of
- *             padded tokens are written as +0.0.  out may be q itself (each
- *             query row is read before the result is written over it); it
- *             must not overlap k, v, lse or the workspace.
+ *             padded tokens are written as +0.0.  On sliding layers
+ *             (window > 0) the call also uses out as scratch: the preparation
+ *             kernel leaves each valid token's normalised FP16 queries in its
+ *             rows and the attention kernel overwrites them with the result;
+ *             on full layers the attention kernel prepares the queries on
+ *             tile load.  Either way out may be q itself (each query row is
+ *             read before anything is written over it); it must not overlap
+ *             k, v, lse or the workspace.
  *  lse        fp32 [32,T] natural-log sum of exponentials including the sink
  *             (lse[h*T + t]); padded tokens get sinks[h].  May be NULL.
  *  workspace  device buffer of at least flint_attn_workspace_bytes(T, n)
@@ -133,12 +138,13 @@ FLINT_API flint_status_t flint_attn_fwd(const void* q, const void* k, const void
 /*
  * The two stages flint_attn_fwd enqueues, exposed so a caller (or a profiler)
  * can time them apart.  flint_attn_prepare runs the preparation kernel: the
- * work plan, the normalised/rotated FP16 keys in the workspace and the
- * outputs of padded query tokens.  flint_attn_attend runs the attention
- * kernel (which normalises and rotates the queries itself) on a workspace
- * that flint_attn_prepare filled with the same arguments; calling it with
- * other arguments is undefined.  Both take the arguments of flint_attn_fwd
- * and validate them the same way.
+ * work plan, the normalised/rotated FP16 keys in the workspace, the outputs
+ * of padded query tokens and, on sliding layers, the normalised/rotated FP16
+ * queries in the rows of out (intermediate values, not a result).
+ * flint_attn_attend runs the attention kernel on a workspace and an out that
+ * flint_attn_prepare filled with the same arguments; calling it with other
+ * arguments, or after out was modified in between, is undefined.  Both take
+ * the arguments of flint_attn_fwd and validate them the same way.
  */
 FLINT_API flint_status_t flint_attn_prepare(const void* q, const void* k, const void* v,
                               const float* q_norm_w, const float* k_norm_w,
