@@ -59,8 +59,11 @@ def recorded_traffic(workload, profiles_dir=None):
     sources changed since it was taken."""
     if profiles_dir is None:
         profiles_dir = os.path.join(os.path.dirname(os.path.abspath(__file__)), "profiles")
-    path = os.path.join(profiles_dir, "attn_fwd_kernel_%s_ncu.md" % workload)
-    if not os.path.exists(path):
+    for name in ("attn_fwd_kernel", "attn_fwd_qprep_kernel"):
+        path = os.path.join(profiles_dir, "%s_%s_ncu.md" % (name, workload))
+        if os.path.exists(path):
+            break
+    else:
         return None
     vals = {}
     with open(path) as f:
@@ -1026,7 +1029,8 @@ def main():
                       frac=round(attn_tflops / peak, 4), kernel_frac=round(attn_tflops / peak, 4),
                       layer_frac=round(value / world / peak, 4),
                       traffic=args.traffic if args.traffic is not None else recorded_traffic(w.name),
-                      kernel="flint::attn_fwd_kernel", peak_source="%s bf16_tflops (burst)" % src,
+                      kernel=("flint::attn_fwd_qprep_kernel" if w.window > 0 else "flint::attn_fwd_kernel"),
+                      peak_source="%s bf16_tflops (burst)" % src,
                       flops_per_launch=flops,
                       kernel_ms=round(r["attn_avg"], 5), prep_kernel_ms=round(r["prep_avg"], 5)),
         e2e=dict(value=round(whole_job_tflops(flops, 1, world, r["e2e_ms"]), 3), unit=UNIT,
