@@ -45,7 +45,7 @@ constexpr int kBwdPartQ = kHD + kHQ;        // per-CTA partial: dq_norm_w[128], 
 constexpr int kBwdSegThreads = 1024;
 
 struct BwdLayout {
-    size_t seg_lo, seg_hi, delta, qh, kh, part_q, part_k, total;
+    size_t seg_lo, seg_hi, flags, delta, qh, kh, part_q, part_k, total;
 };
 
 // Header: status word (offset 0), the tensor-core kernels' unit counters
@@ -55,6 +55,7 @@ inline BwdLayout bwd_layout(int T) {
     size_t o = 256;
     L.seg_lo = o; o = ws_align(o + sizeof(int) * (size_t)T, 256);
     L.seg_hi = o; o = ws_align(o + sizeof(int) * (size_t)T, 256);
+    L.flags = o;  o = ws_align(o + sizeof(int) * (size_t)((T + 127) / 128) * kHKV, 256);
     L.delta = o;  o = ws_align(o + sizeof(float) * (size_t)T * kHQ, 256);
     L.qh = o;     o = ws_align(o + 2 * (size_t)T * kHQ * kHD, 1024);
     L.kh = o;     o = ws_align(o + 2 * (size_t)T * kHKV * kHD, 256);
@@ -350,7 +351,7 @@ flint_status_t set_error(flint_status_t s, const char* msg);
 flint_status_t launch_bwd_tc(const void* qh, const void* kh, const void* v, const void* dout,
                              const float* q_norm_w, const float* k_norm_w, const float* lse,
                              const float* delta, const int* seg_lo, const int* seg_hi, float* dq, float* dk,
-                             float* dv, int* status, int* counters, int T, int window, int sms,
+                             float* dv, int* status, int* counters, int* flags, int T, int window, int sms,
                              cudaStream_t s);
 
 size_t bwd_workspace_bytes(int T) { return bwd_layout(T).total; }
@@ -420,6 +421,7 @@ flint_status_t run_bwd(const void* q, const void* k, const void* v, const float*
 
     cudaError_t e = cudaMemsetAsync(ws, 0, 256, s);
     if (e == cudaSuccess) e = cudaMemsetAsync(bp.seg_lo, 0xff, sizeof(int) * (size_t)T, s);
+    if (e == cudaSuccess) e = cudaMemsetAsync(ws + L.flags, 0, sizeof(int) * (size_t)((T + 127) / 128) * kHKV, s);
     if (e != cudaSuccess) return set_error(FLINT_ERR_CUDA, "backward: workspace reset failed");
     if (nseg > 0) {
         bwd_segments_kernel<<<nseg, kBwdSegThreads, 0, s>>>(bp);
@@ -433,8 +435,8 @@ flint_status_t run_bwd(const void* q, const void* k, const void* v, const float*
     e = cudaGetLastError();
     if (e != cudaSuccess) return set_error(FLINT_ERR_CUDA, "backward: prep launch failed");
     flint_status_t st = launch_bwd_tc(bp.qh, bp.kh, v, dout, q_norm_w, k_norm_w, lse, bp.delta, bp.seg_lo,
-                                      bp.seg_hi, dq, dk, dv, bp.status, reinterpret_cast<int*>(ws + 16), T,
-                                      window, sms, s);
+                                      bp.seg_hi, dq, dk, dv, bp.status, reinterpret_cast<int*>(ws + 16),
+                                      reinterpret_cast<int*>(ws + L.flags), T, window, sms, s);
     if (st != FLINT_OK) return st;
     bwd_adjoint_kernel<<<grid_a, kBwdThreads, 0, s>>>(bp);
     e = cudaGetLastError();

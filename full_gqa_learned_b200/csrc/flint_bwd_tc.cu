@@ -26,6 +26,9 @@
 //   dkv kernel, per key tile, over the query tiles that see it:
 //     S^T = Kh Qh^T, dP^T = V dO^T  (SS)  ->  P^T, dS^T (threads)  ->
 //     dV += P^T dO, dK += dS^T Qh  (TS)
+//     On short sequences a key tile's query tiles are cut into pieces that
+//     different CTAs run; each piece adds its dK, dV to the sum of the
+//     pieces before it, in piece order, behind a per-tile flag.
 //     TMEM: S^T 0..127 (P^T over its first 64), dP^T 128..255 (dS^T over its
 //     first 64), dV 256..383, dK 384..511
 // Each CTA (persistent, 256 threads): warp 0 scheduler + TMA producer, warp 1
@@ -71,13 +74,17 @@ struct BwdTcParams {
     float* dv;               // [T, 4, 128]: dv on exit (valid rows)
     int* status;
     int* counter;            // dynamic unit counter (zeroed before the launch)
+    int* flags;              // dkv: [key tile][KV head] pieces summed so far (zeroed)
     int T, window;
+    int qp;                  // dkv: query tiles per piece of a key tile's range
+    int np;                  // dkv: pieces per key tile at most
 };
 
 struct BtMisc {
     int sched[2][4];         // unit, and its range (start, count)
     uint32_t tmem_base;
     int abort_flag;
+    int fix_ok;              // dkv: the previous piece's flag was seen
     float logit_scale;       // log2(e)/sqrt(128) 2^-(eq+ek)
     float dq_scale;          // 2^-ek / sqrt(128)
     float dk_scale;          // 2^-eq / sqrt(128)
@@ -88,7 +95,8 @@ enum : uint32_t {
     T_A_FULL = 4, T_A_EMPTY = 6,         // dq: K stages; dkv: (Q, dO) stages
     T_B_FULL = 8, T_B_EMPTY = 10,        // dq: V stages; dkv: (K, V) tile (index 0)
     T_C_FULL = 12, T_C_EMPTY = 13,       // dq: (Q, dO) tile
-    T_S_FULL = 14, T_DS_READY = 15, T_ACC_FULL = 16, T_DRAIN = 17
+    T_S_FULL = 14, T_DS_READY = 15, T_ACC_FULL = 16, T_DRAIN = 17,
+    T_GO = 18, T_FIX = 19                // dkv: piece fix-up hand-offs
 };
 
 __device__ __forceinline__ float bt_ex2(float x) {
@@ -428,7 +436,7 @@ bwd_dkv_tc_kernel(const __grid_constant__ CUtensorMap tm_qh, const __grid_consta
     int* status = p.status;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int n_tiles = (p.T + 127) / 128;
-    const int n_units = n_tiles * kHKV;
+    const int n_units = n_tiles * kHKV * p.np;
 
     if (tid == 0) {
         for (int s = 0; s < 2; ++s) {
@@ -443,6 +451,8 @@ bwd_dkv_tc_kernel(const __grid_constant__ CUtensorMap tm_qh, const __grid_consta
         mbar_init(bar(T_DS_READY), 128);
         mbar_init(bar(T_ACC_FULL), 1);
         mbar_init(bar(T_DRAIN), 1);
+        mbar_init(bar(T_GO), 1);
+        mbar_init(bar(T_FIX), 128);
         misc->abort_flag = 0;
         fence_mbar_init();
     }
@@ -459,31 +469,48 @@ bwd_dkv_tc_kernel(const __grid_constant__ CUtensorMap tm_qh, const __grid_consta
     if (warp == 0) {
         // ------------------------------------------------ scheduler + producer (whole warp)
         uint32_t sslot = 0, sph = 0, kvph = 0, st = 0, ph = 0, narm_kv = 0, narm = 0;
+        int last_kt = -1, kqb = 0, kqe = 0;           // query range of the last key tile seen
         bool ok = true;
         for (;;) {
-            int u = 0, qb = 0, qe = 0;
+            // next non-empty unit: piece pc of key tile kt for KV head g,
+            // u = (kt * np + pc) * 4 + g, query tiles [pc qp, (pc+1) qp) of the
+            // tile's range
+            int u = -1, qb = 0, nqt = 0, pc = 0;
             if (lane == 0) {
-                u = atomicAdd(p.counter, 1);
-                if (u >= n_units) u = -1;
-                else k_tile_queries(p, (u / kHKV) * 128, &qb, &qe);
+                for (;;) {
+                    u = atomicAdd(p.counter, 1);
+                    if (u >= n_units) { u = -1; break; }
+                    const int kt = u / (kHKV * p.np);
+                    pc = (u / kHKV) % p.np;
+                    if (kt != last_kt) {
+                        k_tile_queries(p, kt * 128, &kqb, &kqe);
+                        last_kt = kt;
+                    }
+                    const int ntot = (kqe - kqb + kTokPerTile - 1) / kTokPerTile;
+                    if (pc * p.qp < ntot) {
+                        qb = kqb + kTokPerTile * p.qp * pc;
+                        nqt = min(p.qp, ntot - pc * p.qp);
+                        break;
+                    }
+                }
             }
             u = __shfl_sync(0xffffffffu, u, 0);
             qb = __shfl_sync(0xffffffffu, qb, 0);
-            qe = __shfl_sync(0xffffffffu, qe, 0);
-            const int nqt = (qe - qb + kTokPerTile - 1) / kTokPerTile;
+            nqt = __shfl_sync(0xffffffffu, nqt, 0);
+            pc = __shfl_sync(0xffffffffu, pc, 0);
             if (!__all_sync(0xffffffffu, mbar_wait(bar(T_SCHED_EMPTY + sslot), sph ^ 1, abort_flag, status)))
                 break;
             if (lane == 0) {
                 misc->sched[sslot][0] = u;
                 misc->sched[sslot][1] = qb;
                 misc->sched[sslot][2] = nqt;
+                misc->sched[sslot][3] = pc;
                 mbar_arrive(bar(T_SCHED_FULL + sslot));
             }
             __syncwarp();
             sslot ^= 1; if (sslot == 0) sph ^= 1;
             if (u < 0) break;
-            if (nqt == 0) continue;
-            const int g = u % kHKV, j0 = (u / kHKV) * 128;
+            const int g = u % kHKV, j0 = (u / (kHKV * p.np)) * 128;
             ok = __all_sync(0xffffffffu, mbar_wait(bar(T_B_EMPTY), kvph ^ 1, abort_flag, status));
             if (!ok) break;
             if (lane == 0) {
@@ -607,17 +634,18 @@ bwd_dkv_tc_kernel(const __grid_constant__ CUtensorMap tm_qh, const __grid_consta
         const uint32_t lb = (uint32_t)(warp & 3) * 32u;
         const uint32_t t_s = tmem + (lb << 16), t_dp = t_s + 128, t_dv = t_s + 256, t_dk = t_s + 384;
         const float C = misc->logit_scale, dks = misc->dk_scale;
-        uint32_t sslot = 0, sph = 0, s_ph = 0, aph = 0, st = 0, ph = 0;
+        uint32_t sslot = 0, sph = 0, s_ph = 0, aph = 0, st = 0, ph = 0, gph = 0, fph = 0;
         for (;;) {
             if (!__all_sync(0xffffffffu, mbar_wait(bar(T_SCHED_FULL + sslot), sph, abort_flag, status))) break;
             const int u = misc->sched[sslot][0];
             const int qb = misc->sched[sslot][1], nqt = misc->sched[sslot][2];
+            const int pc = misc->sched[sslot][3];
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(T_SCHED_EMPTY + sslot));
             sslot ^= 1; if (sslot == 0) sph ^= 1;
             if (u < 0) break;
             if (nqt == 0) continue;
-            const int g = u % kHKV, j = (u / kHKV) * 128 + r;
+            const int g = u % kHKV, kt = u / (kHKV * p.np), j = kt * 128 + r;
             const bool valid = j < p.T && p.seg_lo[j] >= 0;
             int hi = 0;
             if (valid) hi = p.window > 0 ? min(p.seg_hi[j], j + p.window) : p.seg_hi[j];
@@ -671,6 +699,22 @@ bwd_dkv_tc_kernel(const __grid_constant__ CUtensorMap tm_qh, const __grid_consta
             if (!alive) break;
             if (!__all_sync(0xffffffffu, mbar_wait(bar(T_ACC_FULL), aph, abort_flag, status))) break;
             aph ^= 1;
+            // Pieces of one key tile and head are summed in piece order, so
+            // the result does not depend on which CTA ran which piece: piece
+            // pc > 0 waits until piece pc - 1 has stored, then adds to it.
+            // Every piece was dispensed after its predecessor (lower unit
+            // index) to a CTA that is running, so the wait ends.
+            int* flag = p.flags + kt * kHKV + g;
+            if (pc > 0) {
+                if (tid == 128) {
+                    misc->fix_ok = flag_wait_geq(flag, pc, abort_flag, status) ? 1 : 0;
+                    mbar_arrive(bar(T_GO));
+                }
+                __syncwarp();
+                if (!__all_sync(0xffffffffu, mbar_wait(bar(T_GO), gph, abort_flag, status))) break;
+                gph ^= 1;
+                if (!misc->fix_ok) break;
+            }
             tc_fence_after();
             float* dkd = p.dk + ((size_t)j * kHKV + g) * kHD;
             float* dvd = p.dv + ((size_t)j * kHKV + g) * kHD;
@@ -683,16 +727,28 @@ bwd_dkv_tc_kernel(const __grid_constant__ CUtensorMap tm_qh, const __grid_consta
                 if (valid) {
 #pragma unroll
                     for (int e = 0; e < 32; e += 4) {
-                        *reinterpret_cast<float4*>(dkd + 32 * b + e) =
-                            make_float4(__uint_as_float(a[e]) * dks, __uint_as_float(a[e + 1]) * dks,
-                                        __uint_as_float(a[e + 2]) * dks, __uint_as_float(a[e + 3]) * dks);
-                        *reinterpret_cast<float4*>(dvd + 32 * b + e) =
-                            make_float4(__uint_as_float(c[e]), __uint_as_float(c[e + 1]),
-                                        __uint_as_float(c[e + 2]), __uint_as_float(c[e + 3]));
+                        float4 k4 = make_float4(__uint_as_float(a[e]) * dks, __uint_as_float(a[e + 1]) * dks,
+                                                __uint_as_float(a[e + 2]) * dks, __uint_as_float(a[e + 3]) * dks);
+                        float4 v4 = make_float4(__uint_as_float(c[e]), __uint_as_float(c[e + 1]),
+                                                __uint_as_float(c[e + 2]), __uint_as_float(c[e + 3]));
+                        if (pc > 0) {
+                            // the earlier pieces' sum, from L2 (written by another SM)
+                            const float4 k0 = __ldcg(reinterpret_cast<const float4*>(dkd + 32 * b + e));
+                            const float4 v0 = __ldcg(reinterpret_cast<const float4*>(dvd + 32 * b + e));
+                            k4 = make_float4(k0.x + k4.x, k0.y + k4.y, k0.z + k4.z, k0.w + k4.w);
+                            v4 = make_float4(v0.x + v4.x, v0.y + v4.y, v0.z + v4.z, v0.w + v4.w);
+                        }
+                        __stcg(reinterpret_cast<float4*>(dkd + 32 * b + e), k4);
+                        __stcg(reinterpret_cast<float4*>(dvd + 32 * b + e), v4);
                     }
                 }
             }
             tc_fence_before();
+            // this piece's rows are stored: publish pc + 1 for the next piece
+            mbar_arrive(bar(T_FIX));
+            if (tid == 128 && mbar_wait(bar(T_FIX), fph, abort_flag, status)) flag_release(flag, pc + 1);
+            __syncwarp();
+            fph ^= 1;
         }
     }
     tc_fence_before();
@@ -726,12 +782,37 @@ bool g_bt_attr[64] = {false};
 
 }  // namespace
 
+// Pieces of a key tile's query range for the dk/dv kernel: on short
+// sequences the key tiles (4 per 128 tokens) are too few to balance over the
+// SMs, and on a causal sequence the first tile sees every query while the
+// last sees 128, so each tile's range is cut into up to `np` pieces of `qp`
+// query tiles, about 4 units per SM.  Long sequences keep one piece per tile.
+void bwd_pieces(int T, int window, int sms, int* qp, int* np) {
+    const int n_kt = (T + 127) / 128;
+    const int units = n_kt * kHKV;
+    // query tiles a key tile can see, at most (its range starts at its
+    // first valid key, not on a tile boundary)
+    int nqt_max = (T + kTokPerTile - 1) / kTokPerTile + 1;
+    if (window > 0) nqt_max = min(nqt_max, (128 + window + kTokPerTile - 2) / kTokPerTile + 1);
+    const int target = (4 * sms + units - 1) / (units > 0 ? units : 1);
+    if (target <= 1) {
+        *qp = nqt_max;
+        *np = 1;
+        return;
+    }
+    int q = (nqt_max + target - 1) / target;
+    if (q < 8) q = 8;
+    *qp = q;
+    *np = (nqt_max + q - 1) / q;
+}
+
 // Enqueues the two tensor-core kernels.  qh [T,32,128] and kh [T,4,128] are
-// the FP16 scaled operands (2^eq q~, 2^ek k~); counters: two zeroed ints.
+// the FP16 scaled operands (2^eq q~, 2^ek k~); counters: two zeroed ints;
+// flags: ceil(T/128) x 4 zeroed ints.
 flint_status_t launch_bwd_tc(const void* qh, const void* kh, const void* v, const void* dout,
                              const float* q_norm_w, const float* k_norm_w, const float* lse,
                              const float* delta, const int* seg_lo, const int* seg_hi, float* dq, float* dk,
-                             float* dv, int* status, int* counters, int T, int window, int sms,
+                             float* dv, int* status, int* counters, int* flags, int T, int window, int sms,
                              cudaStream_t s) {
     int dev = 0;
     cudaGetDevice(&dev);
@@ -765,10 +846,12 @@ flint_status_t launch_bwd_tc(const void* qh, const void* kh, const void* v, cons
     p.dk = dk;
     p.dv = dv;
     p.status = status;
+    p.flags = flags;
     p.T = T;
     p.window = window;
+    bwd_pieces(T, window, sms, &p.qp, &p.np);
     const int units_q = ((T + kTokPerTile - 1) / kTokPerTile) * kHKV;
-    const int units_k = ((T + 127) / 128) * kHKV;
+    const int units_k = ((T + 127) / 128) * kHKV * p.np;
     p.counter = counters;
     bwd_dq_tc_kernel<<<units_q < sms ? units_q : sms, kBtThreads, kBtSmemDq, s>>>(tq, tdo, tk, tv, p);
     cudaError_t e = cudaGetLastError();

@@ -71,6 +71,38 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
     }
 }
 
+// ------------------------------------------------------------------ flags between CTAs of one grid
+// Bounded wait until the global word *f reaches at least `want` (acquire at
+// GPU scope).  Gives up when the CTA's abort flag or the status word is set
+// (another CTA failed), or after `limit_ns`, recording FLINT_ERR_TIMEOUT.
+__device__ __forceinline__ bool flag_wait_geq(const int* f, int want, volatile int* abort_flag, int* status,
+                                              unsigned long long limit_ns = kWaitLimitNs) {
+    const unsigned long long t0 = global_ns();
+    for (uint32_t it = 0;; ++it) {
+        int v;
+        asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(f) : "memory");
+        if (v >= want) return true;
+        if ((it & 15u) == 15u) {
+            if (*abort_flag || (status && *reinterpret_cast<volatile int*>(status) != 0)) {
+                *abort_flag = 1;
+                return false;
+            }
+            if (global_ns() - t0 > limit_ns) {
+                if (status) atomicCAS(status, 0, 4 /* FLINT_ERR_TIMEOUT */);
+                *abort_flag = 1;
+                return false;
+            }
+        }
+        __nanosleep(64);
+    }
+}
+// Publishes v in *f after every write this thread has made or observed
+// (fence at GPU scope, then a release store).
+__device__ __forceinline__ void flag_release(int* f, int v) {
+    __threadfence();
+    asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(f), "r"(v) : "memory");
+}
+
 // ------------------------------------------------------------------ programmatic dependent launch
 // The dependent grid (launched with programmatic stream serialization) may
 // start once every CTA of this grid has executed the trigger or exited.

@@ -129,13 +129,17 @@ def test_infinite_and_extreme_sinks():
     assert np.all(got["dq"][:, 0] == 0.0) and got["dsinks"][0] == 0.0 and got["dsinks"][9] == 0.0
 
 
-def test_repeated_calls_are_bitwise_identical():
+@pytest.mark.parametrize("T,window", [(700, 513), (2000, 0)])
+def test_repeated_calls_are_bitwise_identical(T, window):
     """T = 700 gives every warp several work items, so one CTA meets the same
-    head more than once: the per-CTA sums must still be in a fixed order."""
+    head more than once: the per-CTA sums must still be in a fixed order.  On
+    both sequences the dk/dv kernel cuts each key tile's queries into pieces
+    that different CTAs run (10 pieces of 13 query tiles on the causal
+    T = 2000): their sum must be taken in piece order."""
     torch = _torch()
     import full_gqa_learned_b200 as fa
-    w = W.make_small(700, seed=88, window=513, use_rope=True)
-    got, (q, k, v, wq, wk, sk, out, lse, dO, kw) = _run(w, _dout_bits(700, 92))
+    w = W.make_small(T, seed=88, window=window, use_rope=window > 0)
+    got, (q, k, v, wq, wk, sk, out, lse, dO, kw) = _run(w, _dout_bits(T, 92))
     g2 = fa.attn_bwd(q, k, v, wq, wk, sk, out, lse, dO, **kw)
     torch.cuda.synchronize()
     for n, x in g2.items():
