@@ -45,7 +45,7 @@
 
 namespace flint {
 
-constexpr int kBtThreads = 256;
+constexpr int kBtThreads = 384;
 constexpr uint32_t kBtTile = 128 * kHD * 2;          // 32 KiB: 128 rows x 128 x 16-bit
 constexpr uint32_t kBtHalf = kBtTile / 2;
 
@@ -179,7 +179,7 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_qh, const __grid_constan
     if (tid == 0) {
         for (int s = 0; s < 2; ++s) {
             mbar_init(bar(T_SCHED_FULL + s), 1);
-            mbar_init(bar(T_SCHED_EMPTY + s), 1 + 4);     // MMA thread + 4 row warps
+            mbar_init(bar(T_SCHED_EMPTY + s), 1 + 8);     // MMA thread + 8 row warps
             mbar_init(bar(T_A_FULL + s), 1);
             mbar_init(bar(T_A_EMPTY + s), 1);
             mbar_init(bar(T_B_FULL + s), 1);
@@ -188,7 +188,7 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_qh, const __grid_constan
         mbar_init(bar(T_C_FULL), 1);
         mbar_init(bar(T_C_EMPTY), 1);
         mbar_init(bar(T_S_FULL), 1);
-        mbar_init(bar(T_DS_READY), 128);
+        mbar_init(bar(T_DS_READY), 256);
         mbar_init(bar(T_ACC_FULL), 1);
         mbar_init(bar(T_DRAIN), 1);
         misc->abort_flag = 0;
@@ -312,11 +312,12 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_qh, const __grid_constan
                     if (!ok) break;
                     dsph ^= 1;
                     tc_fence_after();
-                    // dQ += dS Kh (K = 128 keys, 8 steps of 16; dS in TMEM)
+                    // dQ += dS Kh (K = 128 keys, 8 steps of 16; dS in TMEM:
+                    // keys 0..63 in columns 0..31, keys 64..127 in 64..95)
 #pragma unroll
                     for (uint32_t kk = 0; kk < 8; ++kk)
-                        mma_ts(tmem + 256, tmem + 8 * kk, dkm + st * kStep + kk * (2048 >> 4), id_dq,
-                               (c > 0 || kk > 0) ? 1u : 0u);
+                        mma_ts(tmem + 256, tmem + 8 * kk + (kk >= 4 ? 32u : 0u), dkm + st * kStep + kk * (2048 >> 4),
+                               id_dq, (c > 0 || kk > 0) ? 1u : 0u);
                     mma_commit(bar(T_A_EMPTY + st));               // K chunk done
                     st ^= 1; if (st == 0) ph ^= 1;
                 }
@@ -330,7 +331,12 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_qh, const __grid_constan
         }
     } else if (warp >= 4) {
         // ------------------------------------------------ rows: dS, then dq~
-        const int r = tid - 128;                        // TMEM lane = tile row
+        // Two warpgroups: warps 4-7 take the key columns 0..63 of every row,
+        // warps 8-11 the columns 64..127; each writes its dS (FP16 pairs)
+        // inside its own columns (0..31, 64..95), so neither overwrites S
+        // the other has yet to read.
+        const int half = (warp - 4) >> 2;
+        const int r = (tid - 128) & 127;                // TMEM lane = tile row
         const int tl = r >> 3, hl = r & 7;
         const uint32_t lb = (uint32_t)(warp & 3) * 32u;
         const uint32_t t_s = tmem + (lb << 16), t_dp = t_s + 128, t_dq = t_s + 256;
@@ -365,7 +371,7 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_qh, const __grid_constan
                 tc_fence_after();
                 const int ks = kb + 128 * c;
 #pragma unroll 1
-                for (int b = 0; b < 4; ++b) {
+                for (int b = 2 * half; b < 2 * half + 2; ++b) {
                     uint32_t sv[32], dv[32], pk[16];
                     tmem_ld32(t_s + 32u * b, sv);
                     tmem_ld32(t_dp + 32u * b, dv);
@@ -383,7 +389,7 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_qh, const __grid_constan
                         }
                         pk[e >> 1] = bt_pack_f16(ds[0], ds[1]);
                     }
-                    tmem_st16(t_s + 16u * b, pk);
+                    tmem_st16(t_s + 16u * b + 32u * half, pk);
                 }
                 tmem_wait_st();
                 tc_fence_before();
@@ -395,7 +401,7 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_qh, const __grid_constan
             tc_fence_after();
             float* dst = p.dq + ((size_t)i * kHQ + h) * kHD;
 #pragma unroll 1
-            for (int b = 0; b < 4; ++b) {
+            for (int b = 2 * half; b < 2 * half + 2; ++b) {
                 uint32_t v[32];
                 tmem_ld32(t_dq + 32u * b, v);
                 tmem_wait_ld();
@@ -441,18 +447,18 @@ bwd_dkv_tc_kernel(const __grid_constant__ CUtensorMap tm_qh, const __grid_consta
     if (tid == 0) {
         for (int s = 0; s < 2; ++s) {
             mbar_init(bar(T_SCHED_FULL + s), 1);
-            mbar_init(bar(T_SCHED_EMPTY + s), 1 + 4);
+            mbar_init(bar(T_SCHED_EMPTY + s), 1 + 8);
             mbar_init(bar(T_A_FULL + s), 1);
             mbar_init(bar(T_A_EMPTY + s), 1);
         }
         mbar_init(bar(T_B_FULL), 1);
         mbar_init(bar(T_B_EMPTY), 1);
         mbar_init(bar(T_S_FULL), 1);
-        mbar_init(bar(T_DS_READY), 128);
+        mbar_init(bar(T_DS_READY), 256);
         mbar_init(bar(T_ACC_FULL), 1);
         mbar_init(bar(T_DRAIN), 1);
         mbar_init(bar(T_GO), 1);
-        mbar_init(bar(T_FIX), 128);
+        mbar_init(bar(T_FIX), 256);
         misc->abort_flag = 0;
         fence_mbar_init();
     }
@@ -608,15 +614,17 @@ bwd_dkv_tc_kernel(const __grid_constant__ CUtensorMap tm_qh, const __grid_consta
                     if (!ok) break;
                     dsph ^= 1;
                     tc_fence_after();
-                    // dV += P^T dO, dK += dS^T Qh (K = 128 query rows, 8 steps of 16)
+                    // dV += P^T dO, dK += dS^T Qh (K = 128 query rows, 8 steps
+                    // of 16; P^T and dS^T in TMEM: query columns 0..63 packed
+                    // into columns 0..31 of their region, 64..127 into 64..95)
 #pragma unroll
                     for (uint32_t kk = 0; kk < 8; ++kk)
-                        mma_ts(tmem + 256, tmem + 8 * kk, ddom + st * kStep + kk * (2048 >> 4), id_dv,
-                               (t > 0 || kk > 0) ? 1u : 0u);
+                        mma_ts(tmem + 256, tmem + 8 * kk + (kk >= 4 ? 32u : 0u), ddom + st * kStep + kk * (2048 >> 4),
+                               id_dv, (t > 0 || kk > 0) ? 1u : 0u);
 #pragma unroll
                     for (uint32_t kk = 0; kk < 8; ++kk)
-                        mma_ts(tmem + 384, tmem + 128 + 8 * kk, dqm + st * kStep + kk * (2048 >> 4), id_dk,
-                               (t > 0 || kk > 0) ? 1u : 0u);
+                        mma_ts(tmem + 384, tmem + 128 + 8 * kk + (kk >= 4 ? 32u : 0u),
+                               dqm + st * kStep + kk * (2048 >> 4), id_dk, (t > 0 || kk > 0) ? 1u : 0u);
                     mma_commit(bar(T_A_EMPTY + st));
                     st ^= 1; if (st == 0) ph ^= 1;
                 }
@@ -630,7 +638,11 @@ bwd_dkv_tc_kernel(const __grid_constant__ CUtensorMap tm_qh, const __grid_consta
         }
     } else if (warp >= 4) {
         // ------------------------------------------------ key rows: P^T, dS^T, then dk~, dv
-        const int r = tid - 128;                        // TMEM lane = key row
+        // Two warpgroups: warps 4-7 take the query columns 0..63 of every
+        // key row, warps 8-11 the columns 64..127 (each writes its P^T and
+        // dS^T inside its own columns), and each stores half of dk~ and dv.
+        const int half = (warp - 4) >> 2;
+        const int r = (tid - 128) & 127;                // TMEM lane = key row
         const uint32_t lb = (uint32_t)(warp & 3) * 32u;
         const uint32_t t_s = tmem + (lb << 16), t_dp = t_s + 128, t_dv = t_s + 256, t_dk = t_s + 384;
         const float C = misc->logit_scale, dks = misc->dk_scale;
@@ -667,29 +679,35 @@ bwd_dkv_tc_kernel(const __grid_constant__ CUtensorMap tm_qh, const __grid_consta
                 const float* cv = colv + st * 256;
                 const int i0 = qb + kTokPerTile * t;
 #pragma unroll 1
-                for (int b = 0; b < 4; ++b) {
+                for (int b = 2 * half; b < 2 * half + 2; ++b) {
                     uint32_t sv[32], dv[32], pp[16], pd[16];
                     tmem_ld32(t_s + 32u * b, sv);
                     tmem_ld32(t_dp + 32u * b, dv);
                     tmem_wait_ld();
 #pragma unroll
-                    for (int e = 0; e < 32; e += 2) {
-                        float pr[2], ds[2];
+                    for (int e = 0; e < 32; e += 4) {
+                        // lse2 and D of columns 32b + e .. +3 (one broadcast load each)
+                        const float4 l4 = *reinterpret_cast<const float4*>(cv + 32 * b + e);
+                        const float4 d4 = *reinterpret_cast<const float4*>(cv + 128 + 32 * b + e);
+                        const float lv[4] = {l4.x, l4.y, l4.z, l4.w}, dd[4] = {d4.x, d4.y, d4.z, d4.w};
+                        float pr[4], ds[4];
 #pragma unroll
-                        for (int q = 0; q < 2; ++q) {
+                        for (int q = 0; q < 4; ++q) {
                             const int n = 32 * b + e + q;            // column: token i0 + n/8, head n%8
                             const int i = i0 + (n >> 3);
                             float x = 0.f;
                             if (valid && i >= j && i < hi)
-                                x = bt_ex2(fmaf(__uint_as_float(sv[e + q]), C, -cv[n]));
+                                x = bt_ex2(fmaf(__uint_as_float(sv[e + q]), C, -lv[q]));
                             pr[q] = x;
-                            ds[q] = x * (__uint_as_float(dv[e + q]) - cv[128 + n]);
+                            ds[q] = x * (__uint_as_float(dv[e + q]) - dd[q]);
                         }
                         pp[e >> 1] = bt_pack_bf16(pr[0], pr[1]);
+                        pp[(e >> 1) + 1] = bt_pack_bf16(pr[2], pr[3]);
                         pd[e >> 1] = bt_pack_f16(ds[0], ds[1]);
+                        pd[(e >> 1) + 1] = bt_pack_f16(ds[2], ds[3]);
                     }
-                    tmem_st16(t_s + 16u * b, pp);
-                    tmem_st16(t_dp + 16u * b, pd);
+                    tmem_st16(t_s + 16u * b + 32u * half, pp);
+                    tmem_st16(t_dp + 16u * b + 32u * half, pd);
                 }
                 tmem_wait_st();
                 tc_fence_before();
@@ -719,7 +737,7 @@ bwd_dkv_tc_kernel(const __grid_constant__ CUtensorMap tm_qh, const __grid_consta
             float* dkd = p.dk + ((size_t)j * kHKV + g) * kHD;
             float* dvd = p.dv + ((size_t)j * kHKV + g) * kHD;
 #pragma unroll 1
-            for (int b = 0; b < 4; ++b) {
+            for (int b = 2 * half; b < 2 * half + 2; ++b) {
                 uint32_t a[32], c[32];
                 tmem_ld32(t_dk + 32u * b, a);
                 tmem_ld32(t_dv + 32u * b, c);
