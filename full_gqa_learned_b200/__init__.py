@@ -195,22 +195,23 @@ def attn_decode(q, k, v, q_norm_w, k_norm_w, sinks, k_cache, v_cache, cache_len,
     """One decode step (see include/flint_attn.h, flint_attn_decode).
 
     q [B,32,128], k/v [B,4,128] bf16: the new token of each sequence;
-    k_cache, v_cache [B,cap,4,128] bf16 (position j in slot j mod cap; the
-    step writes the new token into slot cache_len[b] mod cap); cache_len [B]
+    k_cache, v_cache [B,4,cap,128] bf16, head-major (position j of KV head
+    g in [b, g, j mod cap]; the step writes the new token into slot
+    cache_len[b] mod cap); cache_len [B]
     int32.  Returns (out [B,4096] bf16, lse [32,B] f32 or None).
     """
     import torch
     lib = load_library()
     B = int(q.shape[0]) if q.dim() >= 1 else 0
-    cap = int(k_cache.shape[1]) if k_cache.dim() >= 2 else 0
+    cap = int(k_cache.shape[2]) if k_cache.dim() >= 3 else 0
     _check(q, "q", torch.bfloat16, (B, HQ, HEAD_DIM))
     _check(k, "k", torch.bfloat16, (B, HKV, HEAD_DIM))
     _check(v, "v", torch.bfloat16, (B, HKV, HEAD_DIM))
     _check(q_norm_w, "q_norm_w", torch.float32, (HEAD_DIM,))
     _check(k_norm_w, "k_norm_w", torch.float32, (HEAD_DIM,))
     _check(sinks, "sinks", torch.float32, (HQ,))
-    _check(k_cache, "k_cache", torch.bfloat16, (B, cap, HKV, HEAD_DIM))
-    _check(v_cache, "v_cache", torch.bfloat16, (B, cap, HKV, HEAD_DIM))
+    _check(k_cache, "k_cache", torch.bfloat16, (B, HKV, cap, HEAD_DIM))
+    _check(v_cache, "v_cache", torch.bfloat16, (B, HKV, cap, HEAD_DIM))
     _check(cache_len, "cache_len", torch.int32, (B,))
     dev = q.device
     if out is None:

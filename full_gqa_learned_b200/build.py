@@ -19,9 +19,9 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libflint_attn.so")
-SOURCES = ["flint_abi.cu", "flint_prep.cu", "flint_attn.cu", "flint_static.cu", "flint_decode.cu",
+SOURCES = ["flint_abi.cu", "flint_prep.cu", "flint_attn.cu", "flint_static.cu", "flint_decode.cu", "flint_decode_tc.cu",
            "flint_bwd.cu", "flint_bwd_tc.cu", "flint_gemm.cu"]
-HEADERS = ["flint_common.cuh", "sm100.cuh", "flint_host.cuh"]
+HEADERS = ["flint_common.cuh", "sm100.cuh", "flint_host.cuh", "flint_decode.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

@@ -14,9 +14,14 @@
 // honour per-layer window sizes).  The step appends the new token: its
 // normalised, rotated key (rounded to BF16) and its value go to slot p mod cap.
 //
-// Split-KV: CTA (s, g, b) takes keys lo + 256 s .. lo + 256 s + 255 of KV head
-// g and writes a partial (m, l, O) per query head in log2 units; the combine
-// kernel folds the partials and the sink:
+// This file: the CUDA-core path (any norm weights) and the host side;
+// flint_decode_tc.cu holds the tensor-core path taken when the logit bound
+// is <= 48.  Both write partials in the same format and fold them with
+// decode_fold (flint_decode.cuh).
+//
+// Split-KV: item (s, g, b) takes keys lo + 256 s .. lo + 256 s + 255 of KV
+// head g and writes a partial (m, l, O) per query head in log2 units; the
+// last split of (b, g) to finish folds the partials and the sink:
 //   M = max(sink * log2e, max_s m_s)
 //   L = 2^(sink * log2e - M) + sum_s l_s 2^(m_s - M)
 //   out = sum_s O_s 2^(m_s - M) / L,  lse = (M ln 2 + ln L)
@@ -27,63 +32,13 @@
 
 #include "../../include/flint_attn.h"
 #include "flint_common.cuh"
+#include "flint_decode.cuh"
 #include "sm100.cuh"
 
 namespace flint {
 
 constexpr int kDecKeys = 256;          // keys per split
 constexpr int kDecThreads = 128;       // split kernel: 2 keys per thread for the scores
-constexpr int kCombThreads = kHD;      // combine kernel: one thread per channel
-
-__device__ __forceinline__ float dec_bf16(uint32_t bits16) { return __uint_as_float(bits16 << 16); }
-
-// Normalise (weight form) and, if rope, rotate one 128-channel row held by a
-// warp: lane l owns channels l, l+32, l+64, l+96 (the pairs (l, l+64) and
-// (l+32, l+96) rotate with frequencies l and l+32).  Returns the 4 values.
-__device__ __forceinline__ void dec_norm_rope_row(const __nv_bfloat16* row, const float* w, float eps,
-                                                  bool rope, int pos, const double* inv_freq, int lane,
-                                                  float y[4]) {
-    const uint16_t* r16 = reinterpret_cast<const uint16_t*>(row);
-    float x[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) x[i] = dec_bf16(r16[lane + 32 * i]);
-    float ss = x[0] * x[0] + x[1] * x[1] + x[2] * x[2] + x[3] * x[3];
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-    const float rn = rsqrtf(ss * (1.f / kHD) + eps);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) y[i] = x[i] * rn * w[lane + 32 * i];
-    if (rope) {
-#pragma unroll
-        for (int i = 0; i < 2; ++i) {
-            float c, s;
-            rope_cos_sin(pos, inv_freq[lane + 32 * i], &c, &s);
-            const float a = y[i], b = y[i + 2];
-            y[i] = a * c - b * s;
-            y[i + 2] = b * c + a * s;
-        }
-    }
-}
-
-struct DecodeParams {
-    const __nv_bfloat16* q;      // [B,32,128]
-    const __nv_bfloat16* k;      // [B,4,128]
-    const __nv_bfloat16* v;      // [B,4,128]
-    const float* q_norm_w;
-    const float* k_norm_w;
-    const float* sinks;
-    __nv_bfloat16* k_cache;      // [B,cap,4,128]
-    __nv_bfloat16* v_cache;      // [B,cap,4,128]
-    const int* cache_len;        // [B]
-    __nv_bfloat16* out;          // [B,4096]
-    float* lse;                  // [32,B]
-    int* status;                 // device status word
-    float* part;                 // [B,4,nsplit,8,(2 + 128)]
-    int B, cap, window, use_rope, nsplit;
-    float rope_theta, eps;
-};
-
-constexpr int kPartFloats = 8 * (2 + kHD);   // m[8], l[8], O[8][128]
 
 // 6 CTAs per SM (80 registers): more loads in flight than one CTA's worth
 __global__ void __launch_bounds__(kDecThreads, 6)
@@ -94,10 +49,17 @@ decode_split_kernel(const DecodeParams p) {
     __shared__ __align__(16) float s_o[kDecThreads / 2][2 * kGroup];   // second key half's PV sums
     __shared__ float s_w[2][kHD];              // q_norm_w, k_norm_w
     __shared__ double s_inv[64];
-    __shared__ float s_m[kGroup];
+    __shared__ int s_last;
 
-    const int s = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    // under a logit bound <= 48 the tensor-core tile kernel does the step
+    {
+        const float bnd = decode_logit_bound(p.q_norm_w, p.k_norm_w);
+        if (bnd <= kDecodeBoundMax) return;
+    }
+    // CTA (loop over items (s, g, b)): keys lo + 256 s .. of KV head g of
+    // sequence b; the last split of (b, g) to finish folds all of them
+    auto run_item = [&](const int s, const int g, const int b) {
     const int pos = p.cache_len[b];
     const int lo = p.window > 0 ? max(0, pos - p.window + 1) : 0;
     const int n = pos - lo + 1;
@@ -135,8 +97,8 @@ decode_split_kernel(const DecodeParams p) {
         dec_norm_rope_row(p.k + ((size_t)b * kHKV + g) * kHD, s_w[1], p.eps, p.use_rope != 0, pos, s_inv,
                           lane, y);
         const size_t slot = (size_t)(pos % p.cap);
-        __nv_bfloat16* kdst = p.k_cache + (((size_t)b * p.cap + slot) * kHKV + g) * kHD;
-        __nv_bfloat16* vdst = p.v_cache + (((size_t)b * p.cap + slot) * kHKV + g) * kHD;
+        __nv_bfloat16* kdst = p.k_cache + (((size_t)b * kHKV + g) * p.cap + slot) * kHD;
+        __nv_bfloat16* vdst = p.v_cache + (((size_t)b * kHKV + g) * p.cap + slot) * kHD;
         const __nv_bfloat16* vsrc = p.v + ((size_t)b * kHKV + g) * kHD;
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
@@ -167,7 +129,7 @@ decode_split_kernel(const DecodeParams p) {
             }
         } else if (kj < k1) {
             const uint4* krow = reinterpret_cast<const uint4*>(
-                p.k_cache + (((size_t)b * p.cap + (size_t)(kj % p.cap)) * kHKV + g) * kHD);
+                p.k_cache + (((size_t)b * kHKV + g) * p.cap + (size_t)(kj % p.cap)) * kHD);
             // the whole 256-byte row in flight at once
             uint4 kr[kHD / 8];
 #pragma unroll
@@ -213,7 +175,7 @@ decode_split_kernel(const DecodeParams p) {
         }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-        if (lane == 0) { s_m[h] = mx; part[h] = mx; part[kGroup + h] = sum; }
+        if (lane == 0) { part[h] = mx; part[kGroup + h] = sum; }
     }
     __syncthreads();
 
@@ -227,8 +189,8 @@ decode_split_kernel(const DecodeParams p) {
         const int nk = k1 - k0;
         const int jb = kh * (kDecKeys / 2), je = min(nk, jb + kDecKeys / 2);
         const uint32_t* vnew = reinterpret_cast<const uint32_t*>(p.v + ((size_t)b * kHKV + g) * kHD) + cp;
-        const uint32_t* vbase = reinterpret_cast<const uint32_t*>(p.v_cache + ((size_t)b * p.cap * kHKV + g) * kHD) + cp;
-        const size_t slot_stride = (size_t)kHKV * kHD / 2;        // 32-bit words per cache slot
+        const uint32_t* vbase = reinterpret_cast<const uint32_t*>(p.v_cache + ((size_t)b * kHKV + g) * p.cap * kHD) + cp;
+        const size_t slot_stride = (size_t)kHD / 2;               // 32-bit words per cache slot
         int slot = (k0 + jb) % p.cap;                             // advances by one per key
 #pragma unroll 16
         for (int jj = jb; jj < je; ++jj) {
@@ -258,45 +220,21 @@ decode_split_kernel(const DecodeParams p) {
             }
         }
     }
-}
-
-// Folds the partials of (b, g) with the sinks of its 8 query heads.
-__global__ void __launch_bounds__(kCombThreads)
-decode_combine_kernel(const DecodeParams p) {
-    const int g = blockIdx.x, b = blockIdx.y, c = threadIdx.x;
-    griddep_wait();
-    if (c >= kHD) return;
-    const float* base = p.part + ((size_t)b * kHKV + g) * p.nsplit * kPartFloats;
-    for (int hh = 0; hh < kGroup; ++hh) {
-        const int h = kGroup * g + hh;
-        const float sink = p.sinks[h];
-        float acc = 0.f, L = 0.f, M;
-        if (sink == INFINITY) {
-            M = INFINITY;
-        } else {
-            M = sink * 1.4426950408889634f;
-            for (int s = 0; s < p.nsplit; ++s) M = fmaxf(M, base[s * kPartFloats + hh]);
-            if (M > -INFINITY) {
-                L = (sink > -INFINITY) ? exp2f(sink * 1.4426950408889634f - M) : 0.f;
-                for (int s = 0; s < p.nsplit; ++s) {
-                    const float* ps = base + s * kPartFloats;
-                    const float ms = ps[hh];
-                    if (ms == -INFINITY) continue;
-                    const float a = exp2f(ms - M);
-                    L += ps[kGroup + hh] * a;
-                    acc += ps[2 * kGroup + hh * kHD + c] * a;
-                }
-            }
+    };
+    const int n_items = p.nsplit * kHKV * p.B;
+    for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
+        const int s = item % p.nsplit, g = (item / p.nsplit) % kHKV, b = item / (p.nsplit * kHKV);
+        run_item(s, g, b);
+        // this split's partial is written: the last of the (b, g) splits folds
+        __threadfence();
+        __syncthreads();
+        if (tid == 0) s_last = atomicAdd(p.arrive + b * kHKV + g, 1) == p.nsplit - 1;
+        __syncthreads();
+        if (s_last) {
+            __threadfence();
+            decode_fold(p, b, g, p.nsplit, tid);
         }
-        const float o = (L > 0.f) ? acc / L : 0.f;
-        p.out[((size_t)b * kHQ + h) * kHD + c] = __float2bfloat16_rn(o);
-        if (c == 0 && p.lse) {
-            float v;
-            if (M == INFINITY) v = INFINITY;
-            else if (L > 0.f) v = M * 0.6931471805599453f + logf(L);
-            else v = -INFINITY;
-            p.lse[(size_t)h * p.B + b] = v;
-        }
+        __syncthreads();
     }
 }
 
@@ -308,8 +246,11 @@ size_t decode_nsplit(int cap, int window) {
 }
 
 size_t decode_workspace_bytes(int B, int cap, int window) {
-    return 256 + (size_t)B * kHKV * decode_nsplit(cap, window) * kPartFloats * sizeof(float);
+    const size_t ns = decode_nsplit(cap, window), nt = (size_t)decode_tc_nsplit(cap);
+    return decode_header_bytes(B) + (size_t)B * kHKV * (ns > nt ? ns : nt) * kPartFloats * sizeof(float);
 }
+
+flint_status_t launch_decode_tc(const DecodeParams& p, int sms, cudaStream_t s);
 
 flint_status_t run_decode(const void* q, const void* k, const void* v, const float* q_norm_w,
                           const float* k_norm_w, const float* sinks, void* k_cache, void* v_cache,
@@ -329,33 +270,36 @@ flint_status_t run_decode(const void* q, const void* k, const void* v, const flo
     dp.out = static_cast<__nv_bfloat16*>(out);
     dp.lse = lse;
     dp.status = static_cast<int*>(workspace);
-    dp.part = reinterpret_cast<float*>(static_cast<char*>(workspace) + 256);
+    dp.arrive = reinterpret_cast<int*>(static_cast<char*>(workspace) + 256);
+    dp.part = reinterpret_cast<float*>(static_cast<char*>(workspace) + decode_header_bytes(B));
     dp.B = B;
     dp.cap = cap;
     dp.window = window;
     dp.use_rope = use_rope;
     dp.nsplit = (int)decode_nsplit(cap, window);
+    dp.nsplit_tc = decode_tc_nsplit(cap);
     dp.rope_theta = rope_theta;
     dp.eps = eps;
     (void)workspace_bytes;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    cudaError_t e = cudaMemsetAsync(workspace, 0, sizeof(int), s);
+    // status word, the tile kernel's work counter, the split-arrival counters
+    cudaError_t e = cudaMemsetAsync(workspace, 0, decode_header_bytes(B), s);
     if (e != cudaSuccess) return set_error(FLINT_ERR_CUDA, "decode: status reset failed");
-    decode_split_kernel<<<dim3(dp.nsplit, kHKV, B), kDecThreads, 0, s>>>(dp);
+    // Both kernels are enqueued; each decides from the norm weights whether
+    // it runs (the tile kernel under a logit bound <= 48) and the other
+    // returns at once.  Each writes the output itself (the last split of a
+    // sequence and KV head folds them all).
+    int sms = 0, dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    flint_status_t st = launch_decode_tc(dp, sms > 0 ? sms : 1, s);
+    if (st != FLINT_OK) return st;
+    const long long items = (long long)dp.nsplit * kHKV * B;
+    const long long cap_grid = 6LL * (sms > 0 ? sms : 1);
+    const int grid = (int)(items < cap_grid ? items : cap_grid);
+    decode_split_kernel<<<grid, kDecThreads, 0, s>>>(dp);
     e = cudaGetLastError();
     if (e != cudaSuccess) return set_error(FLINT_ERR_CUDA, "decode: split launch failed");
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(kHKV, B);
-    cfg.blockDim = dim3(kCombThreads);
-    cfg.dynamicSmemBytes = 0;
-    cfg.stream = s;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, decode_combine_kernel, dp);
-    if (e != cudaSuccess) return set_error(FLINT_ERR_CUDA, "decode: combine launch failed");
     return FLINT_OK;
 }
 

@@ -134,6 +134,11 @@ __device__ __forceinline__ void regs_dec() {
 }
 
 // ------------------------------------------------------------------ TMA
+// Asynchronous prefetch of `bytes` (a multiple of 16, 16-byte aligned) of
+// global memory into L2.
+__device__ __forceinline__ void bulk_prefetch_l2(const void* p, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
 __device__ __forceinline__ void tma_prefetch_desc(const void* desc) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(desc) : "memory");
 }
@@ -144,6 +149,16 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const void* desc, uint
         "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
         " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
         "l"(desc), "r"(bar), "r"(c0), "r"(c1), "r"(c2)
+        : "memory");
+}
+
+// 4-D tiled load into shared memory, completion counted on `bar`.
+__device__ __forceinline__ void tma_load_4d(uint32_t dst, const void* desc, uint32_t bar, int c0, int c1,
+                                            int c2, int c3) {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5, %6}], [%2];" ::"r"(dst),
+        "l"(desc), "r"(bar), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
         : "memory");
 }
 
@@ -332,6 +347,11 @@ __host__ __device__ constexpr uint32_t idesc_f16(uint32_t a_bf16, uint32_t b_bf1
            | (b_mn_major << 16)      // B major
            | ((n >> 3) << 17)        // N / 8
            | ((128u >> 4) << 24);    // M / 16
+}
+
+// Same with A stored M-major (the tile's rows run along K).
+__host__ __device__ constexpr uint32_t idesc_f16_amn(uint32_t a_bf16, uint32_t b_bf16, uint32_t n) {
+    return idesc_f16(a_bf16, b_bf16, 0, n) | (1u << 15);
 }
 
 }  // namespace flint

@@ -306,10 +306,15 @@ FLINT_API flint_status_t flint_attn_fwd_static_status(void* stream);
  *  q          bf16 [B,32,128]: the new tokens' projected queries, before q_norm.
  *  k, v       bf16 [B,4,128]: their projected keys (before k_norm) and values.
  *  q_norm_w, k_norm_w, sinks   as for flint_attn_fwd.
- *  k_cache    bf16 [B,cap,4,128]: normalised, rotated keys of earlier
- *             positions; position j of sequence b lives in slot j mod cap, so
- *             a cache of capacity >= window is a ring on sliding layers.
- *  v_cache    bf16 [B,cap,4,128]: values, same slots.
+ *  k_cache    bf16 [B,4,cap,128], head-major: normalised, rotated keys of
+ *             earlier positions; position j of sequence b, KV head g lives in
+ *             k_cache[b][g][j mod cap], so a cache of capacity >= window is a
+ *             ring on sliding layers, and each head's slots are consecutive
+ *             256-byte rows.  The keys are assumed normalised with k_norm_w
+ *             (|k~|_2 <= sqrt(128) max|k_norm_w|, as the step itself writes
+ *             them): the tensor-core path starts its softmax from the bound
+ *             this gives on every logit.
+ *  v_cache    bf16 [B,4,cap,128]: values, same slots.
  *             The step writes the new token's key (normalised, rotated,
  *             rounded to BF16) and value into slot p mod cap.  The window
  *             must fit the cache (p - lo + 1 <= cap); otherwise the device
@@ -330,9 +335,15 @@ FLINT_API flint_status_t flint_attn_fwd_static_status(void* stream);
  *             (read with flint_attn_device_status) and the split partials.
  *  stream     cudaStream_t as void*.
  *
- * Queries, keys and scores are computed in FP32 on CUDA cores; the key
- * range of every (sequence, KV head) is split in blocks of 256 keys whose
- * partial results a second kernel combines with the sink.
+ * When the logit bound 16.45 max|q_norm_w| max|k_norm_w| (log2 units) is at
+ * most 48, a tensor-core kernel streams the cache in tiles of 128 slots:
+ * scores from BF16 keys and queries split into BF16 high and low parts
+ * (FP32 accumulation), probabilities 2^(s - bound) in BF16 for the value
+ * product; splits of up to 8 tiles per (sequence, KV head), the last split
+ * to finish folding them with the sink.  Otherwise queries, keys and scores
+ * are computed in FP32 on CUDA cores over splits of 256 positions, folded
+ * the same way.  One call launches both kernels; the one not taken returns
+ * at once.
  */
 FLINT_API size_t flint_attn_decode_workspace_bytes(int32_t B, int32_t cap, int32_t window);
 FLINT_API flint_status_t flint_attn_decode(const void* q, const void* k, const void* v,

@@ -47,14 +47,14 @@ def decode_step(q, k, v, k_cache, v_cache, cache_len, q_norm_w, k_norm_w, sinks,
     """One decode step for B sequences.
 
     q [B,32,128], k and v [B,4,128]: the new token's projections (BF16 bit
-    patterns or floats); k_cache, v_cache [B,cap,4,128] (BF16 bit patterns or
-    floats); cache_len [B].  Returns out [B,32,128], lse [32,B] and the new
+    patterns or floats); k_cache, v_cache [B,4,cap,128] (BF16 bit patterns or
+    floats; head-major: slot j of KV head g is k_cache[b, g, j]); cache_len [B].  Returns out [B,32,128], lse [32,B] and the new
     token's normalised, rotated keys k~ [B,4,128], all float64.
     """
     q, k, v = _f64(q), _f64(k), _f64(v)
     kc, vc = _f64(k_cache), _f64(v_cache)
     sinks = np.asarray(sinks, np.float64).reshape(HQ)
-    B, cap = kc.shape[0], kc.shape[1]
+    B, cap = kc.shape[0], kc.shape[2]
     q = q.reshape(B, HQ, D)
     k = k.reshape(B, HKV, D)
     v = v.reshape(B, HKV, D)
@@ -71,8 +71,8 @@ def decode_step(q, k, v, k_cache, v_cache, cache_len, q_norm_w, k_norm_w, sinks,
         slots = pos % cap
         for g in range(HKV):
             k_new[b, g] = normalise(k[b, g], k_norm_w, p, use_rope, rope_theta, eps)
-            keys = np.concatenate([kc[b, slots, g], k_new[b, g][None]], axis=0)
-            vals = np.concatenate([vc[b, slots, g], v[b, g][None]], axis=0)
+            keys = np.concatenate([kc[b, g, slots], k_new[b, g][None]], axis=0)
+            vals = np.concatenate([vc[b, g, slots], v[b, g][None]], axis=0)
             for h in range(GROUP * g, GROUP * (g + 1)):
                 qt = normalise(q[b, h], q_norm_w, p, use_rope, rope_theta, eps)
                 s = keys @ qt * scale

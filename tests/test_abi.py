@@ -138,11 +138,17 @@ def call_decode(lib, **kw):
 
 
 def test_decode_workspace_bytes(lib):
-    # status word + partials: 4 KV heads x splits of 128 keys x (8 x 130) floats
+    # header (status, item counter, per-(sequence, KV head) arrival counters:
+    # 256 + 256 bytes for 8 sequences) + partials: 4 KV heads x splits x
+    # (8 x 130) floats, for the larger of the two kernels' split counts
+    # (CUDA cores: 256 positions of the window per split; tensor cores: 8
+    # tiles of 128 cache slots)
+    head = 256 + 256
     a = fa.decode_workspace_bytes(8, 513, 513)
-    assert a >= 256 + 8 * 4 * 2 * 8 * 130 * 4
-    assert fa.decode_workspace_bytes(8, 4096, 0) > a        # full layer: splits follow the capacity
-    assert fa.decode_workspace_bytes(8, 4096, 513) == a     # sliding: the window bounds the splits
+    assert a == head + 8 * 4 * 3 * 8 * 130 * 4
+    assert fa.decode_workspace_bytes(8, 4096, 0) == head + 8 * 4 * 16 * 8 * 130 * 4
+    # a ring larger than the window: the tensor-core splits follow the slots
+    assert fa.decode_workspace_bytes(8, 4096, 513) == head + 8 * 4 * 4 * 8 * 130 * 4
     assert fa.decode_workspace_bytes(-1, 513, 513) == 0
     assert fa.decode_workspace_bytes(8, 0, 513) == 0
     assert fa.decode_workspace_bytes(8, 513, -1) == 0

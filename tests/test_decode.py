@@ -61,8 +61,8 @@ def check_appended(d, t, k_new_ref):
     vc = t["v_cache"].view(__import__("torch").int16).cpu().numpy().view(np.uint16)
     for b in range(d.B):
         slot = int(d.cache_len[b]) % d.cap
-        np.testing.assert_array_equal(vc[b, slot], d.v[b])
-        got = W.bf16_to_f64(kc[b, slot])
+        np.testing.assert_array_equal(vc[b, :, slot], d.v[b])
+        got = W.bf16_to_f64(kc[b, :, slot])
         # BF16 rounding (half a unit, 2^-9 relative) of an FP32 value whose
         # rotation carries ~1e-6 absolute error at positions up to 2^18
         err = np.abs(got - k_new_ref[b])
@@ -71,7 +71,8 @@ def check_appended(d, t, k_new_ref):
 
 @pytest.mark.parametrize("B,cap,window,rope,max_len", [(5, 513, 513, True, 3000), (4, 700, 0, False, 700),
                                                        (3, 300, 0, True, 300), (6, 40, 33, True, 200),
-                                                       (2, 1, 1, True, 50)])
+                                                       (2, 1, 1, True, 50), (3, 1000, 513, True, 5000),
+                                                       (2, 2600, 0, True, 2600)])
 def test_decode_matches_oracle(B, cap, window, rope, max_len):
     d = W.make_decode(B, cap, seed=50 + B + cap, window=window, use_rope=rope, max_len=max_len)
     ref_o, ref_l, k_new = OD.decode_step(d.q, d.k, d.v, d.k_cache, d.v_cache, d.cache_len, d.q_norm_w,
@@ -134,6 +135,26 @@ def test_named_decode_workloads(name):
     d = W.make_decode_named(name)
     ref_o, ref_l, k_new = OD.decode_step(d.q, d.k, d.v, d.k_cache, d.v_cache, d.cache_len, d.q_norm_w,
                                          d.k_norm_w, d.sinks, window=d.window, use_rope=d.use_rope)
+    t = to_dev(d)
+    st, o, l = run(d, t)
+    assert st == 0
+    compare(d, o, l, ref_o, ref_l)
+    check_appended(d, t, k_new)
+
+
+@pytest.mark.parametrize("scale", [1.0, 3.0])
+def test_both_decode_paths(scale):
+    """Norm weights scaled by 3 put the logit bound (16.45 max|w_q| max|w_k|)
+    far above 48: the step then runs the CUDA-core split kernel instead of the
+    tensor-core tile kernel; both must match the oracle.  A ring larger than
+    the window holds stale positions outside it."""
+    d = W.make_decode(4, 600, seed=63, window=513, use_rope=True, max_len=4000)
+    d.q_norm_w = (np.asarray(d.q_norm_w, np.float32) * scale).astype(np.float32)
+    d.k_norm_w = (np.asarray(d.k_norm_w, np.float32) * scale).astype(np.float32)
+    bound = 16.45 * np.abs(d.q_norm_w).max() * np.abs(d.k_norm_w).max()
+    assert (bound <= 48) == (scale == 1.0)
+    ref_o, ref_l, k_new = OD.decode_step(d.q, d.k, d.v, d.k_cache, d.v_cache, d.cache_len, d.q_norm_w,
+                                         d.k_norm_w, d.sinks, window=513, use_rope=True)
     t = to_dev(d)
     st, o, l = run(d, t)
     assert st == 0

@@ -11,14 +11,14 @@ from oracle import decode as OD
 def _cache_from_prefill(w, L, window, use_rope, cap, fill=0.0):
     """Cache of capacity cap holding the exact normalised, rotated keys and the
     values of positions lo..L-1 at slots j mod cap; other slots hold `fill`."""
-    kc = np.full((1, cap, 4, 128), fill)
-    vc = np.full((1, cap, 4, 128), fill)
+    kc = np.full((1, 4, cap, 128), fill)
+    vc = np.full((1, 4, cap, 128), fill)
     kf, vf = oracle._f64(w.k), oracle._f64(w.v)
     lo = max(0, L - window + 1) if window > 0 else 0
     for j in range(lo, L):
         for g in range(4):
-            kc[0, j % cap, g] = OD.normalise(kf[j, g], w.k_norm_w, j, use_rope, 1e4, 1e-6)
-        vc[0, j % cap] = vf[j]
+            kc[0, g, j % cap] = OD.normalise(kf[j, g], w.k_norm_w, j, use_rope, 1e4, 1e-6)
+        vc[0, :, j % cap] = vf[j]
     return kc, vc
 
 
@@ -46,7 +46,7 @@ def test_single_key_closed_form():
     """Empty cache and sink = -inf: the only key is the token itself, so
     out = v and lse = q~ . k~ / sqrt(128)."""
     w = W.make_small(1, seed=40, window=0, use_rope=True, sinks=-np.inf)
-    kc = np.zeros((1, 2, 4, 128))
+    kc = np.zeros((1, 4, 2, 128))
     out, lse, k_new = OD.decode_step(w.q, w.k, w.v, kc, kc, [0], w.q_norm_w, w.k_norm_w, w.sinks,
                                      window=513, use_rope=True)
     q, v = oracle._f64(w.q), oracle._f64(w.v)
@@ -59,7 +59,7 @@ def test_single_key_closed_form():
 
 def test_infinite_sinks():
     w = W.make_small(1, seed=41, window=0, use_rope=False, sinks=np.inf)
-    kc = np.zeros((1, 1, 4, 128))
+    kc = np.zeros((1, 4, 1, 128))
     out, lse, _ = OD.decode_step(w.q, w.k, w.v, kc, kc, [0], w.q_norm_w, w.k_norm_w, w.sinks,
                                  window=0, use_rope=False)
     assert np.all(out == 0) and np.all(lse == np.inf)

@@ -21,8 +21,8 @@ MUTANTS = {
                     "z = e.sum() + (np.exp(sink * scale - m) if sink > -np.inf else 0.0)"),
     "gqa_modulo": ("for h in range(GROUP * g, GROUP * (g + 1)):", "for h in range(g, HQ, HKV):"),
     "no_logit_scale": ("s = keys @ qt * scale", "s = keys @ qt"),
-    "new_token_excluded": [("keys = np.concatenate([kc[b, slots, g], k_new[b, g][None]], axis=0)",
-                            "keys = np.concatenate([kc[b, slots, g], 0.0 * k_new[b, g][None] - 1e30], axis=0)")],
+    "new_token_excluded": [("keys = np.concatenate([kc[b, g, slots], k_new[b, g][None]], axis=0)",
+                            "keys = np.concatenate([kc[b, g, slots], 0.0 * k_new[b, g][None] - 1e30], axis=0)")],
     "lse_log2": ("lse[h, b] = m + np.log(z)", "lse[h, b] = m + np.log2(z)"),
 }
 

@@ -324,8 +324,8 @@ class DecodeWorkload:
     q: np.ndarray          # uint16 [B,32,128]
     k: np.ndarray          # uint16 [B,4,128]
     v: np.ndarray          # uint16 [B,4,128]
-    k_cache: np.ndarray    # uint16 [B,cap,4,128]
-    v_cache: np.ndarray    # uint16 [B,cap,4,128]
+    k_cache: np.ndarray    # uint16 [B,4,cap,128] (head-major)
+    v_cache: np.ndarray    # uint16 [B,4,cap,128]
     cache_len: np.ndarray  # int32 [B]: position of the new token
     q_norm_w: np.ndarray
     k_norm_w: np.ndarray
@@ -341,7 +341,7 @@ class DecodeWorkload:
 
     @property
     def cap(self) -> int:
-        return int(self.k_cache.shape[1])
+        return int(self.k_cache.shape[2])          # [B, 4, cap, 128]
 
     def keys_per_sequence(self) -> np.ndarray:
         """Keys each new token attends to (its window, itself included)."""
@@ -370,8 +370,8 @@ def make_decode(B, cap, seed, *, window, use_rope, max_len, min_len=0, name="dec
     s = rng.standard_normal(HQ).astype(np.float32)
     if sinks is not None:
         s = np.broadcast_to(np.asarray(sinks, dtype=np.float32), (HQ,)).copy()
-    kc = bf16_bits(_normal(rng, (B, cap, HKV, D), 1.0))
-    vc = bf16_bits(_normal(rng, (B, cap, HKV, D), 1.0))
+    kc = bf16_bits(_normal(rng, (B, HKV, cap, D), 1.0))
+    vc = bf16_bits(_normal(rng, (B, HKV, cap, D), 1.0))
     cache_len = rng.integers(min_len, max_len, size=B).astype(np.int32)
     return DecodeWorkload(name, q, k, v, kc, vc, cache_len, wq, wk, s, window=window, use_rope=use_rope)
 
