@@ -294,8 +294,10 @@ flint_status_t run_decode(const void* q, const void* k, const void* v, const flo
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     flint_status_t st = launch_decode_tc(dp, sms > 0 ? sms : 1, s);
     if (st != FLINT_OK) return st;
+    // two CTAs per SM loop over the items (when the tile kernel runs, these
+    // only read the weights and return)
     const long long items = (long long)dp.nsplit * kHKV * B;
-    const long long cap_grid = 6LL * (sms > 0 ? sms : 1);
+    const long long cap_grid = 2LL * (sms > 0 ? sms : 1);
     const int grid = (int)(items < cap_grid ? items : cap_grid);
     decode_split_kernel<<<grid, kDecThreads, 0, s>>>(dp);
     e = cudaGetLastError();

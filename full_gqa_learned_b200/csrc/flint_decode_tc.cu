@@ -85,6 +85,7 @@ struct DtMisc {
     float s_new[2][8];                  // per item parity: the new token's scores, per head (unscaled)
     float red_l[2][4][8];               // per item parity and slot-row warp: its part of l, per head
     int last;                           // this split is the last of its (b, g) to finish
+    float sinks[kHQ];                   // the learned sinks
 };
 static_assert(sizeof(DtMisc) <= 512, "misc block");
 
@@ -192,6 +193,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_kc, const __grid_constan
         tmem_relinquish();
     }
     double* inv_freq = reinterpret_cast<double*>(smem + kDtOffInv);
+    if (warp == 3) misc->sinks[lane] = p.sinks[lane];
     if (warp == 2) {
         const double l2t = log2((double)p.rope_theta);
         inv_freq[lane] = exp2(-(double)lane / 64.0 * l2t);
@@ -575,32 +577,33 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_kc, const __grid_constan
             mbar_arrive(bar(D_O_FREE + ib));
             if (whole) {
                 // fold the one split with the sinks here (as decode_fold):
-                // M = max(sink log2e, B), L = 2^(sink log2e - M) + l 2^(B - M)
+                // M = max(sink log2e, B), L = 2^(sink log2e - M) + l 2^(B - M),
+                // out = O 2^(B - M) / L, lse = (M + log2 L) ln 2; the terms are
+                // within a factor 2^48 of each other, so the approximate
+                // exp2, log2 and reciprocal (relative error ~2^-22) suffice
 #pragma unroll
                 for (int hh = 0; hh < kGroup; ++hh) {
                     const int h = kGroup * it.g + hh;
-                    const float sink = p.sinks[h];
+                    const float sink = misc->sinks[h];
                     const float lh = misc->red_l[ib][0][hh] + misc->red_l[ib][1][hh] + misc->red_l[ib][2][hh] +
                                      misc->red_l[ib][3][hh];
-                    float M, L = 0.f, acc = 0.f;
+                    float ov = 0.f, v;
                     if (sink == INFINITY) {
-                        M = INFINITY;
+                        v = INFINITY;
                     } else {
-                        M = fmaxf(sink * 1.4426950408889634f, B);
-                        L = (sink > -INFINITY) ? exp2f(sink * 1.4426950408889634f - M) : 0.f;
-                        const float a = exp2f(B - M);
-                        L += lh * a;
-                        acc = __uint_as_float(o[hh]) * a;
+                        const float s2 = sink * 1.4426950408889634f;
+                        const float M = fmaxf(s2, B);
+                        const float a = dt_ex2(B - M);
+                        const float L = (sink > -INFINITY ? dt_ex2(s2 - M) : 0.f) + lh * a;
+                        if (L > 0.f) {
+                            ov = __uint_as_float(o[hh]) * (a * __frcp_rn(L));
+                            v = (M + __log2f(L)) * 0.6931471805599453f;
+                        } else {
+                            v = -INFINITY;
+                        }
                     }
-                    const float ov = (L > 0.f) ? acc / L : 0.f;
                     p.out[((size_t)it.b * kHQ + h) * kHD + r] = __float2bfloat16_rn(ov);
-                    if (r == 0 && p.lse) {
-                        float v;
-                        if (M == INFINITY) v = INFINITY;
-                        else if (L > 0.f) v = M * 0.6931471805599453f + logf(L);
-                        else v = -INFINITY;
-                        p.lse[(size_t)h * p.B + it.b] = v;
-                    }
+                    if (r == 0 && p.lse) p.lse[(size_t)h * p.B + it.b] = v;
                 }
             } else {
 #pragma unroll
