@@ -332,19 +332,28 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_adjoint_kernel(const BwdParam
 }
 
 // ---- fixed-order sums of the per-CTA partials
+// One warp per output (dq_norm_w[128], dk_norm_w[128], dsinks[32]): lane l
+// sums the partials b = l, l + 32, ... in order, then the lanes' sums meet in
+// a fixed shuffle tree, so every call adds in the same order.
+constexpr int kBwdFinishOutputs = kHD + kHD + kHQ;
 __global__ void bwd_finish_kernel(const BwdParams p, int grid_q, int grid_k) {
-    const int t = threadIdx.x;
-    if (t < kHD) {
-        float sq = 0.f, sk = 0.f;
-        for (int b = 0; b < grid_q; ++b) sq += p.part_q[(size_t)b * kBwdPartQ + t];
-        for (int b = 0; b < grid_k; ++b) sk += p.part_k[(size_t)b * kHD + t];
-        p.dq_norm_w[t] = sq;
-        p.dk_norm_w[t] = sk;
-    } else if (t < kHD + kHQ) {
-        float s = 0.f;
-        for (int b = 0; b < grid_q; ++b) s += p.part_q[(size_t)b * kBwdPartQ + t];
-        p.dsinks[t - kHD] = s;
+    const int w = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+    if (w >= kBwdFinishOutputs) return;
+    const float* src;
+    int n, stride;
+    float* dst;
+    if (w < kHD) {
+        src = p.part_q + w; n = grid_q; stride = kBwdPartQ; dst = p.dq_norm_w + w;
+    } else if (w < 2 * kHD) {
+        src = p.part_k + (w - kHD); n = grid_k; stride = kHD; dst = p.dk_norm_w + (w - kHD);
+    } else {
+        src = p.part_q + kHD + (w - 2 * kHD); n = grid_q; stride = kBwdPartQ; dst = p.dsinks + (w - 2 * kHD);
     }
+    float s = 0.f;
+    for (int b = lane; b < n; b += 32) s += src[(size_t)b * stride];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    if (lane == 0) *dst = s;
 }
 
 flint_status_t set_error(flint_status_t s, const char* msg);
@@ -441,7 +450,7 @@ flint_status_t run_bwd(const void* q, const void* k, const void* v, const float*
     bwd_adjoint_kernel<<<grid_a, kBwdThreads, 0, s>>>(bp);
     e = cudaGetLastError();
     if (e != cudaSuccess) return set_error(FLINT_ERR_CUDA, "backward: adjoint launch failed");
-    bwd_finish_kernel<<<1, kHD + kHQ, 0, s>>>(bp, grid_a, grid_a);
+    bwd_finish_kernel<<<(kBwdFinishOutputs + 7) / 8, 256, 0, s>>>(bp, grid_a, grid_a);
     e = cudaGetLastError();
     if (e != cudaSuccess) return set_error(FLINT_ERR_CUDA, "backward: finish launch failed");
     return FLINT_OK;
