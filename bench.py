@@ -211,6 +211,20 @@ class ClockSampler:
 
 # ---------------------------------------------------------------- flint arm
 
+def soak(args, work, sync):
+    """About args.soak seconds of untimed load while the clock sampler runs,
+    so that it records the clocks of the part under this workload (a timed
+    region of a few milliseconds ends before nvidia-smi's first sample)."""
+    if args.profile:
+        return
+    time.sleep(0.3)
+    t_end = time.time() + args.soak
+    while time.time() < t_end:
+        for _ in range(20):
+            work()
+        sync()
+
+
 def run_flint(args, rank, world, local_rank):
     import torch
     import torch.distributed as dist
@@ -495,6 +509,7 @@ def run_decode(args, rank, world, local_rank):
     sampler = ClockSampler(local_rank if "CUDA_VISIBLE_DEVICES" not in os.environ else
                            os.environ["CUDA_VISIBLE_DEVICES"].split(",")[local_rank])
     sampler.start()
+    soak(args, lambda: (flush.fill_(1), step()), lambda: torch.cuda.synchronize(dev))
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
     if world > 1:
         import torch.distributed as dist
@@ -614,6 +629,7 @@ def run_bwd(args, rank, world, local_rank):
     sampler = ClockSampler(local_rank if "CUDA_VISIBLE_DEVICES" not in os.environ else
                            os.environ["CUDA_VISIBLE_DEVICES"].split(",")[local_rank])
     sampler.start()
+    soak(args, lambda: (flush.fill_(1), call(d, grads)), lambda: torch.cuda.synchronize(dev))
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
     if world > 1:
         import torch.distributed as dist
@@ -753,6 +769,7 @@ def run_layer(args, rank, world, local_rank):
     sampler = ClockSampler(local_rank if "CUDA_VISIBLE_DEVICES" not in os.environ else
                            os.environ["CUDA_VISIBLE_DEVICES"].split(",")[local_rank])
     sampler.start()
+    soak(args, lambda: (flush.fill_(1), step()), lambda: torch.cuda.synchronize(dev))
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
     if world > 1:
         import torch.distributed as dist
