@@ -24,8 +24,10 @@
 // * Warps 4-7 take one slot row each: the score of each head is the sum of
 //   its hi and lo columns; with the running max started at the bound B
 //   (every term 2^(s - B) <= 1 and normal) no row max and no rescale are
-//   needed, so a split's partial is (m = B, l = sum of terms, O); the
-//   combine kernel folds the splits and the sink.
+//   needed, so a split's partial is (m = B, l = sum of terms, O).  An
+//   item's end (O^T out of TMEM, the output or the partial) waits until the
+//   next item's first tile is with the MMA, so the tiles of consecutive
+//   items follow each other without a wait for the last PV.
 // * Warps 2-3 prepare each item one ahead of the slot rows, into buffers of
 //   the item's parity: q~ (norm, RoPE) of 8 heads as the hi/lo rows of Q^T,
 //   the new token's k~ (FP32) and its scores against the 8 heads, and the
@@ -447,39 +449,111 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_kc, const __grid_constan
         const int wq = warp - 4;                        // this warp's slot of the l partial sums
         const uint32_t lb = (uint32_t)(warp & 3) * 32u;
         const float C = 1.4426950408889634f * 0.08838834764831845f;   // log2(e) / sqrt(128)
+        const bool whole = p.nsplit_tc == 1;            // every split is the whole window
         uint32_t sslot = 0, sph = 0, lph = 0, tt = 0, sst = 0, fph = 0, k_item = 0;
         uint32_t sfph[2] = {0u, 0u}, pfph[2] = {0u, 0u}, irph[2] = {0u, 0u}, oph[2] = {0u, 0u};
+        auto part_of = [&](int u, const DtItem& it) -> float* {
+            return p.part + (((size_t)it.b * kHKV + it.g) * p.nsplit_tc + (u % p.nsplit_tc)) * kPartFloats;
+        };
+        // this split's partial is written: the last split of (b, g) to
+        // finish folds them all into the output (bounded waits)
+        auto finish = [&](int b, int g) -> bool {
+            __threadfence();
+            mbar_arrive(bar(D_FOLD_A));
+            if (!__all_sync(0xffffffffu, mbar_wait(bar(D_FOLD_A), fph, abort_flag, status))) return false;
+            if (tid == 128) misc->last = atomicAdd(p.arrive + b * kHKV + g, 1) == p.nsplit_tc - 1;
+            mbar_arrive(bar(D_FOLD_B));
+            if (!__all_sync(0xffffffffu, mbar_wait(bar(D_FOLD_B), fph, abort_flag, status))) return false;
+            fph ^= 1;
+            if (misc->last) {
+                __threadfence();
+                decode_fold(p, b, g, p.nsplit_tc, r);
+            }
+            return true;
+        };
+        // The end of an item whose tiles are done and whose l sits in
+        // red_l[pib]: O^T out of TMEM once the item's last PV completed, then
+        // the output (a split that is the whole window) or the partial and
+        // the fold.  It runs once the next item's first tile is with the
+        // MMA, by when those PV MMAs have long completed: the slot rows do
+        // not wait for them between items.
+        bool pending = false;
+        DtItem pit = {};
+        int pu = 0;
+        uint32_t pib = 0;
+        auto end_item = [&]() -> bool {
+            pending = false;
+            float* part = part_of(pu, pit);
+            if (!whole && warp == 4 && lane < kGroup) {
+                part[lane] = B;
+                part[kGroup + lane] = misc->red_l[pib][0][lane] + misc->red_l[pib][1][lane] +
+                                      misc->red_l[pib][2][lane] + misc->red_l[pib][3][lane];
+            }
+            // O^T: TMEM lane = channel r, columns 0..7 = heads
+            if (!__all_sync(0xffffffffu, mbar_wait(bar(D_O_FULL + pib), oph[pib], abort_flag, status))) return false;
+            oph[pib] ^= 1u;
+            tc_fence_after();
+            uint32_t o[16];
+            tmem_ld16(tmem + (lb << 16) + 64u + 32u * pib, o);
+            tmem_wait_ld();
+            tc_fence_before();
+            mbar_arrive(bar(D_O_FREE + pib));
+            if (whole) {
+                // fold the one split with the sinks here (as decode_fold):
+                // M = max(sink log2e, B), L = 2^(sink log2e - M) + l 2^(B - M),
+                // out = O 2^(B - M) / L, lse = (M + log2 L) ln 2; the terms are
+                // within a factor 2^48 of each other, so the approximate
+                // exp2, log2 and reciprocal (relative error ~2^-22) suffice
+#pragma unroll
+                for (int hh = 0; hh < kGroup; ++hh) {
+                    const int h = kGroup * pit.g + hh;
+                    const float sink = misc->sinks[h];
+                    const float lh = misc->red_l[pib][0][hh] + misc->red_l[pib][1][hh] + misc->red_l[pib][2][hh] +
+                                     misc->red_l[pib][3][hh];
+                    float ov = 0.f, v;
+                    if (sink == INFINITY) {
+                        v = INFINITY;
+                    } else {
+                        const float s2 = sink * 1.4426950408889634f;
+                        const float M = fmaxf(s2, B);
+                        const float a = dt_ex2(B - M);
+                        const float L = (sink > -INFINITY ? dt_ex2(s2 - M) : 0.f) + lh * a;
+                        if (L > 0.f) {
+                            ov = __uint_as_float(o[hh]) * (a * __frcp_rn(L));
+                            v = (M + __log2f(L)) * 0.6931471805599453f;
+                        } else {
+                            v = -INFINITY;
+                        }
+                    }
+                    p.out[((size_t)pit.b * kHQ + h) * kHD + r] = __float2bfloat16_rn(ov);
+                    if (r == 0 && p.lse) p.lse[(size_t)h * p.B + pit.b] = v;
+                }
+                return true;
+            }
+#pragma unroll
+            for (int h = 0; h < kGroup; ++h) part[2 * kGroup + h * kHD + r] = __uint_as_float(o[h]);
+            return finish(pit.b, pit.g);
+        };
+        bool done = false;                              // the scheduler's end, not a failed wait
         for (;;) {
             if (!__all_sync(0xffffffffu, mbar_wait(bar(D_SCHED_FULL + sslot), sph, abort_flag, status))) break;
             const int u = misc->sched[sslot];
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(D_SCHED_EMPTY + sslot));
             sslot ^= 1; if (sslot == 0) sph ^= 1;
-            if (u < 0) break;
+            if (u < 0) {
+                done = true;
+                break;
+            }
             const DtItem it = dt_item(p, u);
-            float* part = p.part + (((size_t)it.b * kHKV + it.g) * p.nsplit_tc + (u % p.nsplit_tc)) * kPartFloats;
             int nl = 0;
             for (int t = it.t0; t < it.t1; ++t) nl += dt_tile_live(p, it, t) ? 1 : 0;
             if (it.bad && tid == 128) atomicCAS(status, 0, 1 /* FLINT_ERR_INVALID_ARG */);
-            // this split's partial is written: the last split of (b, g) to
-            // finish folds them all into the output (bounded waits)
-            auto finish = [&]() -> bool {
-                __threadfence();
-                mbar_arrive(bar(D_FOLD_A));
-                if (!__all_sync(0xffffffffu, mbar_wait(bar(D_FOLD_A), fph, abort_flag, status))) return false;
-                if (tid == 128) misc->last = atomicAdd(p.arrive + it.b * kHKV + it.g, 1) == p.nsplit_tc - 1;
-                mbar_arrive(bar(D_FOLD_B));
-                if (!__all_sync(0xffffffffu, mbar_wait(bar(D_FOLD_B), fph, abort_flag, status))) return false;
-                fph ^= 1;
-                if (misc->last) {
-                    __threadfence();
-                    decode_fold(p, it.b, it.g, p.nsplit_tc, r);
-                }
-                return true;
-            };
             if (nl == 0) {
+                if (pending && !end_item()) break;
+                float* part = part_of(u, it);
                 if (warp == 4 && lane < kGroup) { part[lane] = -INFINITY; part[kGroup + lane] = 0.f; }
-                if (!finish()) break;
+                if (!finish(it.b, it.g)) break;
                 continue;
             }
             const int s_new = it.pos % p.cap;
@@ -543,13 +617,19 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_kc, const __grid_constan
                 mbar_arrive(bar(D_P_READY + sb));
                 ++tt;
                 if (++sst == kDtStages) sst = 0;
+                // the previous item's end, now that this item's first tile
+                // is with the MMA
+                if (pending && !end_item()) {
+                    alive = false;
+                    break;
+                }
             }
             if (!alive) break;
             // the item's Q^T and scores are no longer read: the query warps
             // may fill this parity's buffers for the item after next
             mbar_arrive(bar(D_ITEM_DONE + ib));
             // ---- l over the split's slots, per head: warp sums, then the
-            // four warps' sums
+            // four warps' sums (read at the item's end)
 #pragma unroll
             for (int h = 0; h < kGroup; ++h) {
                 float x = l[h];
@@ -560,57 +640,13 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_kc, const __grid_constan
             mbar_arrive(bar(D_L_READY));
             if (!__all_sync(0xffffffffu, mbar_wait(bar(D_L_READY), lph, abort_flag, status))) break;
             lph ^= 1;
-            const bool whole = p.nsplit_tc == 1;   // this split is the whole window
-            if (!whole && warp == 4 && lane < kGroup) {
-                part[lane] = B;
-                part[kGroup + lane] = misc->red_l[ib][0][lane] + misc->red_l[ib][1][lane] +
-                                      misc->red_l[ib][2][lane] + misc->red_l[ib][3][lane];
-            }
-            // O^T: TMEM lane = channel r, columns 0..7 = heads
-            if (!__all_sync(0xffffffffu, mbar_wait(bar(D_O_FULL + ib), oph[ib], abort_flag, status))) break;
-            oph[ib] ^= 1u;
-            tc_fence_after();
-            uint32_t o[16];
-            tmem_ld16(tmem + (lb << 16) + 64u + 32u * ib, o);
-            tmem_wait_ld();
-            tc_fence_before();
-            mbar_arrive(bar(D_O_FREE + ib));
-            if (whole) {
-                // fold the one split with the sinks here (as decode_fold):
-                // M = max(sink log2e, B), L = 2^(sink log2e - M) + l 2^(B - M),
-                // out = O 2^(B - M) / L, lse = (M + log2 L) ln 2; the terms are
-                // within a factor 2^48 of each other, so the approximate
-                // exp2, log2 and reciprocal (relative error ~2^-22) suffice
-#pragma unroll
-                for (int hh = 0; hh < kGroup; ++hh) {
-                    const int h = kGroup * it.g + hh;
-                    const float sink = misc->sinks[h];
-                    const float lh = misc->red_l[ib][0][hh] + misc->red_l[ib][1][hh] + misc->red_l[ib][2][hh] +
-                                     misc->red_l[ib][3][hh];
-                    float ov = 0.f, v;
-                    if (sink == INFINITY) {
-                        v = INFINITY;
-                    } else {
-                        const float s2 = sink * 1.4426950408889634f;
-                        const float M = fmaxf(s2, B);
-                        const float a = dt_ex2(B - M);
-                        const float L = (sink > -INFINITY ? dt_ex2(s2 - M) : 0.f) + lh * a;
-                        if (L > 0.f) {
-                            ov = __uint_as_float(o[hh]) * (a * __frcp_rn(L));
-                            v = (M + __log2f(L)) * 0.6931471805599453f;
-                        } else {
-                            v = -INFINITY;
-                        }
-                    }
-                    p.out[((size_t)it.b * kHQ + h) * kHD + r] = __float2bfloat16_rn(ov);
-                    if (r == 0 && p.lse) p.lse[(size_t)h * p.B + it.b] = v;
-                }
-            } else {
-#pragma unroll
-                for (int h = 0; h < kGroup; ++h) part[2 * kGroup + h * kHD + r] = __uint_as_float(o[h]);
-                if (!finish()) break;
-            }
+            pending = true;
+            pit = it;
+            pu = u;
+            pib = ib;
         }
+        // the last item's end
+        if (done && pending) end_item();
     }
     tc_fence_before();
     __syncthreads();
