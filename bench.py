@@ -563,9 +563,9 @@ def decode_line(args, world, d, total_ms, clocks):
                     keys=int(d.keys_per_sequence().sum()), l2="flushed before every timed step (256 MiB write)",
                     per_rank="independent replica"),
         roofline=dict(bound="hbm", achieved=round(gbs, 3), peak=peak, unit="GB/s", frac=round(gbs / peak, 4),
-                      traffic=None, kernel="flint::decode_tc_kernel + decode_split_kernel (whole step; one of them returns at once)",
+                      traffic=None, kernel="flint::decode_tc_kernel (whole step: reset kernel, tile kernel, CUDA-core kernel returning at once)",
                       peak_source="%s hbm_gbs" % src, bytes_per_step=nbytes),
-        gpu_launches=2 * args.steps, clocks=clocks)
+        gpu_launches=3 * args.steps, clocks=clocks)
 
 
 # ---------------------------------------------------------------- backward leg

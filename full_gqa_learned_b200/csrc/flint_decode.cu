@@ -57,6 +57,9 @@ decode_split_kernel(const DecodeParams p) {
         const float bnd = decode_logit_bound(p.q_norm_w, p.k_norm_w);
         if (bnd <= kDecodeBoundMax) return;
     }
+    // launched as a programmatic dependent of the tile kernel (which waited
+    // for the header reset before it returned): everything below comes after
+    griddep_wait();
     // CTA (loop over items (s, g, b)): keys lo + 256 s .. of KV head g of
     // sequence b; the last split of (b, g) to finish folds all of them
     auto run_item = [&](const int s, const int g, const int b) {
@@ -240,6 +243,15 @@ decode_split_kernel(const DecodeParams p) {
 
 flint_status_t set_error(flint_status_t s, const char* msg);
 
+// Zeroes the status word, the tile kernel's work counter and the
+// split-arrival counters of one call.  The tile kernel is launched as its
+// programmatic dependent: its setup overlaps this, and it waits for this
+// grid before it touches those words.
+__global__ void decode_zero_kernel(int* hdr, int n_words) {
+    griddep_launch_dependents();
+    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n_words; i += gridDim.x * blockDim.x) hdr[i] = 0;
+}
+
 size_t decode_nsplit(int cap, int window) {
     const int nmax = window > 0 ? (window < cap ? window : cap) : cap;
     return (size_t)((nmax + kDecKeys - 1) / kDecKeys);
@@ -283,12 +295,17 @@ flint_status_t run_decode(const void* q, const void* k, const void* v, const flo
     (void)workspace_bytes;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     // status word, the tile kernel's work counter, the split-arrival counters
-    cudaError_t e = cudaMemsetAsync(workspace, 0, decode_header_bytes(B), s);
+    const int hdr_words = (int)(decode_header_bytes(B) / sizeof(int));
+    const int zgrid = (hdr_words + 255) / 256 < 64 ? (hdr_words + 255) / 256 : 64;
+    decode_zero_kernel<<<zgrid, 256, 0, s>>>(dp.status, hdr_words);
+    cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return set_error(FLINT_ERR_CUDA, "decode: status reset failed");
-    // Both kernels are enqueued; each decides from the norm weights whether
-    // it runs (the tile kernel under a logit bound <= 48) and the other
-    // returns at once.  Each writes the output itself (the last split of a
-    // sequence and KV head folds them all).
+    // Both kernels are enqueued, each a programmatic dependent of the launch
+    // before it, so their launches and setup overlap the work ahead of them;
+    // each decides from the norm weights whether it runs (the tile kernel
+    // under a logit bound <= 48) and the other returns at once.  Each writes
+    // the output itself (the last split of a sequence and KV head folds them
+    // all).
     int sms = 0, dev = 0;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
@@ -299,8 +316,17 @@ flint_status_t run_decode(const void* q, const void* k, const void* v, const flo
     const long long items = (long long)dp.nsplit * kHKV * B;
     const long long cap_grid = 2LL * (sms > 0 ? sms : 1);
     const int grid = (int)(items < cap_grid ? items : cap_grid);
-    decode_split_kernel<<<grid, kDecThreads, 0, s>>>(dp);
-    e = cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kDecThreads);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, decode_split_kernel, dp);
     if (e != cudaSuccess) return set_error(FLINT_ERR_CUDA, "decode: split launch failed");
     return FLINT_OK;
 }

@@ -153,6 +153,9 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_kc, const __grid_constan
     int* counter = p.status + 1;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int n_items = p.B * kHKV * p.nsplit_tc;
+    // The CUDA-core split kernel behind this one may be scheduled now: it
+    // reads the weights and returns, or waits for this grid.
+    griddep_launch_dependents();
 
     // this kernel runs only under a logit bound <= 48; otherwise the
     // CUDA-core split kernel does the step (every CTA decides the same way)
@@ -161,7 +164,12 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_kc, const __grid_constan
         if (lane == 0) misc->bound = bnd;
     }
     __syncthreads();
-    if (!(misc->bound <= kDecodeBoundMax)) return;
+    if (!(misc->bound <= kDecodeBoundMax)) {
+        // the split kernel waits for this grid only: this grid's end must
+        // come after the header reset
+        griddep_wait();
+        return;
+    }
 
     if (tid == 0) {
         for (uint32_t s = 0; s < kDtStages; ++s) {
@@ -207,6 +215,9 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_kc, const __grid_constan
         if (row >= 8) *reinterpret_cast<uint4*>(smem + kDtOffP + o) = make_uint4(0u, 0u, 0u, 0u);
     }
     fence_proxy_async_smem();
+    // the status word, the work counter and the split-arrival counters are
+    // read and written only after the reset kernel before this one completed
+    griddep_wait();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -680,8 +691,8 @@ flint_status_t dt_map(EncodeTiledFn enc, CUtensorMap* m, const void* base, int B
 }  // namespace
 
 // Enqueues the tensor-core decode kernel (a no-op when the logit bound is
-// above 48).  The status word and the unit counter after it are zeroed by
-// the caller.
+// above 48) as a programmatic dependent of the kernel that zeroes the status
+// word, the unit counter after it and the split-arrival counters.
 flint_status_t launch_decode_tc(const DecodeParams& p, int sms, cudaStream_t s) {
     int dev = 0;
     cudaGetDevice(&dev);
@@ -701,8 +712,17 @@ flint_status_t launch_decode_tc(const DecodeParams& p, int sms, cudaStream_t s) 
     if (st != FLINT_OK) return st;
     const long long items = (long long)p.B * kHKV * p.nsplit_tc;
     const int grid = (int)(items < sms ? items : sms);
-    decode_tc_kernel<<<grid, kDtThreads, kDtSmem, s>>>(tk, tv, p);
-    cudaError_t e = cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kDtThreads);
+    cfg.dynamicSmemBytes = kDtSmem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, decode_tc_kernel, tk, tv, p);
     if (e != cudaSuccess) return fail(FLINT_ERR_CUDA, "decode (tensor cores) launch: %s", cudaGetErrorString(e));
     return FLINT_OK;
 }

@@ -342,8 +342,9 @@ FLINT_API flint_status_t flint_attn_fwd_static_status(void* stream);
  * product; splits of up to 8 tiles per (sequence, KV head), the last split
  * to finish folding them with the sink.  Otherwise queries, keys and scores
  * are computed in FP32 on CUDA cores over splits of 256 positions, folded
- * the same way.  One call launches both kernels; the one not taken returns
- * at once.
+ * the same way.  One call launches a small kernel that resets the status
+ * and counters in the workspace, then both kernels (each a programmatic
+ * dependent of the launch before it); the one not taken returns at once.
  */
 FLINT_API size_t flint_attn_decode_workspace_bytes(int32_t B, int32_t cap, int32_t window);
 FLINT_API flint_status_t flint_attn_decode(const void* q, const void* k, const void* v,
