@@ -81,12 +81,14 @@ enum : uint32_t {
 
 struct DtMisc {
     int sched[2];
+    int sched_pos[2];                   // the scheduled item's position (cache_len of its sequence)
     uint32_t tmem_base;
     int abort_flag;
     float bound;                        // B, log2 units
     float s_new[2][8];                  // per item parity: the new token's scores, per head (unscaled)
     float red_l[2][4][8];               // per item parity and slot-row warp: its part of l, per head
     int last;                           // this split is the last of its (b, g) to finish
+    int first_pos;                      // the first item's position (read early, for its cache line)
     float sinks[kHQ];                   // the learned sinks
 };
 static_assert(sizeof(DtMisc) <= 512, "misc block");
@@ -98,7 +100,7 @@ struct DtItem {
     bool bad;                           // ill-formed position or window
 };
 
-__device__ __forceinline__ DtItem dt_item(const DecodeParams& p, int i) {
+__device__ __forceinline__ DtItem dt_item(const DecodeParams& p, int i, int pos) {
     DtItem it;
     const int ns = p.nsplit_tc;
     it.b = i / (kHKV * ns);
@@ -107,7 +109,7 @@ __device__ __forceinline__ DtItem dt_item(const DecodeParams& p, int i) {
     const int nt = decode_tc_tiles(p.cap), per = decode_tc_tiles_per_split(p.cap);
     it.t0 = sp * per;
     it.t1 = min(nt, it.t0 + per);
-    it.pos = p.cache_len[it.b];
+    it.pos = pos;
     it.lo = p.window > 0 ? max(0, it.pos - p.window + 1) : 0;
     it.n = it.pos - it.lo + 1;
     it.bad = it.pos < 0 || it.pos >= FLINT_MAX_TOKENS || it.n > p.cap;
@@ -156,6 +158,17 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_kc, const __grid_constan
     // The CUDA-core split kernel behind this one may be scheduled now: it
     // reads the weights and returns, or waits for this grid.
     griddep_launch_dependents();
+    // Each CTA's first item is its own index (later ones come from the
+    // counter), so its rows can be on their way to L2 before every CTA's
+    // first cache tiles fill the memory queues: the query warps' loads of
+    // them would otherwise wait behind those.
+    if (warp == 2 && lane == 0 && (int)blockIdx.x < n_items) {
+        const int fb = (int)blockIdx.x / (kHKV * p.nsplit_tc), fg = ((int)blockIdx.x / p.nsplit_tc) % kHKV;
+        bulk_prefetch_l2(p.q + ((size_t)fb * kHQ + kGroup * fg) * kHD, kGroup * kHD * 2);
+        bulk_prefetch_l2(p.k + ((size_t)fb * kHKV + fg) * kHD, kHD * 2);
+        bulk_prefetch_l2(p.v + ((size_t)fb * kHKV + fg) * kHD, kHD * 2);
+        misc->first_pos = p.cache_len[fb];    // its line, too
+    }
 
     // this kernel runs only under a logit bound <= 48; otherwise the
     // CUDA-core split kernel does the step (every CTA decides the same way)
@@ -230,21 +243,27 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_kc, const __grid_constan
             uint32_t sslot = 0, sph = 0, st = 0, ph = 0, narm = 0;
             // items are published one ahead of the item being loaded, so the
             // query warps prepare the next item while this one streams
-            auto publish = [&](int v) -> bool {
+            // with the item, its position: the consumers take it from here
+            // instead of each reading cache_len at every item change
+            auto publish = [&](int v, int vpos) -> bool {
                 if (!mbar_wait(bar(D_SCHED_EMPTY + sslot), sph ^ 1, abort_flag, status)) return false;
                 misc->sched[sslot] = v;
+                misc->sched_pos[sslot] = vpos;
                 mbar_arrive(bar(D_SCHED_FULL + sslot));
                 sslot ^= 1; if (sslot == 0) sph ^= 1;
                 return true;
             };
-            int u = atomicAdd(counter, 1);
-            if (u >= n_items) u = -1;
-            bool pub = publish(u);
+            // the first item is the CTA's index; the counter hands out the
+            // rest, from gridDim.x on
+            int u = (int)blockIdx.x < n_items ? (int)blockIdx.x : -1;
+            int upos = u >= 0 ? p.cache_len[u / (kHKV * p.nsplit_tc)] : 0;
+            bool pub = publish(u, upos);
             for (; pub;) {
                 if (u < 0) break;
-                int un = atomicAdd(counter, 1);
+                int un = atomicAdd(counter, 1) + (int)gridDim.x;
                 if (un >= n_items) un = -1;
-                if (!publish(un)) break;
+                const int unpos = un >= 0 ? p.cache_len[un / (kHKV * p.nsplit_tc)] : 0;
+                if (!publish(un, unpos)) break;
                 if (un >= 0) {
                     // the next item's q, k and v rows into L2 (its prologue reads them)
                     const int nb = un / (kHKV * p.nsplit_tc), ng = (un / p.nsplit_tc) % kHKV;
@@ -252,7 +271,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_kc, const __grid_constan
                     bulk_prefetch_l2(p.k + ((size_t)nb * kHKV + ng) * kHD, kHD * 2);
                     bulk_prefetch_l2(p.v + ((size_t)nb * kHKV + ng) * kHD, kHD * 2);
                 }
-                const DtItem it = dt_item(p, u);
+                const DtItem it = dt_item(p, u, upos);
                 bool ok = true;
                 for (int t = it.t0; t < it.t1 && ok; ++t) {
                     if (!dt_tile_live(p, it, t)) continue;
@@ -270,6 +289,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_kc, const __grid_constan
                 }
                 if (!ok) break;
                 u = un;
+                upos = unpos;
             }
             // drain: every armed load has landed before shared memory is released
             volatile int never = 0;
@@ -304,11 +324,11 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_kc, const __grid_constan
             };
             for (; ok;) {
                 if (!mbar_wait(bar(D_SCHED_FULL + sslot), sph, abort_flag, status)) break;
-                const int u = misc->sched[sslot];
+                const int u = misc->sched[sslot], upos = misc->sched_pos[sslot];
                 mbar_arrive(bar(D_SCHED_EMPTY + sslot));
                 sslot ^= 1; if (sslot == 0) sph ^= 1;
                 if (u < 0) break;
-                const DtItem it = dt_item(p, u);
+                const DtItem it = dt_item(p, u, upos);
                 int nl = 0;
                 for (int t = it.t0; t < it.t1; ++t) nl += dt_tile_live(p, it, t) ? 1 : 0;
                 if (nl == 0) continue;
@@ -395,12 +415,12 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_kc, const __grid_constan
         uint32_t idph[2] = {0u, 0u};
         for (;;) {
             if (!__all_sync(0xffffffffu, mbar_wait(bar(D_SCHED_FULL + sslot), sph, abort_flag, status))) break;
-            const int u = misc->sched[sslot];
+            const int u = misc->sched[sslot], upos = misc->sched_pos[sslot];
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(D_SCHED_EMPTY + sslot));
             sslot ^= 1; if (sslot == 0) sph ^= 1;
             if (u < 0) break;
-            const DtItem it = dt_item(p, u);
+            const DtItem it = dt_item(p, u, upos);
             int nl = 0;
             for (int t = it.t0; t < it.t1; ++t) nl += dt_tile_live(p, it, t) ? 1 : 0;
             if (nl == 0) continue;
@@ -548,7 +568,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_kc, const __grid_constan
         bool done = false;                              // the scheduler's end, not a failed wait
         for (;;) {
             if (!__all_sync(0xffffffffu, mbar_wait(bar(D_SCHED_FULL + sslot), sph, abort_flag, status))) break;
-            const int u = misc->sched[sslot];
+            const int u = misc->sched[sslot], upos = misc->sched_pos[sslot];
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(D_SCHED_EMPTY + sslot));
             sslot ^= 1; if (sslot == 0) sph ^= 1;
@@ -556,7 +576,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_kc, const __grid_constan
                 done = true;
                 break;
             }
-            const DtItem it = dt_item(p, u);
+            const DtItem it = dt_item(p, u, upos);
             int nl = 0;
             for (int t = it.t0; t < it.t1; ++t) nl += dt_tile_live(p, it, t) ? 1 : 0;
             if (it.bad && tid == 128) atomicCAS(status, 0, 1 /* FLINT_ERR_INVALID_ARG */);
