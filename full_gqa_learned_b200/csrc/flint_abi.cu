@@ -300,7 +300,8 @@ flint_status_t run_stages(int stages, const void* q, const void* k, const void* 
     pp.rope_theta = rope_theta;
     pp.eps = eps;
     // ws_layout is always evaluated with max(nseg, 1) segments
-    int prep_blocks = 1 + (T + 31) / 32;
+    const long long prep_warps = (long long)T * prep_parts(T, f16 || qprep);
+    int prep_blocks = (int)(1 + (prep_warps + 31) / 32 < 1 + 4LL * sms ? 1 + (prep_warps + 31) / 32 : 1 + 4LL * sms);
     if (prep_blocks > 1 + 4 * sms) prep_blocks = 1 + 4 * sms;
     if (prep_blocks < 2) prep_blocks = 2;
     if (stages & kStagePrepare) {

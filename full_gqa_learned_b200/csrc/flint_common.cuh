@@ -110,6 +110,14 @@ __device__ __forceinline__ void rope_cos_sin(int pos, double inv_freq, float* c,
     __sincosf((float)r, s, c);
 }
 
+// Warps per token in the preparation kernel: a call of at most 2,048 tokens
+// that also prepares queries gives each token 1 + 8 warps (its keys, then
+// its query heads four at a time), so that enough loads are in flight; one
+// warp per token otherwise.
+__host__ __device__ inline int prep_parts(int T, bool queries) {
+    return (queries && T <= 2048) ? 1 + kHQ / kHKV : 1;
+}
+
 // Stages of one forward call (host side).
 enum Stage : int {
     kStagePrepare = 1, kStageAttend = 2, kStageBoth = 3,

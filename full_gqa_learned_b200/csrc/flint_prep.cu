@@ -288,11 +288,21 @@ __device__ void prepare_tokens(const PrepParams& p) {
     const int nwarps_total = (gridDim.x - 1) * (blockDim.x >> 5);
     const float kscale = s_kscale;
     const bool rope = p.use_rope != 0;
-    for (int t = (blockIdx.x - 1) * (blockDim.x >> 5) + warp; t < p.T; t += nwarps_total) {
+    // A call of few tokens that also prepares queries spreads each token over
+    // 1 + 8 warps (its keys, then its query heads four at a time), so that
+    // enough loads are in flight; otherwise one warp takes a token, and its
+    // RoPE table serves all of the token's heads.
+    const int nparts = prep_parts(p.T, p.f16 || p.qprep);
+    const int nwork = p.T * nparts;               // at most 2,048 x 9, or T
+    for (int wi = (blockIdx.x - 1) * (blockDim.x >> 5) + warp; wi < nwork; wi += nwarps_total) {
+        const int t = nparts == 1 ? wi : wi / nparts, part = nparts == 1 ? 0 : wi - t * nparts;
+        // query passes hq0 .. hq1 - 1 of this warp (4 heads each); the keys
+        // and the padded-row outputs go with part 0
+        const int hq0 = nparts == 1 ? 0 : (part > 0 ? part - 1 : 0), hq1 = nparts == 1 ? kHQ / kHKV : part;
         // ---- the lane's 8 (cos, sin) pairs f = 8*sub + e at the token's
         // document-local position, shared by its 4 key heads
         float cc[8], sn[8];
-        if (rope && (p.f16 || p.qprep || !p.keys_ready)) {
+        if (rope && (p.f16 || p.qprep || (!p.keys_ready && part == 0))) {
             int pos;
             if (p.pos_ids) pos = p.pos_ids[t];
             else if (p.mode == kMaskThd) pos = t - (t < s_thd_end ? thd_segment_start(p.cu_seqlens, p.nseg, t) : s_thd_end);
@@ -316,11 +326,11 @@ __device__ void prepare_tokens(const PrepParams& p) {
         // lanes past the slice normalise a valid row and store nothing.
         const bool kstore = head < p.ng;
         const size_t krow = ((size_t)t * p.ng + (kstore ? head : 0)) * kHD;
-        if (p.f16)
+        if (part == 0 && p.f16)
             norm_rope_row(p.kf + krow, kn + krow, s_wk, p.eps, kscale, sub, rope, cc, sn, kstore);
-        else if (!p.keys_ready)
+        else if (part == 0 && !p.keys_ready)
             norm_rope_row(p.k + krow, kn + krow, s_wk, p.eps, kscale, sub, rope, cc, sn, kstore);
-        if (p.f16) {
+        if (part == 0 && p.f16) {
             // FP16 policy: the values cast to FP16 (4 heads x 128 per token,
             // 16 per lane)
             __half* vh = reinterpret_cast<__half*>(p.ws + L.vh) + (size_t)t * kHKV * kHD;
@@ -339,6 +349,7 @@ __device__ void prepare_tokens(const PrepParams& p) {
         else if (p.mode == kMaskPad) padded = p.pad_mask[t] == 0;
         else padded = false;
         if (padded) {
+            if (part != 0) continue;
             // ---- padded query token: zero output row, lse = sink
             uint4 z = make_uint4(0, 0, 0, 0);
             const int nh = kGroup * p.ng;                  // query heads in the tensors
@@ -352,7 +363,7 @@ __device__ void prepare_tokens(const PrepParams& p) {
             const float* qrow = p.qf + (size_t)t * kHQ * kHD;
             __half* qdst = reinterpret_cast<__half*>(p.ws + L.qn) + (size_t)t * kHQ * kHD;
 #pragma unroll 2
-            for (int hq = 0; hq < kHQ / kHKV; ++hq) {
+            for (int hq = hq0; hq < hq1; ++hq) {
                 const int hh = kHKV * hq + head;
                 norm_rope_row(qrow + hh * kHD, qdst + hh * kHD, s_wq, p.eps, s_qscale, sub, rope, cc, sn);
             }
@@ -366,7 +377,7 @@ __device__ void prepare_tokens(const PrepParams& p) {
             const __nv_bfloat16* qrow = p.q + (size_t)t * nh * kHD;
             __half* qdst = reinterpret_cast<__half*>(p.out + (size_t)t * nh * kHD);
 #pragma unroll 2
-            for (int hq = 0; hq < kGroup; ++hq) {
+            for (int hq = hq0; hq < hq1; ++hq) {
                 const int hh = kHKV * hq + head;
                 const bool qstore = hh < nh;
                 const int hs = qstore ? hh : 0;
