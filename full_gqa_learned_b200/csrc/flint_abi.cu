@@ -20,6 +20,7 @@
 #include "flint_host.cuh"
 
 namespace flint {
+template <bool kSplit>
 __global__ void prep_kernel(PrepParams p);
 __global__ void attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q,
                                 const __grid_constant__ CUtensorMap tm_k,
@@ -300,12 +301,16 @@ flint_status_t run_stages(int stages, const void* q, const void* k, const void* 
     pp.rope_theta = rope_theta;
     pp.eps = eps;
     // ws_layout is always evaluated with max(nseg, 1) segments
+    const bool prep_split = prep_parts(T, f16 || qprep) > 1;
     const long long prep_warps = (long long)T * prep_parts(T, f16 || qprep);
     int prep_blocks = (int)(1 + (prep_warps + 31) / 32 < 1 + 4LL * sms ? 1 + (prep_warps + 31) / 32 : 1 + 4LL * sms);
     if (prep_blocks > 1 + 4 * sms) prep_blocks = 1 + 4 * sms;
     if (prep_blocks < 2) prep_blocks = 2;
     if (stages & kStagePrepare) {
-        prep_kernel<<<prep_blocks, 1024, 0, s>>>(pp);
+        if (prep_split)
+            prep_kernel<true><<<prep_blocks, 1024, 0, s>>>(pp);
+        else
+            prep_kernel<false><<<prep_blocks, 1024, 0, s>>>(pp);
         e = cudaGetLastError();
         if (e != cudaSuccess) return fail(FLINT_ERR_CUDA, "prep launch: %s", cudaGetErrorString(e));
     }

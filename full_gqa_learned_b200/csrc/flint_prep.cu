@@ -261,6 +261,9 @@ __device__ __forceinline__ void norm_rope_row(const In* src, __half* dst, const 
     }
 }
 
+// kSplit: the call spreads each token over prep_parts() warps (small calls
+// that prepare queries); otherwise one warp takes each token.
+template <bool kSplit>
 __device__ void prepare_tokens(const PrepParams& p) {
     __shared__ double s_inv_freq[64];
     __shared__ float s_wk[kHD], s_wq[kHD];
@@ -292,13 +295,13 @@ __device__ void prepare_tokens(const PrepParams& p) {
     // 1 + 8 warps (its keys, then its query heads four at a time), so that
     // enough loads are in flight; otherwise one warp takes a token, and its
     // RoPE table serves all of the token's heads.
-    const int nparts = prep_parts(p.T, p.f16 || p.qprep);
+    const int nparts = kSplit ? prep_parts(p.T, true) : 1;
     const int nwork = p.T * nparts;               // at most 2,048 x 9, or T
     for (int wi = (blockIdx.x - 1) * (blockDim.x >> 5) + warp; wi < nwork; wi += nwarps_total) {
-        const int t = nparts == 1 ? wi : wi / nparts, part = nparts == 1 ? 0 : wi - t * nparts;
+        const int t = kSplit ? wi / nparts : wi, part = kSplit ? wi - t * nparts : 0;
         // query passes hq0 .. hq1 - 1 of this warp (4 heads each); the keys
         // and the padded-row outputs go with part 0
-        const int hq0 = nparts == 1 ? 0 : (part > 0 ? part - 1 : 0), hq1 = nparts == 1 ? kHQ / kHKV : part;
+        const int hq0 = kSplit ? (part > 0 ? part - 1 : 0) : 0, hq1 = kSplit ? part : kHQ / kHKV;
         // ---- the lane's 8 (cos, sin) pairs f = 8*sub + e at the token's
         // document-local position, shared by its 4 key heads
         float cc[8], sn[8];
@@ -387,6 +390,7 @@ __device__ void prepare_tokens(const PrepParams& p) {
     }
 }
 
+template <bool kSplit>
 __global__ void __launch_bounds__(1024, 1) prep_kernel(PrepParams p) {
     // The attention kernel may be scheduled as soon as every block of this
     // grid has started (it is launched as a programmatic dependent and waits
@@ -395,7 +399,9 @@ __global__ void __launch_bounds__(1024, 1) prep_kernel(PrepParams p) {
     // an SM, no block of this grid is still waiting for one.
     griddep_launch_dependents();
     if (blockIdx.x == 0) build_plan(p);
-    else prepare_tokens(p);
+    else prepare_tokens<kSplit>(p);
 }
+template __global__ void prep_kernel<false>(PrepParams);
+template __global__ void prep_kernel<true>(PrepParams);
 
 }  // namespace flint
