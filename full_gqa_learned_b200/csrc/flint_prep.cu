@@ -11,10 +11,13 @@
 // RMSNorm with k_norm_w (weight form; HF discussion #26 on RecursiveSI/flint),
 // then on sliding layers NeoX RoPE at the document-local position
 // (FlintAttention._apply_rope), scaled by a power of two and rounded to FP16
-// into the workspace.  Queries are used by one tile only; the attention kernel
-// normalises and rotates them itself.  Padded query tokens get their final
-// outputs here: zeros and lse = sink (FlintAttention.forward, attention_mask:
-// the sink remains valid for padded queries).
+// into the workspace.  Queries are used by one tile only: on full layers the
+// attention kernel normalises and rotates them itself; on sliding layers
+// (units of ~5 chunks, too short to hide that prologue) these blocks do it,
+// into the token's own output rows as FP16, and on calls of at most 2,048
+// tokens they spread each token over nine warps.  Padded query tokens get
+// their final outputs here: zeros and lse = sink (FlintAttention.forward,
+// attention_mask: the sink remains valid for padded queries).
 #include "flint_common.cuh"
 #include "sm100.cuh"
 
