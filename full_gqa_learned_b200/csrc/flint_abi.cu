@@ -301,10 +301,13 @@ flint_status_t run_stages(int stages, const void* q, const void* k, const void* 
     pp.rope_theta = rope_theta;
     pp.eps = eps;
     // ws_layout is always evaluated with max(nseg, 1) segments
-    const bool prep_split = prep_parts(T, f16 || qprep) > 1;
-    const long long prep_warps = (long long)T * prep_parts(T, f16 || qprep);
-    int prep_blocks = (int)(1 + (prep_warps + 31) / 32 < 1 + 4LL * sms ? 1 + (prep_warps + 31) / 32 : 1 + 4LL * sms);
-    if (prep_blocks > 1 + 4 * sms) prep_blocks = 1 + 4 * sms;
+    // block 0 plans; the others take warps' worth of token work, at most
+    // four blocks per SM (they loop over the rest)
+    const int prep_n = prep_parts(T, f16 || qprep);
+    const bool prep_split = prep_n > 1;
+    long long prep_blocks_ll = 1 + ((long long)T * prep_n + 31) / 32;
+    if (prep_blocks_ll > 1 + 4LL * sms) prep_blocks_ll = 1 + 4LL * sms;
+    int prep_blocks = (int)prep_blocks_ll;
     if (prep_blocks < 2) prep_blocks = 2;
     if (stages & kStagePrepare) {
         if (prep_split)
