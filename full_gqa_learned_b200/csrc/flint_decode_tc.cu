@@ -6,15 +6,17 @@
 // column, HF discussion #26 on RecursiveSI/flint), reorganised so that the
 // step streams the cache at HBM speed:
 //
-// * A persistent CTA per SM takes work items (sequence b, KV head g, split)
-//   from a counter.  A split is a run of 128-slot tiles of the cache; tiles
+// * A persistent CTA per SM takes work items (sequence b, KV head g, split):
+//   its own index first, then the rest from a counter, each published to the
+//   CTA's warps with its position.  A split is a run of 128-slot tiles of the
+//   cache; tiles
 //   with no slot in the token's window are skipped.  Slot s holds position
 //   pos - ((pos - s) mod cap), which is in the window when (pos - s) mod cap
 //   < n = pos - lo + 1.
 // * Warp 0 streams the K and V tiles by TMA (three 64 KiB stages of K and V,
 //   128-byte swizzle, the same layout as the attention kernel's tiles) ahead
 //   of the MMAs, across items, and prefetches the next item's q, k, v rows
-//   into L2.
+//   into L2 (the first item's at kernel entry, before the first tiles).
 // * Warp 1 issues, per tile, S^T = K Q^T (M = 128 slots, N = 16: the 8
 //   query heads as BF16 high parts and as the BF16 rounding of the
 //   remainders, so hi + lo carries q~ to about 2^-17) and, once the slot
