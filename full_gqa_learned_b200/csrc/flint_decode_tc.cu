@@ -9,10 +9,9 @@
 // * A persistent CTA per SM takes work items (sequence b, KV head g, split):
 //   its own index first, then the rest from a counter, each published to the
 //   CTA's warps with its position.  A split is a run of 128-slot tiles of the
-//   cache; tiles
-//   with no slot in the token's window are skipped.  Slot s holds position
-//   pos - ((pos - s) mod cap), which is in the window when (pos - s) mod cap
-//   < n = pos - lo + 1.
+//   cache; tiles with no slot in the token's window are skipped.  Slot s
+//   holds position pos - ((pos - s) mod cap), which is in the window when
+//   (pos - s) mod cap < n = pos - lo + 1.
 // * Warp 0 streams the K and V tiles by TMA (three 64 KiB stages of K and V,
 //   128-byte swizzle, the same layout as the attention kernel's tiles) ahead
 //   of the MMAs, across items, and prefetches the next item's q, k, v rows
