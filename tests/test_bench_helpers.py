@@ -66,3 +66,18 @@ def test_backward_workloads_are_selectable():
     import workloads as W
     for name in W.CONFIGS:
         assert (bench.BWD_PREFIX + name)[len(bench.BWD_PREFIX):] == name
+
+
+def test_soak_loads_for_its_duration_and_skips_under_profile():
+    class A:
+        pass
+    a = A()
+    a.profile, a.soak = True, 5.0
+    calls = []
+    bench.soak(a, lambda: calls.append(1), lambda: None)
+    assert calls == []                      # profiler runs take no soak
+    a.profile, a.soak = False, 0.05
+    syncs = []
+    bench.soak(a, lambda: calls.append(1), lambda: syncs.append(1))
+    assert len(calls) >= 20 and len(calls) % 20 == 0   # whole groups of 20 steps
+    assert len(syncs) == len(calls) // 20
